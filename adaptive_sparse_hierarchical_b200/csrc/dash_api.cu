@@ -1,0 +1,246 @@
+// dash_api.cu -- the C ABI declared in include/dash.h: argument checks, workspace layout and
+// the launch sequence of each entry point.  No allocation, no synchronisation.
+#include <cmath>
+#include <cstdint>
+
+#include "dash_common.cuh"
+
+using namespace dash;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool pow2_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+int esize(int dtype) { return dtype == DASH_BF16 ? 2 : 4; }
+
+// Shape checks shared by every entry point.
+int check_params(const dash_params* p)
+{
+    if (!p) return DASH_EINVAL;
+    if (p->batch < 1 || p->seqlen < 1 || p->h_q < 1 || p->h_kv < 1 || p->h_q % p->h_kv) return DASH_EINVAL;
+    if (!(p->alpha > 1.f && p->alpha <= 2.f)) return DASH_EINVAL;
+    if (!(p->gamma >= 0.f) || !std::isfinite(p->gamma)) return DASH_EINVAL;
+    if (!(p->inv_sigma >= 0.f) || !std::isfinite(p->inv_sigma)) return DASH_EINVAL;
+    if (p->dtype != DASH_F32 && p->dtype != DASH_BF16) return DASH_EINVAL;
+    if (p->chunk < 1 || p->d_h < 1) return DASH_EINVAL;
+    if (p->d_h != 64 && p->d_h != 128) return DASH_EUNSUPPORTED;
+    if (p->chunk != 16 && p->chunk != 32 && p->chunk != 64 && p->chunk != 128) return DASH_EUNSUPPORTED;
+    if (!pow2_group(p->h_q / p->h_kv)) return DASH_EUNSUPPORTED;
+    return DASH_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
+bool strides_ok(const long long st[3], int dtype)
+{
+    for (int k = 0; k < 3; ++k)
+        if (st[k] < 0 || (st[k] * esize(dtype)) % 16) return false;
+    return true;
+}
+
+Shape make_shape(const dash_params* p)
+{
+    Shape s;
+    s.batch = p->batch; s.n = p->seqlen; s.hq = p->h_q; s.hkv = p->h_kv; s.g = p->h_q / p->h_kv;
+    s.d = p->d_h; s.B = p->chunk; s.T = p->seqlen / p->chunk;
+    s.alpha = p->alpha; s.gamma = p->gamma; s.inv_sigma = p->inv_sigma;
+    for (int k = 0; k < 3; ++k) {
+        s.qs[k] = p->q_strides[k]; s.ks[k] = p->k_strides[k];
+        s.vs[k] = p->v_strides[k]; s.os[k] = p->o_strides[k];
+    }
+    return s;
+}
+
+long long route_cap(const dash_params* p)
+{
+    // sum_{i < n} floor(i / B) = tri_offset(n, B)
+    return tri_offset(p->seqlen, p->chunk);
+}
+
+struct PrefillLayout { size_t kbar, counts, idx, bias, total; };
+PrefillLayout prefill_layout(const dash_params* p)
+{
+    PrefillLayout L;
+    const size_t bh = (size_t)p->batch * p->h_kv;
+    const size_t T = (size_t)(p->seqlen / p->chunk);
+    const size_t cap = (size_t)route_cap(p);
+    L.kbar = 0;
+    L.counts = L.kbar + up(bh * T * p->d_h * 4);
+    L.idx = L.counts + up(bh * (size_t)p->seqlen * 4);
+    L.bias = L.idx + up(bh * cap * 4);
+    L.total = L.bias + up(bh * cap * 4);
+    return L;
+}
+
+struct DecodeLayout { size_t x, part, counts, idx, bias, total; int splits; };
+DecodeLayout decode_layout(const dash_params* p)
+{
+    DecodeLayout L;
+    const Shape s = make_shape(p);
+    const size_t bh = (size_t)p->batch * p->h_kv;
+    const size_t T = (size_t)s.T;
+    L.splits = decode_splits(s, s.T);
+    L.x = 0;
+    L.part = L.x + up(bh * s.g * (T > 0 ? T : 1) * 4);
+    L.counts = L.part + up(bh * (size_t)L.splits * s.g * (p->d_h + 2) * 4);
+    L.idx = L.counts + up(bh * 4);
+    L.bias = L.idx + up(bh * (T > 0 ? T : 1) * 4);
+    L.total = L.bias + up(bh * (T > 0 ? T : 1) * 4);
+    return L;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? DASH_OK : DASH_ELAUNCH; }
+
+}  // namespace
+
+extern "C" {
+
+size_t dash_workspace_size(const dash_params* p, int op)
+{
+    if (check_params(p) != DASH_OK) return 0;
+    if (op == DASH_OP_PREFILL) return prefill_layout(p).total;
+    if (op == DASH_OP_DECODE) return decode_layout(p).total;
+    return 0;
+}
+
+long long dash_route_capacity(const dash_params* p)
+{
+    if (check_params(p) != DASH_OK) return 0;
+    return route_cap(p);
+}
+
+int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const void* K, const void* V,
+                       const float* qbar, void* O, float* kbar_out, const dash_route_out* route, void* workspace,
+                       size_t ws_bytes, void* stream);
+
+int dash_prefill(const dash_params* p, const void* Q, const void* K, const void* V, const float* qbar,
+                 void* O, float* kbar_out, const dash_route_out* route, void* workspace, size_t ws_bytes,
+                 void* stream)
+{
+    return dash_prefill_stage(p, -1, Q, K, V, qbar, O, kbar_out, route, workspace, ws_bytes, stream);
+}
+
+int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const void* K, const void* V,
+                       const float* qbar, void* O, float* kbar_out, const dash_route_out* route, void* workspace,
+                       size_t ws_bytes, void* stream)
+{
+    if (stage < -1 || stage > DASH_STAGE2) return DASH_EINVAL;
+    int rc = check_params(p);
+    if (rc != DASH_OK) return rc;
+    if (!Q || !K || !V || !qbar || !O) return DASH_EINVAL;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(qbar)) return DASH_EALIGN;
+    if (!strides_ok(p->q_strides, p->dtype) || !strides_ok(p->k_strides, p->dtype) ||
+        !strides_ok(p->v_strides, p->dtype) || !strides_ok(p->o_strides, p->dtype))
+        return DASH_EALIGN;
+    const Shape s = make_shape(p);
+    int P = 0;
+    route_prefill_smem(s, &P);
+    if (P == 0) return DASH_EUNSUPPORTED;
+    const PrefillLayout L = prefill_layout(p);
+    if (!workspace || ws_bytes < L.total) return DASH_EWORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DASH_EALIGN;
+    if (kbar_out && !aligned16(kbar_out)) return DASH_EALIGN;
+    char* ws = static_cast<char*>(workspace);
+    float* kbar = kbar_out ? kbar_out : reinterpret_cast<float*>(ws + L.kbar);
+    Routes rt;
+    rt.counts = route && route->counts ? route->counts : reinterpret_cast<int*>(ws + L.counts);
+    rt.idx = route && route->chunk_idx ? route->chunk_idx : reinterpret_cast<int*>(ws + L.idx);
+    rt.bias = route && route->bias ? route->bias : reinterpret_cast<float*>(ws + L.bias);
+    rt.bitmask = route ? route->bitmask : nullptr;
+    rt.cap = route_cap(p);
+    rt.words = (s.T + 31) / 32;
+    if (!aligned4(rt.counts) || !aligned4(rt.idx) || !aligned4(rt.bias) || (rt.bitmask && !aligned4(rt.bitmask)))
+        return DASH_EALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (stage == -1 || stage == DASH_STAGE0) {
+        rc = launch_status(launch_stage0(s, p->dtype, K, qbar, nullptr, kbar, s.T, nullptr, st));
+        if (rc != DASH_OK) return rc;
+    }
+    if (stage == -1 || stage == DASH_STAGE1) {
+        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, rt, st));
+        if (rc != DASH_OK) return rc;
+    }
+    if (stage == -1 || stage == DASH_STAGE2) rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt, st));
+    return rc;
+}
+
+int dash_summary_build(const dash_params* p, const void* K_cache, const float* qbar, const int* seqlens,
+                       float* kbar_cache, float* partial_state, void* stream)
+{
+    int rc = check_params(p);
+    if (rc != DASH_OK) return rc;
+    if (!K_cache || !qbar || !seqlens || !kbar_cache || !partial_state) return DASH_EINVAL;
+    if (!aligned16(K_cache) || !strides_ok(p->k_strides, p->dtype) || !aligned16(qbar)) return DASH_EALIGN;
+    if (!aligned4(seqlens) || !aligned4(kbar_cache) || !aligned4(partial_state)) return DASH_EALIGN;
+    const Shape s = make_shape(p);
+    return launch_status(launch_stage0(s, p->dtype, K_cache, qbar, seqlens, kbar_cache, s.T, partial_state,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int dash_summary_append(const dash_params* p, const void* k_new, const void* v_new, const float* qbar,
+                        void* K_cache, void* V_cache, float* kbar_cache, float* partial_state, int* seqlens,
+                        void* stream)
+{
+    int rc = check_params(p);
+    if (rc != DASH_OK) return rc;
+    if (!k_new || !v_new || !qbar || !K_cache || !V_cache || !kbar_cache || !partial_state || !seqlens)
+        return DASH_EINVAL;
+    if (p->h_kv > 32) return DASH_EUNSUPPORTED;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(qbar))
+        return DASH_EALIGN;
+    if (!strides_ok(p->k_strides, p->dtype) || !strides_ok(p->v_strides, p->dtype)) return DASH_EALIGN;
+    if (!aligned4(seqlens) || !aligned4(kbar_cache) || !aligned4(partial_state)) return DASH_EALIGN;
+    const Shape s = make_shape(p);
+    return launch_status(launch_append(s, p->dtype, k_new, v_new, qbar, K_cache, V_cache, kbar_cache, s.T,
+                                       partial_state, seqlens, static_cast<cudaStream_t>(stream)));
+}
+
+int dash_decode(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
+                const float* kbar_cache, const int* seqlens, void* O, const dash_route_out* route,
+                void* workspace, size_t ws_bytes, void* stream)
+{
+    int rc = check_params(p);
+    if (rc != DASH_OK) return rc;
+    if (!q || !K_cache || !V_cache || !kbar_cache || !seqlens || !O) return DASH_EINVAL;
+    if (!aligned16(q) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(O) || !aligned16(kbar_cache))
+        return DASH_EALIGN;
+    if (!strides_ok(p->k_strides, p->dtype) || !strides_ok(p->v_strides, p->dtype)) return DASH_EALIGN;
+    if (!aligned4(seqlens)) return DASH_EALIGN;
+    const DecodeLayout L = decode_layout(p);
+    if (!workspace || ws_bytes < L.total) return DASH_EWORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DASH_EALIGN;
+    const Shape s = make_shape(p);
+    char* ws = static_cast<char*>(workspace);
+    Routes rt;
+    rt.counts = route && route->counts ? route->counts : reinterpret_cast<int*>(ws + L.counts);
+    rt.idx = route && route->chunk_idx ? route->chunk_idx : reinterpret_cast<int*>(ws + L.idx);
+    rt.bias = route && route->bias ? route->bias : reinterpret_cast<float*>(ws + L.bias);
+    rt.bitmask = route ? route->bitmask : nullptr;
+    rt.cap = s.T;
+    rt.words = (s.T + 31) / 32;
+    DecodeWs dw;
+    dw.x = reinterpret_cast<float*>(ws + L.x);
+    dw.part = reinterpret_cast<float*>(ws + L.part);
+    dw.splits = L.splits;
+    return launch_status(launch_decode(s, p->dtype, q, K_cache, V_cache, kbar_cache, s.T, seqlens, O, rt, dw,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+const char* dash_status_string(int status)
+{
+    switch (status) {
+    case DASH_OK: return "ok";
+    case DASH_EINVAL: return "invalid argument";
+    case DASH_EUNSUPPORTED: return "unsupported configuration (d_h, chunk, group size or sequence too long)";
+    case DASH_EWORKSPACE: return "workspace missing or too small";
+    case DASH_EALIGN: return "pointer or stride misaligned";
+    case DASH_ELAUNCH: return "kernel launch failed";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// dash_common.cuh -- shared device helpers and internal launcher declarations of the
+// B200 DashAttention library.  Internal only: the public interface is include/dash.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dash.h"
+
+namespace dash {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Shape and hyper-parameters as the kernels see them.
+struct Shape {
+    int batch, n, hq, hkv, g, d, B, T;   // T = floor(n / B) complete chunks
+    float alpha, gamma, inv_sigma;
+    long long qs[3], ks[3], vs[3], os[3];
+};
+
+// Route storage: where Stage 1 writes and Stage 2 reads.
+struct Routes {
+    int* counts;        // [b, hkv, rows]
+    int* idx;           // [b, hkv, cap]
+    float* bias;        // [b, hkv, cap]
+    uint32_t* bitmask;  // [b, hkv, rows, words] or null
+    long long cap;      // entries per (b, r)
+    int words;          // ceil(T / 32)
+};
+
+// Start of position i's list inside one (b, r) route arena: positions with c = floor(i/B)
+// hold c entries each, so the lists before i take B * c*(c-1)/2 + (i - c*B) * c entries.
+__host__ __device__ inline long long tri_offset(int i, int B)
+{
+    long long c = i / B;
+    return (long long)B * (c * (c - 1) / 2) + (long long)(i - c * B) * c;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ int warp_isum(int v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// 16-byte vector of elements of type T converted to fp32.
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void load(const float* p, float* out)
+    {
+        float4 v = *reinterpret_cast<const float4*>(p);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    }
+};
+template <> struct Vec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out)
+    {
+        uint4 v = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            out[2 * k] = __uint_as_float(w[k] << 16);
+            out[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
+    }
+};
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---- launchers (each returns cudaGetLastError() of its launches) -------------------------
+// Stage 0: summaries of complete chunks of positions [0, len_b) and, if state != null, the
+// running state of the incomplete chunk.  len == null means every sequence has length s.n.
+cudaError_t launch_stage0(const Shape& s, int dtype, const void* K, const float* qbar,
+                          const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st);
+cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const void* v_new,
+                          const float* qbar, void* Kc, void* Vc, float* kbar, int kbar_T,
+                          float* state, int* seqlens, cudaStream_t st);
+// Stage 1 for prefill: routes of every position.
+cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
+                                 const Routes& rt, cudaStream_t st);
+size_t route_prefill_smem(const Shape& s, int* positions_per_block);
+// Stage 2 for prefill.
+cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,
+                                  const void* V, void* O, const Routes& rt, cudaStream_t st);
+// Decode: Stage 1 (logits, thresholds, GQA aggregation) and Stage 2 (split + merge).
+struct DecodeWs {
+    float* x;        // [b, hkv, g, T]  scaled logits, then head weights
+    float* part;     // [b, hkv, splits, g, d + 2]
+    int splits;      // partial slots per (b, r)
+};
+cudaError_t launch_route_decode(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
+                                const int* seqlens, const Routes& rt, float* X, cudaStream_t st);
+cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* Kc, const void* Vc,
+                          const float* kbar, int kbar_T, const int* seqlens, void* O,
+                          const Routes& rt, const DecodeWs& ws, cudaStream_t st);
+int decode_splits(const Shape& s, int kbar_T);
+
+}  // namespace dash

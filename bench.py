@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Benchmark of the DashAttention forward pass on B200.
+
+Default (N=1): the 1B-class prefill layer (b=1, n=32768, 16 query / 2 KV heads, d=128, chunk 64,
+alpha 1.5, gamma tuned for 25% routed chunks), one step = Stage 0 + Stage 1 + Stage 2 over the
+whole sequence, plus the decode workload (b=8, 131072-token caches, 32/2 heads, one append +
+decode per step) reported under "decode".  Under torchrun every rank runs its own replica
+(no data-path collective): scaling is weak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dash|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "prefill Mtok/s and decode µs/token at 32K–128K ctx; % of HBM / bf16 TC roofline"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def args_():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dash", choices=["dash", "reference"])
+    ap.add_argument("--workload", default="prefill_32k")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------- ranks
+class Ranks:
+    def __init__(self, want_gpu=True):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = None
+        if self.world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as dist
+            backend = "nccl" if (want_gpu and torch.cuda.is_available()) else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+            self.dist = dist
+            self.backend = backend
+
+    def barrier(self):
+        if self.dist:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        """Max over ranks (timing only; not a data-path collective)."""
+        if not self.dist:
+            return x
+        import torch
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist:
+            self.dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------- clocks
+class Clocks:
+    """Samples nvidia-smi clocks / throttle reasons while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------- prefill
+def stage2_routed_flops(counts, n, B, g, d, hq):
+    """4 d sum_{b,h,i} (|S_i^r| B + |D_i|): routed chunks' tokens plus the diagonal tokens."""
+    diag = sum((i % B) + 1 for i in range(n))
+    return 4.0 * d * (float(counts.sum()) * B * g + counts.shape[0] * hq * diag)
+
+
+def run_prefill(wl, steps, warmup, ranks, pk, pk_kind):
+    import torch
+    import adaptive_sparse_hierarchical_b200 as D
+
+    dev = torch.device("cuda", ranks.local)
+    x = wl.make()
+    tq = {k: torch.from_numpy(x[k]).to(dev, torch.bfloat16) for k in ("Q", "K", "V")}
+    qbar = torch.from_numpy(x["qbar"]).to(dev)
+    pf = D.Prefill(tq["Q"], tq["K"], tq["V"], qbar, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
+                   inv_sigma=wl.inv_sigma, want_route=True)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(rec=None):
+        if rec:
+            rec[0].record(stream)
+        pf.stage(0)
+        if rec:
+            rec[1].record(stream)
+        pf.stage(1)
+        if rec:
+            rec[2].record(stream)
+        pf.stage(2)
+        if rec:
+            rec[3].record(stream)
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    counts = pf.counts.cpu().numpy()
+    flops = stage2_routed_flops(counts, wl.n, wl.chunk, wl.h_q // wl.h_kv, wl.d, wl.h_q)
+    recs = [[ev() for _ in range(4)] for _ in range(steps)]
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    with Clocks(ranks.local) as clk:
+        for k in range(steps):
+            flush.fill_(k & 0xff)                 # evict K/V/Q from L2 between steps (not timed)
+            step(recs[k])
+        torch.cuda.synchronize(dev)
+    ranks.barrier()
+    st = [[recs[k][j].elapsed_time(recs[k][j + 1]) for j in range(3)] for k in range(steps)]
+    per_step = [sum(s) for s in st]
+    ms = ranks.max(statistics.mean(per_step))
+    stage_ms = [statistics.mean(s[j] for s in st) for j in range(3)]
+    t2 = stage_ms[2] / 1e3
+    achieved = flops / t2 / 1e12
+    peak = pk["bf16_tflops"]
+    tokens = wl.batch * wl.n
+    out = {
+        "ms_per_step": ms, "value": ranks.world * tokens / (ms / 1e3) / 1e6,
+        "stages_ms": {"stage0_summary": stage_ms[0], "stage1_route": stage_ms[1], "stage2_attend": stage_ms[2]},
+        "routed_fraction": float(counts.sum()) / (wl.batch * wl.h_kv * sum(i // wl.chunk for i in range(wl.n))),
+        "roofline": {"kernel": "stage2 attend_prefill_mma_kernel", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_kind": f"bf16 dense burst, of {pk_kind}",
+                     "flops_per_launch": flops, "launch_ms": stage_ms[2]},
+        "clocks": clk.summary(),
+        "gpu_launches": 3 * steps,
+    }
+    # e2e: host (pinned) inputs copied in, result copied out, every step
+    hq = {k: tq[k].cpu().pin_memory() for k in ("Q", "K", "V")}
+    ho = torch.empty(tq["Q"].shape, dtype=torch.bfloat16).pin_memory()
+    e_s, e_e = ev(), ev()
+
+    def e2e_step():
+        for k in ("Q", "K", "V"):
+            tq[k].copy_(hq[k], non_blocking=True)
+        pf()
+        ho.copy_(pf.O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    e_s.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e_e.record(stream)
+    torch.cuda.synchronize(dev)
+    ems = ranks.max(e_s.elapsed_time(e_e) / steps)
+    nbytes = lambda t: t.numel() * t.element_size()
+    out["e2e"] = {"value": ranks.world * tokens / (ems / 1e3) / 1e6, "unit": "Mtok/s", "ms_per_step": ems,
+                  "h2d_bytes_per_step": sum(nbytes(hq[k]) for k in hq), "d2h_bytes_per_step": nbytes(ho)}
+    out["_inputs"] = x
+    return out
+
+
+# ---------------------------------------------------------------------------------------- decode
+def run_decode(steps, warmup, ranks, pk, pk_kind):
+    import torch
+    import adaptive_sparse_hierarchical_b200 as D
+    from adaptive_sparse_hierarchical_b200 import workloads as W
+
+    wl = W.get("decode_128k")
+    dev = torch.device("cuda", ranks.local)
+    x = wl.make()
+    prefix = wl.extra["prefix"]
+    nst = min(steps, wl.extra["steps"])
+    st = D.DecodeState(wl.batch, wl.n, wl.h_q, wl.h_kv, wl.d, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
+                       device=dev, qbar=torch.from_numpy(x["qbar"]).to(dev))
+    counts = torch.zeros((wl.batch, wl.h_kv), dtype=torch.int32, device=dev)
+    idx = torch.zeros((wl.batch, wl.h_kv, st.T), dtype=torch.int32, device=dev)
+    bias = torch.zeros((wl.batch, wl.h_kv, st.T), dtype=torch.float32, device=dev)
+    st.route = D.route_out(counts, idx, bias)
+    K0 = torch.from_numpy(x["K"][:, :prefix]).to(dev, torch.bfloat16)
+    V0 = torch.from_numpy(x["V"][:, :prefix]).to(dev, torch.bfloat16)
+    kn = torch.from_numpy(np.ascontiguousarray(x["K"][:, prefix:prefix + wl.extra["steps"]].swapaxes(0, 1))).to(dev, torch.bfloat16)
+    vn = torch.from_numpy(np.ascontiguousarray(x["V"][:, prefix:prefix + wl.extra["steps"]].swapaxes(0, 1))).to(dev, torch.bfloat16)
+    qn = torch.from_numpy(np.ascontiguousarray(x["Q"].swapaxes(0, 1))).to(dev, torch.bfloat16)
+    del x
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    snapshot = (st.K.clone(), st.V.clone())
+
+    def reset():
+        st.K.copy_(snapshot[0]); st.V.copy_(snapshot[1])
+        st.seqlens.fill_(prefix)
+        D.dash_summary_build(st.p, st.K, st.qbar, st.seqlens, st.kbar, st.state)
+
+    st.K[:, :prefix].copy_(K0); st.V[:, :prefix].copy_(V0)
+    snapshot = (st.K.clone(), st.V.clone())
+    del K0, V0
+    reset()
+    for s in range(max(warmup, 3)):
+        st.step(qn[s], kn[s], vn[s])
+    reset()
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    evs = [(ev(), ev(), ev()) for _ in range(nst)]
+    routed = []
+    with Clocks(ranks.local) as clk:
+        for s in range(nst):
+            evs[s][0].record(stream)
+            st.append(kn[s], vn[s])
+            evs[s][1].record(stream)
+            st.decode(qn[s])
+            evs[s][2].record(stream)
+            if s % 50 == 0:
+                routed.append((s, counts.clone()))
+        torch.cuda.synchronize(dev)
+    ranks.barrier()
+    step_ms = [a.elapsed_time(c) for a, b, c in evs]
+    dec_ms = [b.elapsed_time(c) for a, b, c in evs]
+    ms = ranks.max(statistics.mean(step_ms))
+    # routed K+V bytes per step (numerator of the HBM roofline), from sampled steps' counts
+    byts = []
+    for s, c in routed:
+        L = prefix + s + 1
+        diag = (L - 1) % wl.chunk + 1
+        byts.append(2 * wl.d * 2 * (float(c.sum()) * wl.chunk + wl.batch * wl.h_kv * diag))
+    bps = statistics.mean(byts)
+    achieved = bps / (statistics.mean(dec_ms) / 1e3) / 1e9
+    res = {"workload": "decode_128k: b=8, 131072-token caches (+1 per step), 32/2 heads, d=128, B=64, alpha 1.5, "
+                       f"gamma {wl.gamma} (~25% routed)",
+           "us_per_step": ms * 1e3, "us_per_token": ms * 1e3 / (wl.batch * ranks.world) * ranks.world / ranks.world,
+           "steps": nst, "append_us": statistics.mean(a.elapsed_time(b) for a, b, c in evs) * 1e3,
+           "decode_us": statistics.mean(dec_ms) * 1e3,
+           "routed_fraction": float(routed[-1][1].sum()) / (wl.batch * wl.h_kv * ((prefix + routed[-1][0]) // wl.chunk)),
+           "roofline": {"kernel": "decode (route + split attend + merge)", "bound": "hbm", "achieved": achieved,
+                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                        "peak_kind": f"hbm copy, of {pk_kind}", "bytes_per_step": bps},
+           "clocks": clk.summary(), "gpu_launches": 6 * nst,
+           "l2": "KV caches (1.07 GB) larger than L2"}
+    res["us_per_token"] = res["us_per_step"] / wl.batch
+    return res
+
+
+# ---------------------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, x, nrows):
+    """Time the float64 oracle on a bounded sample of the workload: Stage 0 over the whole
+    sequence (its share per token is charged) plus Stages 1-2 for `nrows` evenly spaced query
+    positions with all heads.  Returns (tokens per second, seconds, threads)."""
+    import oracle
+
+    pos = np.linspace(0, wl.n - 1, nrows).astype(np.int32)
+    t0 = time.perf_counter()
+    kbar = oracle.stage0(x["K"], x["qbar"], wl.chunk)
+    t1 = time.perf_counter()
+    oracle.rows(x["Q"][:, pos], np.broadcast_to(pos, (wl.batch, nrows)), x["K"], x["V"], kbar, chunk=wl.chunk,
+                alpha=wl.alpha, gamma=wl.gamma, inv_sigma=wl.inv_sigma)
+    t2 = time.perf_counter()
+    secs = (t1 - t0) * nrows / wl.n + (t2 - t1)
+    return wl.batch * nrows / secs, t2 - t0, oracle.num_threads()
+
+
+def reference_arm(args, ranks):
+    """The CPU oracle as the reference arm: each step is a bounded sample of the workload."""
+    from adaptive_sparse_hierarchical_b200 import workloads as W
+
+    wl = W.get(args.workload)
+    x = wl.make()
+    nrows = 256
+    for _ in range(args.warmup):
+        oracle_sample(wl, x, 8)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, s, thr = oracle_sample(wl, x, nrows)
+        vals.append(v)
+        secs.append(s)
+    tps = statistics.mean(vals)
+    value = tps / 1e6
+    sample = (f"{nrows} evenly spaced query positions (all {wl.h_q} heads) per step + Stage 0 share, "
+              f"of {wl.name}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(secs) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, args),
+            "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": thr, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, args):
+    return {"workload": f"{wl.name}: b={wl.batch}, n={wl.n}, h_q={wl.h_q}, h_kv={wl.h_kv}, d={wl.d}, "
+                        f"chunk={wl.chunk}, alpha={wl.alpha}, gamma={wl.gamma}, sigma=1",
+            "batch": wl.batch, "seq_len": wl.n, "h_q": wl.h_q, "h_kv": wl.h_kv, "d_h": wl.d, "chunk": wl.chunk,
+            "alpha": wl.alpha, "gamma": wl.gamma, "parallelism": f"replicas x{args.gpus}",
+            "l2": "flushed between steps (256 MB write, outside the per-step events)"}
+
+
+def main():
+    args = args_()
+    if args.impl == "reference":
+        ranks = Ranks(want_gpu=False) if int(os.environ.get("WORLD_SIZE", "1")) > 1 else Ranks(want_gpu=False)
+        if ranks.rank == 0:
+            reference_arm(args, ranks)
+        ranks.close()
+        return
+    import torch
+    from adaptive_sparse_hierarchical_b200 import workloads as W
+    from adaptive_sparse_hierarchical_b200.build import build
+
+    build()
+    ranks = Ranks()
+    torch.cuda.set_device(ranks.local)
+    pk, pk_kind = peaks()
+    wl = W.get(args.workload)
+    pre = run_prefill(wl, args.steps, args.warmup, ranks, pk, pk_kind)
+    x = pre.pop("_inputs")
+    line = {"metric": METRIC, "value": pre["value"], "unit": "Mtok/s", "n_gpus": ranks.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, planted chunks; see DESIGN.md)",
+            "config": config_of(wl, args), "roofline": pre["roofline"], "e2e": pre["e2e"],
+            "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "stages_ms": pre["stages_ms"],
+            "routed_fraction": pre["routed_fraction"]}
+    if not args.no_decode:
+        line["decode"] = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind)
+        line["gpu_launches"] += line["decode"]["gpu_launches"]
+    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
+        v, secs, thr = oracle_sample(wl, x, args.cpu_rows)
+        line["cpu_baseline"] = {"value": v / 1e6, "unit": "Mtok/s", "cores": thr, "kind": "oracle",
+                                "sample": f"{args.cpu_rows} evenly spaced query positions x {wl.h_q} heads + "
+                                          f"Stage 0 share ({secs:.1f} s)"}
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.close()
+
+
+if __name__ == "__main__":
+    main()

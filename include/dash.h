@@ -1,0 +1,141 @@
+/*
+ * dash.h -- C ABI of the B200 DashAttention forward-pass library (libdash_b200.so).
+ *
+ * DashAttention ("DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention",
+ * xllm-io paper review page, section 3 "core formulas"; gist.science technical summary,
+ * "Methodology") is three-stage sparse attention:
+ *   Stage 0 (Eq. 4)   chunk summaries  kbar_c^(r) = sum_{t in chunk c} softmax_t(<qbar^(r),k_t>/sqrt(d)) k_t
+ *   Stage 1 (Eq. 6)   routing          what_i^(h) = alpha-entmax(gamma * <q_i^(h), kbar_c^(r)>/sqrt(d))
+ *                     GQA average      w_i^(r) = mean_{h in group r} what_i^(h); routed set R = support
+ *   Stage 2 (Prop. 4.1) biased softmax o_i = softmax_j(<q_i,k_j>/sqrt(d) + d_ij) V over the routed
+ *                     chunks' tokens and the diagonal tokens c(i)B..i, with
+ *                     d_ij = (log w_{i,c(j)} - mean_{c in R} log w_{i,c}) / sigma on routed tokens, 0 on
+ *                     the diagonal (equivalent to Eq. 9 with the Eq. 11-12 prior).
+ * A query at position i routes over the complete chunks c < floor(i/B); its own chunk is always
+ * the diagonal branch.  Head h uses KV head floor(h / (h_q/h_kv)).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless stated; the caller allocates and owns every
+ *     buffer, including the workspace.  The library never allocates, frees or synchronises.
+ *   - Every call only enqueues kernels on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream) and returns; results are ready when the stream reaches them.
+ *   - Layouts: Q, O [batch, n, h_q, d_h], K, V [batch, n, h_kv, d_h] addressed through element
+ *     strides {batch, position, head}; the d_h elements of one head are contiguous.  Element type
+ *     is `dtype` (fp32 or bf16).  qbar, kbar and every routing/bias value are fp32.
+ *   - Alignment: Q, K, V, O base pointers and strides*sizeof(element) must be multiples of 16
+ *     bytes; other pointers 4 bytes.
+ *   - Return value: DASH_OK (0) or a negative DASH_E* status.  Arguments are checked before any
+ *     launch; on an error nothing is enqueued.  DASH_ELAUNCH reports a failed kernel launch.
+ */
+#ifndef DASH_H
+#define DASH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    DASH_OK = 0,
+    DASH_EINVAL = -1,       /* bad shape / hyper-parameter / null required pointer */
+    DASH_EUNSUPPORTED = -2, /* valid but not built: d_h, chunk, group size or dtype */
+    DASH_EWORKSPACE = -3,   /* workspace smaller than dash_workspace_size() */
+    DASH_EALIGN = -4,       /* pointer or stride alignment */
+    DASH_ELAUNCH = -5       /* a kernel launch failed (cudaGetLastError) */
+};
+
+enum { DASH_F32 = 0, DASH_BF16 = 1 };
+enum { DASH_OP_PREFILL = 0, DASH_OP_DECODE = 1 };
+
+typedef struct {
+    int batch;
+    int seqlen;     /* prefill: sequence length n; decode/append: K/V cache capacity (positions) */
+    int h_q, h_kv;  /* h_q % h_kv == 0; group size g_q = h_q / h_kv in {1, 2, 4, 8, 16} */
+    int d_h;        /* head dimension: 64 or 128 */
+    int chunk;      /* B: 16, 32, 64 or 128 */
+    float alpha;    /* entmax alpha in (1, 2] (section 3 background formula) */
+    float gamma;    /* routing scale gamma >= 0 (Eq. 6); 0 routes every visible chunk uniformly */
+    float inv_sigma;/* 1/sigma of Eq. 11 / Prop. 4.1; 1 = plain prior, 0 = sigma -> infinity */
+    int dtype;      /* DASH_F32 or DASH_BF16 for Q, K, V, O */
+    long long q_strides[3], k_strides[3], v_strides[3], o_strides[3]; /* elements: b, pos, head */
+} dash_params;
+
+/* Routing lists written by Stage 1 and read by Stage 2 (section 3, Stage 1 kernel: the routed
+ * support after the GQA average).  Any pointer may be NULL; the lists then live in the workspace.
+ *   counts    int32 [batch, h_kv, n]                |R_i| for KV head r at position i
+ *   chunk_idx int32 [batch, h_kv, dash_route_capacity(p)]  routed chunk ids, ascending; row i's
+ *             list starts at tri(i) = B*c*(c-1)/2 + (i - c*B)*c with c = floor(i/B)
+ *   bias      fp32, same layout as chunk_idx: d_ij of Prop. 4.1 for the listed chunk
+ *   bitmask   uint32 [batch, h_kv, n, ceil(T_c/32)] bit c set iff chunk c is routed (the pages'
+ *             bit-packed block mask, 32 columns per word); written only when non-NULL. */
+typedef struct {
+    int* counts;
+    int* chunk_idx;
+    float* bias;
+    uint32_t* bitmask;
+} dash_route_out;
+
+/* Bytes of device workspace `op` (DASH_OP_PREFILL or DASH_OP_DECODE) needs for these params;
+ * 0 on invalid params.  The workspace must be 256-byte aligned. */
+size_t dash_workspace_size(const dash_params* p, int op);
+
+/* Routing-list entries per (batch, KV head) for prefill: sum over positions of floor(i/B). */
+long long dash_route_capacity(const dash_params* p);
+
+/* Causal prefill forward (Stages 0, 1, 2) of Q, K, V [batch, n, *, d_h] into O.
+ *   qbar      fp32 [h_kv, d_h]  learned summary query of Eq. 4 (read only)
+ *   kbar_out  fp32 [batch, h_kv, floor(n/B), d_h] Stage-0 summaries, or NULL (then in workspace)
+ *   route     optional routing outputs (see dash_route_out), or NULL */
+int dash_prefill(const dash_params* p, const void* Q, const void* K, const void* V,
+                 const float* qbar, void* O, float* kbar_out, const dash_route_out* route,
+                 void* workspace, size_t ws_bytes, void* stream);
+
+/* One stage of dash_prefill on its own (same arguments): stage 0 writes the summaries, stage 1
+ * reads them and writes the routing lists, stage 2 reads both and writes O.  Running the three
+ * stages in order on one stream with the same buffers equals dash_prefill; the intermediate
+ * results must stay in kbar_out / route / workspace between the calls. */
+enum { DASH_STAGE0 = 0, DASH_STAGE1 = 1, DASH_STAGE2 = 2 };
+int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const void* K, const void* V,
+                       const float* qbar, void* O, float* kbar_out, const dash_route_out* route,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Build the summary cache of already-filled K caches (Eq. 4): for each sequence b with length
+ * L_b = seqlens[b] (device int32), writes kbar_cache[b, r, c] for every complete chunk
+ * c < floor(L_b/B) and the running state of the incomplete chunk into partial_state.
+ *   kbar_cache     fp32 [batch, h_kv, floor(seqlen/B), d_h]
+ *   partial_state  fp32 [batch, h_kv, d_h + 2]: acc[d_h], running max m, running sum l of the
+ *                  online softmax over the incomplete chunk's keys, in base 2: m is the largest
+ *                  <qbar,k> log2(e)/sqrt(d_h) so far, l = sum 2^(a - m), acc = sum 2^(a - m) k
+ *                  (m = -inf, l = 0, acc = 0 when the chunk is empty); acc / l is the running
+ *                  summary */
+int dash_summary_build(const dash_params* p, const void* K_cache, const float* qbar,
+                       const int* seqlens, float* kbar_cache, float* partial_state, void* stream);
+
+/* Incremental decoding, step 1 of 2: append one token per sequence.  k_new, v_new
+ * [batch, h_kv, d_h] (contiguous, dtype) are written at position L_b = seqlens[b] of the caches
+ * (k/v strides from p), the incomplete-chunk state is updated with the new key (online softmax of
+ * Eq. 4), the chunk's summary is written to kbar_cache when the key completes it (the summary is
+ * fixed from then on), and seqlens[b] becomes L_b + 1.  Requires L_b < seqlen. */
+int dash_summary_append(const dash_params* p, const void* k_new, const void* v_new,
+                        const float* qbar, void* K_cache, void* V_cache, float* kbar_cache,
+                        float* partial_state, int* seqlens, void* stream);
+
+/* Incremental decoding, step 2 of 2: the query q [batch, h_q, d_h] (contiguous, dtype) of each
+ * sequence sits at position L_b - 1 (L_b = seqlens[b] after the append) and attends over cache
+ * positions 0..L_b-1: Stage 1 over the cached summaries of chunks c < floor((L_b-1)/B), then
+ * Stage 2 split along the routed chunks, then a log-sum-exp merge.  O [batch, h_q, d_h]
+ * (contiguous, dtype).  route: optional, counts [batch, h_kv], chunk_idx / bias
+ * [batch, h_kv, floor(seqlen/B)]. */
+int dash_decode(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
+                const float* kbar_cache, const int* seqlens, void* O, const dash_route_out* route,
+                void* workspace, size_t ws_bytes, void* stream);
+
+/* Static text for a status code. */
+const char* dash_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DASH_H */

@@ -128,6 +128,26 @@ def chunk_summary(K, qbar, b: int, r: int, t0: int, t1: int) -> np.ndarray:
     return out
 
 
+def route_counts(Qrows, pos, K, kbar, *, chunk, alpha, gamma, nthreads: int = 0):
+    """Stage 1 only: |R| per (b, h_kv, row) for the given query rows (no Stage 2)."""
+    Qrows = _f32(Qrows)
+    b, nrows, hq, d = Qrows.shape
+    hkv = kbar.shape[1]
+    kbar = np.ascontiguousarray(kbar, dtype=np.float64)
+    T = kbar.shape[2]
+    pos = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, dtype=np.int32), (b, nrows)))
+    counts = np.zeros((b, hkv, nrows), dtype=np.int32)
+    cf = _cfg(b, K.shape[1], hq, hkv, d, chunk, alpha, gamma, 1.0)
+    dummy = np.zeros((1, 1, hkv, d), np.float32)
+    st = _strides(dummy)
+    nd = ctypes.POINTER(ctypes.c_double)()
+    _load().orc_rows(ctypes.byref(cf), _p(Qrows, ctypes.c_float), _p(pos, ctypes.c_int), nrows,
+                     _p(dummy, ctypes.c_float), _p(st, ctypes.c_longlong), _p(dummy, ctypes.c_float),
+                     _p(st, ctypes.c_longlong), _p(kbar, ctypes.c_double), T, 0, nd,
+                     _p(counts, ctypes.c_int), nd, nd, nd, int(nthreads))
+    return counts
+
+
 def rows(Qrows, pos, K, V, kbar, *, chunk, alpha, gamma, inv_sigma=1.0, prior_form=False,
          want_route=False, nthreads: int = 0):
     """Full forward for selected query rows.

@@ -326,6 +326,7 @@ static void attend_prior_form(const orc_cfg* cf, const float* q, const float* K,
 /* Outputs: O [batch][nrows][h_q][d]; optional counts [batch][h_kv][nrows] = |R|, and optional  */
 /* w, bias, margin [batch][h_kv][nrows][kbar_T] (entries past floor(pos/B) are left at 0).     */
 /* prior_form = 1 computes Stage 2 from Eq. 9 / 11-12 instead of Proposition 4.1.              */
+/* O = NULL skips Stage 2 (routing statistics only).                                          */
 /* ------------------------------------------------------------------------------------------ */
 
 void orc_rows(const orc_cfg* cf, const float* Qrows, const int* pos, int nrows,
@@ -352,7 +353,7 @@ void orc_rows(const orc_cfg* cf, const float* Qrows, const int* pos, int nrows,
         const float* q = Qrows + (((long long)b * nrows + t) * cf->h_q + (long long)r * g) * d;
         const double* kb = kbar + ((long long)b * hkv + r) * (long long)kbar_T * d;
         int nR = orc_route_row(cf, q, d, kb, nvis, w, bias, margin);
-        for (int hh = 0; hh < g; ++hh) {
+        for (int hh = 0; hh < g && O; ++hh) {
             double* o = O + (((long long)b * nrows + t) * cf->h_q + (long long)r * g + hh) * d;
             if (prior_form)
                 attend_prior_form(cf, q + (long long)hh * d, K, ks, V, vs, b, r, i, nvis, w, o);

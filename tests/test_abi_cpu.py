@@ -1,0 +1,86 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point include/dash.h declares,
+and rejects bad arguments before launching anything (no GPU needed for these paths)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import adaptive_sparse_hierarchical_b200 as D
+from adaptive_sparse_hierarchical_b200 import _lib as L
+from adaptive_sparse_hierarchical_b200.build import LIB, build
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build()
+
+
+def _p(**kw):
+    base = dict(batch=1, seqlen=1024, h_q=8, h_kv=2, d_h=128, chunk=64, alpha=1.5, gamma=8.0, dtype=L.DASH_BF16,
+                q_strides=(1024 * 8 * 128, 8 * 128, 128), k_strides=(1024 * 2 * 128, 256, 128),
+                v_strides=(1024 * 2 * 128, 256, 128), o_strides=(1024 * 8 * 128, 8 * 128, 128))
+    base.update(kw)
+    return L.params(**base)
+
+
+def test_header_symbols_exported():
+    syms = L.header_symbols()
+    assert set(syms) == {"dash_workspace_size", "dash_route_capacity", "dash_prefill", "dash_prefill_stage",
+                         "dash_summary_build",
+                         "dash_summary_append", "dash_decode", "dash_status_string"}
+    lib = D.load()
+    for s in syms:
+        assert hasattr(lib, s), s
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(syms) <= exported
+
+
+def test_route_capacity_is_triangular_sum():
+    for n, B in [(1, 64), (63, 64), (64, 64), (65, 64), (1000, 32), (32768, 64), (5, 16)]:
+        p = _p(seqlen=n, chunk=B)
+        assert L.dash_route_capacity(p) == sum(i // B for i in range(n))
+
+
+def test_workspace_sizes_cover_layout():
+    p = _p()
+    T, cap = 1024 // 64, L.dash_route_capacity(_p())
+    need = 2 * T * 128 * 4 + 2 * 1024 * 4 + 2 * 2 * cap * 4
+    assert L.dash_workspace_size(p, L.DASH_OP_PREFILL) >= need
+    assert L.dash_workspace_size(p, L.DASH_OP_DECODE) > 0
+    assert L.dash_workspace_size(p, 7) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(h_q=6, h_kv=4), L.DASH_EINVAL),
+    (dict(alpha=1.0), L.DASH_EINVAL),
+    (dict(alpha=2.5), L.DASH_EINVAL),
+    (dict(gamma=-1.0), L.DASH_EINVAL),
+    (dict(inv_sigma=-0.5), L.DASH_EINVAL),
+    (dict(batch=0), L.DASH_EINVAL),
+    (dict(dtype=7), L.DASH_EINVAL),
+    (dict(d_h=96), L.DASH_EUNSUPPORTED),
+    (dict(chunk=48), L.DASH_EUNSUPPORTED),
+    (dict(h_q=6, h_kv=2), L.DASH_EUNSUPPORTED),
+    (dict(h_q=64, h_kv=2), L.DASH_EUNSUPPORTED),
+])
+def test_bad_params_rejected_before_launch(kw, code):
+    assert L.dash_prefill(_p(**kw), 256, 256, 256, 256, 256, workspace=256, ws_bytes=1 << 40, check=False) == code
+    assert L.dash_workspace_size(_p(**kw), L.DASH_OP_PREFILL) == 0
+
+
+def test_missing_pointers_workspace_and_alignment():
+    p = _p()
+    ws = L.dash_workspace_size(p, L.DASH_OP_PREFILL)
+    assert L.dash_prefill(p, 0, 256, 256, 256, 256, workspace=256, ws_bytes=ws, check=False) == L.DASH_EINVAL
+    assert L.dash_prefill(p, 256, 256, 256, 256, 256, check=False) == L.DASH_EWORKSPACE
+    assert L.dash_prefill(p, 256, 256, 256, 256, 256, workspace=256, ws_bytes=ws - 1, check=False) == L.DASH_EWORKSPACE
+    assert L.dash_prefill(p, 264, 256, 256, 256, 256, workspace=256, ws_bytes=ws, check=False) == L.DASH_EALIGN
+    assert L.dash_prefill(p, 256, 256, 256, 256, 256, workspace=384, ws_bytes=ws, check=False) == L.DASH_EALIGN
+    bad = _p(k_strides=(1024 * 2 * 128, 250, 128))
+    assert L.dash_prefill(bad, 256, 256, 256, 256, 256, workspace=256, ws_bytes=ws, check=False) == L.DASH_EALIGN
+
+
+def test_status_strings():
+    for rc in (0, -1, -2, -3, -4, -5, -99):
+        assert isinstance(L.dash_status_string(rc), str) and L.dash_status_string(rc)

@@ -1,0 +1,128 @@
+"""GPU parity of incremental decoding (dash_summary_build / dash_summary_append / dash_decode
+through the C ABI) against the float64 oracle: summary cache, incomplete-chunk state, routes and
+outputs, step after step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import adaptive_sparse_hierarchical_b200 as D
+from adaptive_sparse_hierarchical_b200 import inputs, workloads as W
+
+from parity import check_outputs, check_routes
+
+pytestmark = pytest.mark.gpu
+
+
+def _tdt(dtype):
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def _state(x, lengths, capacity, *, chunk, alpha, gamma, dtype, inv_sigma=1.0):
+    b, _, hkv, d = x["K"].shape
+    hq = x["Q"].shape[2]
+    st = D.DecodeState(b, capacity, hq, hkv, d, chunk=chunk, alpha=alpha, gamma=gamma, inv_sigma=inv_sigma,
+                       dtype=_tdt(dtype), qbar=torch.from_numpy(x["qbar"]).cuda())
+    L0 = int(max(lengths))
+    st.fill(torch.from_numpy(x["K"][:, :L0]).to("cuda", _tdt(dtype)),
+            torch.from_numpy(x["V"][:, :L0]).to("cuda", _tdt(dtype)), lengths)
+    counts = torch.zeros((b, hkv), dtype=torch.int32, device="cuda")
+    idx = torch.zeros((b, hkv, max(capacity // chunk, 1)), dtype=torch.int32, device="cuda")
+    bias = torch.zeros((b, hkv, max(capacity // chunk, 1)), dtype=torch.float32, device="cuda")
+    st.route = D.route_out(counts, idx, bias)
+    st.rt = (counts, idx, bias)
+    return st
+
+
+def _check_summaries(st, x, chunk):
+    K = x["K"]
+    lens = st.seqlens.cpu().numpy()
+    kb = st.kbar.cpu().numpy()
+    state = st.state.cpu().numpy()
+    b, _, hkv, d = K.shape
+    for bb in range(b):
+        L = int(lens[bb])
+        ref = oracle.stage0(K[bb:bb + 1, :L], x["qbar"], chunk)[0]
+        np.testing.assert_allclose(kb[bb, :, :L // chunk], ref, atol=2e-5, rtol=1e-5)
+        if L % chunk:
+            for r in range(hkv):
+                part = oracle.chunk_summary(K, x["qbar"], bb, r, (L // chunk) * chunk, L)
+                np.testing.assert_allclose(state[bb, r, :d] / state[bb, r, d + 1], part, atol=2e-5, rtol=1e-5)
+
+
+def _check_step(st, x, q, lengths, *, chunk, alpha, gamma, dtype, inv_sigma=1.0):
+    b, _, hkv, d = x["K"].shape
+    hq = x["Q"].shape[2]
+    O = st.O.float().cpu().numpy()
+    oref, rt = oracle.decode(q, x["K"], x["V"], x["qbar"], lengths, chunk=chunk, alpha=alpha, gamma=gamma,
+                             inv_sigma=inv_sigma, want_route=True)
+    counts, idx, _ = (t.cpu().numpy() for t in st.rt)
+    T = x["K"].shape[1] // chunk
+    gs = {(bb, r, 0): idx[bb, r, :counts[bb, r]] for bb in range(b) for r in range(hkv)}
+    pos = (np.asarray(lengths) - 1).reshape(b, 1)
+    # oracle route arrays are [b, hkv, 1, T']; pad T' to the cache's chunk count
+    mism, _ = check_routes(gs, rt, chunk, pos, T)
+    return check_outputs(O[:, None], oref[:, None], dtype, hq // hkv, mism, rt, chunk, pos, T)
+
+
+@pytest.mark.parametrize("dtype,d,B,g", [("bf16", 128, 64, 4), ("bf16", 64, 32, 16), ("f32", 128, 64, 8),
+                                         ("bf16", 128, 128, 8), ("bf16", 128, 16, 2)])
+def test_decode_steps_small(dtype, d, B, g):
+    hkv, cap, b = 2, 1024, 3
+    x = inputs.planted(21, b, cap, g * hkv, hkv, d, B, dtype=dtype, chunk_frac=0.1)
+    lengths = np.array([300, 511, B])
+    st = _state(x, lengths, cap, chunk=B, alpha=1.5, gamma=6.0, dtype=dtype)
+    _check_summaries(st, x, B)
+    for step in range(70):
+        L = lengths.copy()
+        k = torch.from_numpy(x["K"][np.arange(b), L]).to("cuda", _tdt(dtype)).contiguous()
+        v = torch.from_numpy(x["V"][np.arange(b), L]).to("cuda", _tdt(dtype)).contiguous()
+        qn = x["Q"][np.arange(b), L]
+        q = torch.from_numpy(qn).to("cuda", _tdt(dtype)).contiguous()
+        st.step(q, k, v)
+        torch.cuda.synchronize()
+        lengths = L + 1
+        assert np.array_equal(st.seqlens.cpu().numpy(), lengths)
+        if step % 7 == 0 or step == 69:
+            _check_step(st, x, qn, lengths, chunk=B, alpha=1.5, gamma=6.0, dtype=dtype)
+    _check_summaries(st, x, B)
+
+
+def test_decode_matches_prefill_rows():
+    """Decode of position i equals prefill row i (same kernels' numerics up to bf16 rounding)."""
+    b, n, hq, hkv, d, B = 2, 700, 8, 2, 128, 64
+    x = inputs.planted(22, b, n, hq, hkv, d, B, dtype="bf16")
+    tq = {k: torch.from_numpy(x[k]).to("cuda", torch.bfloat16) for k in ("Q", "K", "V")}
+    pf = D.Prefill(tq["Q"], tq["K"], tq["V"], torch.from_numpy(x["qbar"]).cuda(), chunk=B, alpha=1.5, gamma=6.0)
+    Opf = pf().float()
+    st = _state(x, [600, 640], 1024, chunk=B, alpha=1.5, gamma=6.0, dtype="bf16")
+    for _ in range(40):
+        L = st.seqlens.cpu().numpy()
+        k = tq["K"][torch.arange(b), torch.from_numpy(L).long()].contiguous()
+        v = tq["V"][torch.arange(b), torch.from_numpy(L).long()].contiguous()
+        q = tq["Q"][torch.arange(b), torch.from_numpy(L).long()].contiguous()
+        o = st.step(q, k, v).float()
+        ref = Opf[torch.arange(b), torch.from_numpy(L).long()]
+        assert (o - ref).abs().max().item() < 2e-2
+
+
+def test_decode_128k_full_size_sampled():
+    """Full-size decode workload (b=8, 131072-token caches, 32/2 heads, d=128, B=64, ~25% routed):
+    fill, then append+decode steps; steps 0, 15 and 31 are checked against the oracle."""
+    wl = W.get("decode_128k")
+    x = wl.make()   # K, V for every position; queries for positions prefix..prefix+steps-1
+    prefix = wl.extra["prefix"]
+    st = _state(x, [prefix] * wl.batch, wl.n, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, dtype="bf16")
+    Kt = torch.from_numpy(x["K"][:, prefix:prefix + 32]).to("cuda", torch.bfloat16)
+    Vt = torch.from_numpy(x["V"][:, prefix:prefix + 32]).to("cuda", torch.bfloat16)
+    Qt = torch.from_numpy(x["Q"][:, :32]).to("cuda", torch.bfloat16)
+    for s in range(32):
+        st.step(Qt[:, s].contiguous(), Kt[:, s].contiguous(), Vt[:, s].contiguous())
+        if s in (0, 15, 31):
+            torch.cuda.synchronize()
+            lengths = np.full(wl.batch, prefix + s + 1)
+            stt = _check_step(st, x, x["Q"][:, s], lengths, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
+                              dtype="bf16")
+            print("decode_128k step", s, stt)
+    frac = st.rt[0].sum().item() / (wl.batch * 2 * ((prefix + 31) // 64))
+    assert 0.15 < frac < 0.35, frac

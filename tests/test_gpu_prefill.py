@@ -1,0 +1,147 @@
+"""GPU parity of the prefill path (dash_prefill through the C ABI) against the float64 oracle on
+the same seeded inputs: Stage 0 summaries, Stage 1 routed sets and biases, Stage 2 outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import adaptive_sparse_hierarchical_b200 as D
+from adaptive_sparse_hierarchical_b200 import inputs, workloads as W
+
+from parity import check_outputs, check_routes, gpu_sets
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda", torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
+def run_prefill(x, *, chunk, alpha, gamma, inv_sigma=1.0, dtype="bf16", bitmask=False):
+    Q, K, V = (_dev(x[k], dtype) for k in ("Q", "K", "V"))
+    qbar = torch.from_numpy(x["qbar"]).cuda()
+    pf = D.Prefill(Q, K, V, qbar, chunk=chunk, alpha=alpha, gamma=gamma, inv_sigma=inv_sigma, want_route=True,
+                   bitmask=bitmask)
+    O = pf()
+    torch.cuda.synchronize()
+    return O, pf
+
+
+def compare(x, pf, O, *, chunk, alpha, gamma, inv_sigma=1.0, dtype="bf16", positions=None):
+    b, n, hq, d = x["Q"].shape
+    hkv = x["K"].shape[2]
+    T = n // chunk
+    if positions is None:
+        positions = np.arange(n)
+    Oref, kbar, rt = oracle.prefill(x["Q"], x["K"], x["V"], x["qbar"], chunk=chunk, alpha=alpha, gamma=gamma,
+                                    inv_sigma=inv_sigma, positions=positions, want_route=True)
+    np.testing.assert_allclose(pf.kbar.cpu().numpy(), kbar, atol=2e-5, rtol=1e-5)
+    gs = gpu_sets(pf.counts.cpu().numpy(), pf.chunk_idx.cpu().numpy(), positions, chunk)
+    mism, nrows = check_routes(gs, rt, chunk, positions, T)
+    assert len(mism) <= max(1, 0.01 * nrows), f"{len(mism)} of {nrows} rows differ"
+    # biases of matching rows (chunks clear of the threshold)
+    idx = pf.chunk_idx.cpu().numpy()
+    bias = pf.bias.cpu().numpy()
+    cnts = pf.counts.cpu().numpy()
+    from parity import tri_offset
+    worst = 0.0
+    for (bb, r, t), lst in gs.items():
+        if (bb, r, t) in mism or len(lst) == 0:
+            continue
+        i = int(positions[t])
+        off = tri_offset(i, chunk)
+        mg = np.abs(rt["margin"][bb, r, t, lst])
+        if mg.min() < 1e-3:
+            continue
+        worst = max(worst, np.abs(bias[bb, r, off:off + cnts[bb, r, i]] - rt["bias"][bb, r, t, lst]).max())
+    assert worst < 5e-3, worst
+    Og = O.float().cpu().numpy()[:, positions]
+    return check_outputs(Og, Oref, dtype, hq // hkv, mism, rt, chunk, positions, T)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "tiny_f32_sparse", "tiny_bf16_sparse"])
+def test_tiny_workloads(name):
+    wl = W.get(name)
+    x = wl.make()
+    O, pf = run_prefill(x, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, dtype=wl.dtype)
+    st = compare(x, pf, O, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, dtype=wl.dtype)
+    print(name, st)
+
+
+CASES = [
+    # n, hq, hkv, d, B, gamma, alpha, inv_sigma, dtype
+    (1000, 8, 2, 128, 64, 6.0, 1.5, 1.0, "bf16"),
+    (777, 16, 2, 64, 32, 10.0, 1.5, 1.0, "bf16"),
+    (1300, 16, 1, 128, 128, 8.0, 1.5, 0.5, "bf16"),
+    (500, 4, 4, 64, 16, 5.0, 2.0, 1.0, "bf16"),
+    (257, 2, 1, 128, 64, 4.0, 1.25, 0.0, "bf16"),
+    (640, 16, 16, 128, 64, 7.0, 1.75, 1.0, "bf16"),
+    (600, 8, 2, 128, 32, 6.0, 1.5, 1.0, "f32"),
+    (300, 4, 1, 64, 16, 6.0, 2.0, 2.0, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"n{c[0]}_g{c[1] // c[2]}_d{c[3]}_B{c[4]}_{c[8]}" for c in CASES])
+def test_ragged_shapes(case):
+    n, hq, hkv, d, B, gamma, alpha, inv_sigma, dtype = case
+    x = inputs.planted(11, 2 if n < 700 else 1, n, hq, hkv, d, B, dtype=dtype, chunk_frac=0.1, strength=2.0)
+    O, pf = run_prefill(x, chunk=B, alpha=alpha, gamma=gamma, inv_sigma=inv_sigma, dtype=dtype)
+    compare(x, pf, O, chunk=B, alpha=alpha, gamma=gamma, inv_sigma=inv_sigma, dtype=dtype)
+
+
+@pytest.mark.parametrize("n", [1, 2, 63, 64, 65])
+def test_degenerate_lengths(n):
+    """Single token, sequences shorter than one chunk, exactly one chunk and one past it."""
+    x = inputs.planted(12, 1, n, 8, 2, 128, 64, dtype="bf16")
+    O, pf = run_prefill(x, chunk=64, alpha=1.5, gamma=6.0)
+    compare(x, pf, O, chunk=64, alpha=1.5, gamma=6.0)
+
+
+def test_gamma_zero_is_dense_causal_attention():
+    """gamma = 0 routes every visible chunk with zero bias: the output is dense causal attention,
+    checked against torch's own SDPA on the GPU (fp32 math on the same bf16 inputs)."""
+    x = inputs.planted(13, 1, 1536, 16, 2, 128, 64, dtype="bf16")
+    O, pf = run_prefill(x, chunk=64, alpha=1.5, gamma=0.0)
+    q, k, v = (torch.from_numpy(x[t]).cuda().permute(0, 2, 1, 3) for t in ("Q", "K", "V"))
+    k = k.repeat_interleave(8, dim=1)
+    v = v.repeat_interleave(8, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True).permute(0, 2, 1, 3)
+    err = (O.float() - ref).abs()
+    assert err.max().item() < 2e-2 and (err.mean() / ref.abs().mean()).item() < 1e-2
+    cnt = pf.counts.cpu().numpy()[0]
+    assert np.array_equal(cnt, np.broadcast_to(np.arange(1536) // 64, cnt.shape))
+
+
+def test_bitmask_matches_lists():
+    x = inputs.planted(14, 1, 2048, 8, 2, 128, 32, dtype="bf16")
+    O, pf = run_prefill(x, chunk=32, alpha=1.5, gamma=8.0, bitmask=True)
+    bm = pf.bitmask.cpu().numpy().view(np.uint32)
+    cnt, idx = pf.counts.cpu().numpy(), pf.chunk_idx.cpu().numpy()
+    from parity import tri_offset
+    for r in range(2):
+        for i in range(0, 2048, 37):
+            off = tri_offset(i, 32)
+            lst = idx[0, r, off:off + cnt[0, r, i]]
+            bits = np.unpackbits(bm[0, r, i].view(np.uint8), bitorder="little")
+            assert np.array_equal(np.nonzero(bits)[0], lst)
+
+
+def _sample_positions(n, B, k, seed):
+    rng = np.random.default_rng(seed)
+    edges = [0, 1, B - 1, B, B + 1, 2 * B - 1, n // 2, n - B, n - 2, n - 1]
+    starts = rng.integers(1, n // B, k // 4) * B
+    pos = np.concatenate([edges, starts, starts - 1, rng.integers(0, n, k - 2 * (k // 4) - len(edges))])
+    return np.unique(np.clip(pos, 0, n - 1))
+
+
+def test_prefill_32k_full_size_sampled():
+    """The benchmark workload at full size (b=1, n=32768, 16/2 heads, d=128, B=64, ~25% routed),
+    in the benchmark's launch configuration; outputs checked on sampled rows."""
+    wl = W.get("prefill_32k")
+    x = wl.make()
+    O, pf = run_prefill(x, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma)
+    pos = _sample_positions(wl.n, wl.chunk, 192, 0)
+    st = compare(x, pf, O, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, positions=pos)
+    frac = pf.counts.sum().item() / (2 * sum(i // 64 for i in range(wl.n)))
+    assert 0.2 < frac < 0.3, frac
+    print("prefill_32k", st, "routed fraction", frac)
