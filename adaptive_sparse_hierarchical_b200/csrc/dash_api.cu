@@ -210,6 +210,8 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
         return DASH_EALIGN;
     if (!strides_ok(p->k_strides, p->dtype) || !strides_ok(p->v_strides, p->dtype)) return DASH_EALIGN;
     if (!aligned4(seqlens)) return DASH_EALIGN;
+    // the routing step keeps every head's logits of one (sequence, KV head) in shared memory
+    if ((size_t)(p->h_q / p->h_kv) * (size_t)(p->seqlen / p->chunk) * 4 > 225 * 1024) return DASH_EUNSUPPORTED;
     const DecodeLayout L = decode_layout(p);
     if (!workspace || ws_bytes < L.total) return DASH_EWORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DASH_EALIGN;

@@ -15,12 +15,12 @@
 // from the left end (the tangent of a convex decreasing function stays below it, so the steps
 // never pass the root) finish to float precision.
 #include "dash_common.cuh"
+#include "stage2_mma.cuh"
 
 namespace dash {
 namespace {
 
-constexpr int kBisect = 20;
-constexpr int kNewton = 2;
+constexpr int kMaxIter = 32;
 
 __device__ __forceinline__ float ent_pow(float u, float p, int mode)
 {
@@ -34,39 +34,50 @@ __device__ __forceinline__ float ent_dpow(float u, float p, int mode)
 }
 __device__ __forceinline__ int ent_mode(float alpha) { return alpha == 2.f ? 1 : alpha == 1.5f ? 2 : 0; }
 
-// Warp-cooperative threshold of one row held in shared memory, x[0..nv).  Returns tau.
+// Threshold tau of alpha-entmax for one row, cooperatively.  each(fn) applies fn(x) to this
+// thread's entries; red(f, fd) sums both over the cooperating threads (uniform results).
+// Newton steps on g(t) = f(t)^(alpha-1), f(t) = sum [x - t]_+^p, p = 1/(alpha-1): g is a p-norm
+// of (x - t)_+, hence convex and decreasing, and exactly linear while the support is fixed, so
+// from t = max x - 1 (where f >= 1) the iterates rise monotonically to the root in a few steps.
+// The bracket [lo, hi] guards against rounding; a step leaving it falls back to bisection.
+template <typename Each, typename Red>
+__device__ float entmax_threshold(Each each, Red red, float mx, int nv, float alpha)
+{
+    const float p = 1.f / (alpha - 1.f);
+    const int mode = ent_mode(alpha);
+    float lo = mx - 1.f;
+    float hi = mx - exp2f(-(alpha - 1.f) * __log2f((float)nv));
+    float t = lo;
+    for (int it = 0; it < kMaxIter; ++it) {
+        float f = 0.f, fd = 0.f;
+        each([&](float x) {
+            const float u = x - t;
+            if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
+        });
+        red(f, fd);
+        if (f >= 1.f) lo = t; else hi = t;
+        float tn = 0.5f * (lo + hi);
+        if (fd > 0.f && f > 0.f) {
+            const float gg = mode == 2 ? sqrtf(f) : mode == 1 ? f : exp2f((alpha - 1.f) * __log2f(f));
+            tn = t + (gg - 1.f) * f / (gg * fd);
+        }
+        if (fabsf(tn - t) <= 2e-7f * fmaxf(1.f, fabsf(t)) || fabsf(f - 1.f) <= 1e-6f) { t = tn; break; }
+        if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+        t = tn;
+    }
+    return t;
+}
+
+// Warp-cooperative threshold of one row held in shared memory, x[0..nv).
 __device__ float warp_threshold(const float* x, int nv, float alpha)
 {
     const int lane = threadIdx.x & 31;
-    const float p = 1.f / (alpha - 1.f);
-    const int mode = ent_mode(alpha);
     float mx = -INFINITY;
     for (int c = lane; c < nv; c += 32) mx = fmaxf(mx, x[c]);
     mx = warp_max(mx);
-    float lo = mx - 1.f;
-    float hi = mx - exp2f(-(alpha - 1.f) * __log2f((float)nv));
-    for (int it = 0; it < kBisect; ++it) {
-        const float t = 0.5f * (lo + hi);
-        float f = 0.f;
-        for (int c = lane; c < nv; c += 32) {
-            float u = x[c] - t;
-            if (u > 0.f) f += ent_pow(u, p, mode);
-        }
-        f = warp_sum(f);
-        if (f >= 1.f) lo = t; else hi = t;
-    }
-    float t = lo;
-    for (int it = 0; it < kNewton; ++it) {
-        float f = 0.f, fd = 0.f;
-        for (int c = lane; c < nv; c += 32) {
-            float u = x[c] - t;
-            if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
-        }
-        f = warp_sum(f) - 1.f;
-        fd = warp_sum(fd) * p;
-        if (fd > 0.f) t = fminf(fmaxf(t + f / fd, lo), hi);
-    }
-    return t;
+    return entmax_threshold(
+        [&](auto fn) { for (int c = lane; c < nv; c += 32) fn(x[c]); },
+        [](float& a, float& b) { a = warp_sum(a); b = warp_sum(b); }, mx, nv, alpha);
 }
 
 // Ordered compaction of one position's routed chunks by one warp; writes the list, the count
@@ -221,6 +232,128 @@ __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __
 }
 
 // ------------------------------------------------------------------------------------------
+// Prefill, bf16 queries: the chunk logits run on the tensor cores.  A query is exact in bf16;
+// each fp32 summary is split exactly into three bf16 planes (hi + mid + lo = kbar, 8 mantissa
+// bits each), so three bf16 MMAs with fp32 accumulation reproduce the fp32 dot product.
+// Block = 8 warps, ROWS = 16*RG query rows = ROWS/g positions of one (sequence, KV head).
+// Shared memory: one 64-chunk summary tile as three swizzled bf16 planes, logits [ROWS][Ts].
+// ------------------------------------------------------------------------------------------
+template <int D, int RG>
+__global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __nv_bfloat16* __restrict__ Q,
+                                                               const float* __restrict__ kbar, Routes rt, int Ts)
+{
+    constexpr int ROWS = 16 * RG;
+    constexpr int PLANE = 64 * D * 2;
+    extern __shared__ __align__(128) char smem[];
+    char* kt = smem;
+    float* S = reinterpret_cast<float*>(smem + 3 * PLANE);
+    const int G = s.g, P = ROWS / G;
+    const int nblk = (s.n + P - 1) / P;
+    const int br = blockIdx.x % (s.batch * s.hkv);
+    const int pb = nblk - 1 - blockIdx.x / (s.batch * s.hkv);   // heaviest blocks first
+    const int b = br / s.hkv, r = br % s.hkv;
+    const int i0 = pb * P;
+    const int ilast = min(i0 + P, s.n) - 1;
+    const int nvmax = min(ilast / s.B, s.T);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int* counts = rt.counts + (long long)br * s.n;
+    int* idx = rt.idx + (long long)br * rt.cap;
+    float* bias = rt.bias + (long long)br * rt.cap;
+    uint32_t* bm = rt.bitmask ? rt.bitmask + (long long)br * s.n * rt.words : nullptr;
+    if (nvmax == 0) {
+        for (int p = tid; p < P && i0 + p < s.n; p += blockDim.x) counts[i0 + p] = 0;
+        if (bm)
+            for (int k = tid; k < P * rt.words; k += blockDim.x)
+                if (i0 + k / rt.words < s.n) bm[(long long)i0 * rt.words + k] = 0u;
+        return;
+    }
+    const int rg = warp % RG;
+    uint32_t qf[D / 16][4];
+    load_q_frags<D>(qf, [&](int rr) -> const __nv_bfloat16* {
+        const int R = rg * 16 + rr, i = i0 + R / G;
+        if (i >= s.n) return nullptr;
+        return Q + (long long)b * s.qs[0] + (long long)i * s.qs[1] + (long long)(r * G + R % G) * s.qs[2];
+    });
+    const float xs = (s.alpha - 1.f) * s.gamma * rsqrtf((float)D);
+    const float* kb = kbar + (long long)br * s.T * D;
+    const int mi = lane >> 3, rr8 = lane & 7, t4 = lane & 3;
+    for (int c0 = 0; c0 < nvmax; c0 += 64) {
+        __syncthreads();
+        for (int v = tid; v < 64 * (D / 4); v += 256) {
+            const int cc = v / (D / 4), e = (v % (D / 4)) * 4;
+            float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c0 + cc < nvmax) val = *reinterpret_cast<const float4*>(kb + (long long)(c0 + cc) * D + e);
+            const float xv[4] = {val.x, val.y, val.z, val.w};
+            __nv_bfloat16 hb[4], mb[4], lb[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                hb[k] = __float2bfloat16_rn(xv[k]);
+                const float rem = xv[k] - __bfloat162float(hb[k]);
+                mb[k] = __float2bfloat16_rn(rem);
+                lb[k] = __float2bfloat16_rn(rem - __bfloat162float(mb[k]));
+            }
+            const uint32_t off = swz<D>(cc, e);
+            *reinterpret_cast<uint2*>(kt + off) = *reinterpret_cast<uint2*>(hb);
+            *reinterpret_cast<uint2*>(kt + PLANE + off) = *reinterpret_cast<uint2*>(mb);
+            *reinterpret_cast<uint2*>(kt + 2 * PLANE + off) = *reinterpret_cast<uint2*>(lb);
+        }
+        __syncthreads();
+        for (int u = warp; u < RG * 4; u += 8) {
+            const int slice = u / RG;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = swz<D>(slice * 16 + rr8 + (mi >> 1) * 8, kk * 16 + (mi & 1) * 8);
+#pragma unroll
+                for (int pl = 0; pl < 3; ++pl) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(smem_u32(kt + pl * PLANE) + off, b0, b1, b2, b3);
+                    mma_bf16(acc[0], qf[kk], b0, b1);
+                    mma_bf16(acc[1], qf[kk], b2, b3);
+                }
+            }
+            const int ra = rg * 16 + (lane >> 2), rb = ra + 8;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int col = c0 + slice * 16 + j * 8 + 2 * t4;
+                *reinterpret_cast<float2*>(S + ra * Ts + col) = make_float2(acc[j][0] * xs, acc[j][1] * xs);
+                *reinterpret_cast<float2*>(S + rb * Ts + col) = make_float2(acc[j][2] * xs, acc[j][3] * xs);
+            }
+        }
+    }
+    __syncthreads();
+    for (int row = warp; row < ROWS; row += 8) {
+        const int i = i0 + row / G;
+        if (i >= s.n) continue;
+        const int nv = min(i / s.B, s.T);
+        if (nv == 0) continue;
+        float* x = S + row * Ts;
+        const float tau = warp_threshold(x, nv, s.alpha);
+        const float p = 1.f / (s.alpha - 1.f);
+        const int mode = ent_mode(s.alpha);
+        for (int c = lane; c < nv; c += 32) {
+            const float u = x[c] - tau;
+            x[c] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
+        }
+    }
+    __syncthreads();
+    for (int p = warp; p < P; p += 8) {
+        const int i = i0 + p;
+        if (i >= s.n) continue;
+        const int nv = min(i / s.B, s.T);
+        const float* W = S + p * G * Ts;
+        auto wsum = [&](int c) {
+            float a = 0.f;
+            for (int h = 0; h < G; ++h) a += W[h * Ts + c];
+            return a;
+        };
+        const long long off = tri_offset(i, s.B);
+        warp_emit(wsum, nv, 1.f / G, s.inv_sigma, idx + off, bias + off, counts + i,
+                  bm ? bm + (long long)i * rt.words : nullptr, rt.words);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // Decode: the single query of sequence b sits at position L_b - 1 (L_b = seqlens[b]) and sees
 // the cached summaries of chunks c < floor((L_b - 1)/B).
 // (a) logits: one block per (32-chunk tile, sequence, KV head), all g heads of the group.
@@ -261,86 +394,83 @@ __global__ void __launch_bounds__(256) dec_logits_kernel(Shape s, const T* __res
     }
 }
 
-// (b) threshold: one block per (head, sequence, KV head); block-wide reductions.
-__device__ float block_sum(float v, float* red)
+// (b) thresholds, GQA average, bias and ordered compaction for one (sequence, KV head): the
+// logits of the g heads are copied to shared memory, one warp per head solves its threshold,
+// then the whole block averages the heads and writes the ascending route list.
+__global__ void __launch_bounds__(512) dec_route_kernel(Shape s, int kbar_T, const int* __restrict__ seqlens,
+                                                        const float* __restrict__ X, Routes rt)
 {
-    v = warp_sum(v);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float t = lane < nw ? red[lane] : 0.f;
-    return warp_sum(t);
-}
-__device__ float block_max(float v, float* red)
-{
-    v = warp_max(v);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float t = lane < nw ? red[lane] : -INFINITY;
-    return warp_max(t);
-}
-
-__global__ void __launch_bounds__(256) dec_tau_kernel(Shape s, int kbar_T, const int* __restrict__ seqlens,
-                                                      float* X)
-{
-    __shared__ float red[32];
-    const int h = blockIdx.x, br = blockIdx.y, b = br / s.hkv;
-    const int nv = min((seqlens[b] - 1) / s.B, kbar_T);
-    if (nv <= 0) return;
-    float* x = X + ((long long)br * s.g + h) * kbar_T;
-    const float p = 1.f / (s.alpha - 1.f);
-    const int mode = ent_mode(s.alpha);
-    float mx = -INFINITY;
-    for (int c = threadIdx.x; c < nv; c += blockDim.x) mx = fmaxf(mx, x[c]);
-    mx = block_max(mx, red);
-    float lo = mx - 1.f, hi = mx - exp2f(-(s.alpha - 1.f) * __log2f((float)nv));
-    for (int it = 0; it < kBisect; ++it) {
-        const float t = 0.5f * (lo + hi);
-        float f = 0.f;
-        for (int c = threadIdx.x; c < nv; c += blockDim.x) {
-            const float u = x[c] - t;
-            if (u > 0.f) f += ent_pow(u, p, mode);
-        }
-        f = block_sum(f, red);
-        if (f >= 1.f) lo = t; else hi = t;
-    }
-    float t = lo;
-    for (int it = 0; it < kNewton; ++it) {
-        float f = 0.f, fd = 0.f;
-        for (int c = threadIdx.x; c < nv; c += blockDim.x) {
-            const float u = x[c] - t;
-            if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
-        }
-        f = block_sum(f, red) - 1.f;
-        fd = block_sum(fd, red) * p;
-        if (fd > 0.f) t = fminf(fmaxf(t + f / fd, lo), hi);
-    }
-    __syncthreads();
-    for (int c = threadIdx.x; c < nv; c += blockDim.x) {
-        const float u = x[c] - t;
-        x[c] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
-    }
-}
-
-// (c) GQA average, bias and compaction: one warp per (sequence, KV head).
-__global__ void __launch_bounds__(32) dec_emit_kernel(Shape s, int kbar_T, const int* __restrict__ seqlens,
-                                                      const float* __restrict__ X, Routes rt)
-{
-    const int br = blockIdx.x, b = br / s.hkv;
+    extern __shared__ float xsm[];   // [g][kbar_T]
+    __shared__ float red_f[16];
+    __shared__ int red_i[16], wpos[17];
+    const int br = blockIdx.x, b = br / s.hkv, G = s.g;
     const int nv = max(0, min((seqlens[b] - 1) / s.B, kbar_T));
-    const float* W = X + (long long)br * s.g * kbar_T;
-    const int g = s.g;
-    auto wsum = [&](int c) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+    const float* Xb = X + (long long)br * G * kbar_T;
+    for (int v = tid; v < G * nv; v += blockDim.x) {
+        const int h = v / nv, c = v % nv;
+        xsm[h * kbar_T + c] = Xb[(long long)h * kbar_T + c];
+    }
+    __syncthreads();
+    if (nv > 0 && warp < G) {
+        float* x = xsm + warp * kbar_T;
+        const float tau = warp_threshold(x, nv, s.alpha);
+        const float p = 1.f / (s.alpha - 1.f);
+        const int mode = ent_mode(s.alpha);
+        for (int c = lane; c < nv; c += 32) {
+            const float u = x[c] - tau;
+            x[c] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
+        }
+    }
+    __syncthreads();
+    const float inv_g = 1.f / G;
+    auto wof = [&](int c) {
         float a = 0.f;
-        for (int h = 0; h < g; ++h) a += W[(long long)h * kbar_T + c];
-        return a;
+        for (int h = 0; h < G; ++h) a += xsm[h * kbar_T + c];
+        return a * inv_g;
     };
-    warp_emit(wsum, nv, 1.f / g, s.inv_sigma, rt.idx + (long long)br * rt.cap,
-              rt.bias + (long long)br * rt.cap, rt.counts + br,
-              rt.bitmask ? rt.bitmask + (long long)br * rt.words : nullptr, rt.words);
+    float sl = 0.f;
+    int cnt = 0;
+    for (int c = tid; c < nv; c += blockDim.x) {
+        const float w = wof(c);
+        if (w > 0.f) { sl += __logf(w); ++cnt; }
+    }
+    sl = warp_sum(sl);
+    cnt = warp_isum(cnt);
+    if (lane == 0) { red_f[warp] = sl; red_i[warp] = cnt; }
+    __syncthreads();
+    float tot = 0.f;
+    int tcnt = 0;
+    for (int k = 0; k < nw; ++k) { tot += red_f[k]; tcnt += red_i[k]; }
+    const float mu = tcnt > 0 ? tot / tcnt : 0.f;
+    int* idx = rt.idx + (long long)br * rt.cap;
+    float* bias = rt.bias + (long long)br * rt.cap;
+    uint32_t* mrow = rt.bitmask ? rt.bitmask + (long long)br * rt.words : nullptr;
+    int base = 0;
+    for (int c0 = 0; c0 < nv; c0 += blockDim.x) {
+        const int c = c0 + tid;
+        const float w = c < nv ? wof(c) : 0.f;
+        const bool on = w > 0.f;
+        const uint32_t m = __ballot_sync(0xffffffffu, on);
+        if (lane == 0) red_i[warp] = __popc(m);
+        __syncthreads();
+        if (tid == 0) {
+            wpos[0] = 0;
+            for (int k = 0; k < nw; ++k) wpos[k + 1] = wpos[k] + red_i[k];
+        }
+        __syncthreads();
+        if (on) {
+            const int k = base + wpos[warp] + __popc(m & ((1u << lane) - 1u));
+            idx[k] = c;
+            bias[k] = (__logf(w) - mu) * s.inv_sigma;
+        }
+        if (mrow && lane == 0 && c0 + 32 * warp < nv) mrow[(c0 + 32 * warp) >> 5] = m;
+        base += wpos[nw];
+        __syncthreads();
+    }
+    if (mrow)
+        for (int wd = ((nv + 31) >> 5) + tid; wd < rt.words; wd += blockDim.x) mrow[wd] = 0u;
+    if (tid == 0) rt.counts[br] = base;
 }
 
 template <typename T, int D>
@@ -361,6 +491,42 @@ cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, co
     return cudaGetLastError();
 }
 
+// Shared memory of the tensor-core routing kernel for RG row groups.
+size_t route_tc_smem(const Shape& s, int RG)
+{
+    const int Ts = (s.T + 63) / 64 * 64 + 8;
+    return 3 * (size_t)64 * s.d * 2 + (size_t)16 * RG * Ts * 4;
+}
+
+template <int D, int RG>
+cudaError_t route_tc_t(const Shape& s, const void* Q, const float* kbar, const Routes& rt, cudaStream_t st)
+{
+    const size_t smem = route_tc_smem(s, RG);
+    const int Ts = (s.T + 63) / 64 * 64 + 8;
+    auto k = route_prefill_tc_kernel<D, RG>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int P = 16 * RG / s.g;
+    const long long nblk = (s.n + P - 1) / P;
+    const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
+    if (grid == 0) return cudaSuccess;
+    k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, kbar, rt, Ts);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t route_tc_d(const Shape& s, const void* Q, const float* kbar, const Routes& rt, cudaStream_t st,
+                       bool* used)
+{
+    constexpr size_t kLimit = 225 * 1024;
+    *used = true;
+    if (16 * 4 >= s.g && route_tc_smem(s, 4) <= kLimit) return route_tc_t<D, 4>(s, Q, kbar, rt, st);
+    if (16 * 2 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, kbar, rt, st);
+    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, kbar, rt, st);
+    *used = false;
+    return cudaSuccess;
+}
+
 template <typename T, int D>
 cudaError_t dec_route_t(const Shape& s, const void* q, const float* kbar, int kbar_T,
                         const int* seqlens, const Routes& rt, float* X, cudaStream_t st)
@@ -368,10 +534,11 @@ cudaError_t dec_route_t(const Shape& s, const void* q, const float* kbar, int kb
     if (kbar_T > 0) {
         dim3 g1((kbar_T + 31) / 32, s.batch * s.hkv);
         dec_logits_kernel<T, D><<<g1, 256, 0, st>>>(s, (const T*)q, kbar, kbar_T, seqlens, X);
-        dim3 g2(s.g, s.batch * s.hkv);
-        dec_tau_kernel<<<g2, 256, 0, st>>>(s, kbar_T, seqlens, X);
     }
-    dec_emit_kernel<<<s.batch * s.hkv, 32, 0, st>>>(s, kbar_T, seqlens, X, rt);
+    const size_t smem = (size_t)s.g * (kbar_T > 0 ? kbar_T : 1) * 4;
+    cudaError_t e = cudaFuncSetAttribute(dec_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dec_route_kernel<<<s.batch * s.hkv, 32 * s.g, smem, st>>>(s, kbar_T, seqlens, X, rt);
     return cudaGetLastError();
 }
 
@@ -396,9 +563,14 @@ size_t route_prefill_smem(const Shape& s, int* positions_per_block)
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
                                  const Routes& rt, cudaStream_t st)
 {
-    if (dtype == DASH_BF16)
+    if (dtype == DASH_BF16) {
+        bool used = false;
+        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, kbar, rt, st, &used) : route_tc_d<64>(s, Q, kbar, rt, st, &used);
+        if (used) return e;
+        // very long rows (T * 16 rows of logits beyond shared memory): CUDA-core variant
         return s.d == 128 ? route_prefill_t<__nv_bfloat16, 128>(s, Q, kbar, rt, st)
                           : route_prefill_t<__nv_bfloat16, 64>(s, Q, kbar, rt, st);
+    }
     return s.d == 128 ? route_prefill_t<float, 128>(s, Q, kbar, rt, st)
                       : route_prefill_t<float, 64>(s, Q, kbar, rt, st);
 }
