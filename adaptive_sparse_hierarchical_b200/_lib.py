@@ -53,6 +53,8 @@ def load():
         vp, sz = ctypes.c_void_p, ctypes.c_size_t
         lib.dash_workspace_size.argtypes = [P, ctypes.c_int]
         lib.dash_workspace_size.restype = sz
+        lib.dash_error_word_offset.argtypes = [P, ctypes.c_int]
+        lib.dash_error_word_offset.restype = ctypes.c_longlong
         lib.dash_route_capacity.argtypes = [P]
         lib.dash_route_capacity.restype = ctypes.c_longlong
         lib.dash_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, R, vp, sz, vp]
@@ -117,6 +119,10 @@ def route_out(counts=None, chunk_idx=None, bias=None, bitmask=None):
 
 def dash_workspace_size(p: dash_params, op: int) -> int:
     return int(load().dash_workspace_size(ctypes.byref(p), op))
+
+
+def dash_error_word_offset(p: dash_params, op: int) -> int:
+    return int(load().dash_error_word_offset(ctypes.byref(p), op))
 
 
 def dash_route_capacity(p: dash_params) -> int:

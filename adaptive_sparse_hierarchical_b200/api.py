@@ -59,6 +59,11 @@ class Prefill:
         L.dash_prefill_stage(self.p, k, self.Q, self.K, self.V, self.qbar, self.O, self.kbar, self.route,
                              self.workspace, stream=stream)
 
+    def error_word(self) -> int:
+        """Status word of the last call (0 = every bounded wait completed)."""
+        off = L.dash_error_word_offset(self.p, L.DASH_OP_PREFILL)
+        return int(self.workspace[off:off + 4].view(torch.int32).item())
+
     def __call__(self, stream=None):
         L.dash_prefill(self.p, self.Q, self.K, self.V, self.qbar, self.O, self.kbar, self.route, self.workspace,
                        stream=stream)

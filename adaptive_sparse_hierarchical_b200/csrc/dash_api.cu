@@ -61,7 +61,7 @@ long long route_cap(const dash_params* p)
     return tri_offset(p->seqlen, p->chunk);
 }
 
-struct PrefillLayout { size_t kbar, counts, idx, bias, total; };
+struct PrefillLayout { size_t kbar, counts, idx, bias, err, total; };
 PrefillLayout prefill_layout(const dash_params* p)
 {
     PrefillLayout L;
@@ -72,7 +72,8 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.counts = L.kbar + up(bh * T * p->d_h * 4);
     L.idx = L.counts + up(bh * (size_t)p->seqlen * 4);
     L.bias = L.idx + up(bh * cap * 4);
-    L.total = L.bias + up(bh * cap * 4);
+    L.err = L.bias + up(bh * cap * 4);
+    L.total = L.err + kAlign;
     return L;
 }
 
@@ -105,6 +106,12 @@ size_t dash_workspace_size(const dash_params* p, int op)
     if (op == DASH_OP_PREFILL) return prefill_layout(p).total;
     if (op == DASH_OP_DECODE) return decode_layout(p).total;
     return 0;
+}
+
+long long dash_error_word_offset(const dash_params* p, int op)
+{
+    if (check_params(p) != DASH_OK || op != DASH_OP_PREFILL) return -1;
+    return (long long)prefill_layout(p).err;
 }
 
 long long dash_route_capacity(const dash_params* p)
@@ -164,7 +171,11 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
         rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, rt, st));
         if (rc != DASH_OK) return rc;
     }
-    if (stage == -1 || stage == DASH_STAGE2) rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt, st));
+    if (stage == -1 || stage == DASH_STAGE2) {
+        int* err = reinterpret_cast<int*>(ws + L.err);
+        if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return DASH_ELAUNCH;
+        rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt, err, st));
+    }
     return rc;
 }
 

@@ -100,7 +100,13 @@ cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const
 size_t route_prefill_smem(const Shape& s, int* positions_per_block);
 // Stage 2 for prefill.
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,
-                                  const void* V, void* O, const Routes& rt, cudaStream_t st);
+                                  const void* V, void* O, const Routes& rt, int* err, cudaStream_t st);
+// tcgen05 / TMEM / TMA variant (bf16, d = 128, chunk 64 or 128); err receives a non-zero code
+// when one of its bounded waits times out.
+bool attend_tc_supported(const Shape& s, int dtype);
+cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
+                                     const Routes& rt, int* err, cudaStream_t st);
+bool legacy_stage2();
 // Decode: Stage 1 (logits, thresholds, GQA aggregation) and Stage 2 (split + merge).
 struct DecodeWs {
     float* x;        // [b, hkv, g, T]  scaled logits, then head weights

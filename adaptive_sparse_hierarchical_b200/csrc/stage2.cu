@@ -7,6 +7,7 @@
 //   o = sum_{j in R u D} exp(z_j + d_j) v_j / sum exp(z_j + d_j),  z_j = <q,k_j>/sqrt(d),
 //   d_j = bias of chunk c(j) for routed tokens, 0 for the diagonal tokens c(i)B..i.
 #include <climits>
+#include <cstdlib>
 
 #include "stage2_mma.cuh"
 
@@ -445,12 +446,24 @@ cudaError_t rows_t(const Shape& s, const void* Q, const void* K, const void* V, 
 }  // namespace
 
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K, const void* V,
-                                  void* O, const Routes& rt, cudaStream_t st)
+                                  void* O, const Routes& rt, int* err, cudaStream_t st)
 {
+    if (attend_tc_supported(s, dtype) && !legacy_stage2()) return launch_attend_prefill_tc(s, Q, K, V, O, rt, err, st);
     if (dtype == DASH_BF16)
         return s.d == 128 ? prefill_bf16_d<128>(s, Q, K, V, O, rt, st) : prefill_bf16_d<64>(s, Q, K, V, O, rt, st);
     return s.d == 128 ? rows_t<float, 128>(s, Q, K, V, O, rt, nullptr, st)
                       : rows_t<float, 64>(s, Q, K, V, O, rt, nullptr, st);
+}
+
+bool legacy_stage2()
+{
+    // DASH_STAGE2=mma selects the warp-level mma.sync kernel for comparison runs.
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("DASH_STAGE2");
+        v = (e && e[0] == 'm') ? 1 : 0;
+    }
+    return v == 1;
 }
 
 int decode_splits(const Shape& s, int kbar_T)

@@ -1,0 +1,425 @@
+// stage2_tc.cu -- Stage 2 prefill on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// DashAttention (xllm-io paper review, section 3, Proposition 4.1 and the "Stage 2" kernel row):
+// per query row, o = softmax(<q,k_j>/sqrt(d) + d_j) V over the tokens of the routed chunks
+// (d_j = the chunk's bias) and the diagonal tokens c(i)B..i (d_j = 0), in one online-softmax pass
+// over the routed chunks.
+//
+// One block = 128 query rows = (128/g positions) x (g heads) of one (sequence, KV head); the
+// heads of a position share one routing list, so the block walks the union of its positions'
+// routed chunks plus their diagonal chunks, ascending, in tiles of 64 keys.  Rows that did not
+// route a tile get -inf there.  Roles (6 warps):
+//   warp 0      TMA producer: the Q tile once, then K and V tiles into a 4-slot ring
+//   warp 1      allocates TMEM and issues the MMAs from one thread:
+//               S = Q K^T  (M=128, N=64, K=128; two S buffers in TMEM)
+//               O += P V   (M=128, N=128, K=64; O accumulates in TMEM)
+//   warps 2-5   softmax, one thread per row (TMEM lane): S from TMEM, bias / causal mask,
+//               running max and sum in base 2, P (bf16) to shared memory; O in TMEM is rescaled
+//               only when a row's maximum grows by more than 2^8, otherwise the stale maximum
+//               is kept (values stay <= 2^8, exact in the final normalisation).
+// Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
+#include <climits>
+#include <cudaTypedefs.h>
+
+#include "dash_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace dash {
+namespace {
+
+constexpr int kRows = 128, kKT = 64, kD = 128, kNS = 4;
+constexpr int kQBytes = kRows * kD * 2;           // 32 KB, two 16 KB d-halves
+constexpr int kKVHalf = kKT * 64 * 2;             // 8 KB: [64 keys][64 d]
+constexpr int kSlot = 4 * kKVHalf;                // K (2 halves) + V (2 halves) = 32 KB
+constexpr int kPBytes = kRows * kKT * 2;          // 16 KB
+constexpr int kTmemCols = 256;                    // S0 [0,64), S1 [64,128), O [128,256)
+constexpr int kOffQ = 0, kOffSlots = kQBytes, kOffP = kOffSlots + kNS * kSlot;
+constexpr int kOffBar = kOffP + 2 * kPBytes;      // 196608
+constexpr int kNumBars = 1 + 2 * kNS + 2 + 2 + 2 + 2 + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, njobs
+constexpr int kOffJobs = kOffMisc + 32;
+
+constexpr uint32_t kIdescS = tc::idesc_bf16(128, 64, false, false);
+constexpr uint32_t kIdescPV = tc::idesc_bf16(128, 128, false, true);
+
+struct Bars {
+    uint32_t q_full, kv_full[kNS], kv_empty[kNS], s_full[2], s_free[2], p_full[2], pv_done[2], drain;
+};
+
+__device__ __forceinline__ Bars make_bars(uint32_t base)
+{
+    Bars b;
+    uint32_t a = base + kOffBar;
+    b.q_full = a; a += 8;
+    for (int k = 0; k < kNS; ++k) { b.kv_full[k] = a; a += 8; }
+    for (int k = 0; k < kNS; ++k) { b.kv_empty[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.s_full[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.s_free[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.p_full[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.pv_done[k] = a; a += 8; }
+    b.drain = a;
+    return b;
+}
+
+__global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                   const __grid_constant__ CUtensorMap tmK,
+                                                                   const __grid_constant__ CUtensorMap tmV,
+                                                                   Shape s, Routes rt,
+                                                                   __nv_bfloat16* __restrict__ O, int* err)
+{
+    extern __shared__ char smem_raw[];
+    char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = tc::smem_addr(sm);
+    const Bars bar = make_bars(base);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+    int* njobs_s = reinterpret_cast<int*>(sm + kOffMisc + 8);
+    int* jobs = reinterpret_cast<int*>(sm + kOffJobs);
+    uint32_t* umask = reinterpret_cast<uint32_t*>(sm + kOffP);   // scratch until P is used
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = s.g, P = kRows / G;
+    const int nblk = (s.n + P - 1) / P;
+    const int br = blockIdx.x % (s.batch * s.hkv);
+    const int pb = nblk - 1 - blockIdx.x / (s.batch * s.hkv);   // heaviest blocks first
+    const int b = br / s.hkv, r = br % s.hkv;
+    const int i0 = pb * P;
+    const int* counts = rt.counts + (long long)br * s.n;
+    const int* ridx = rt.idx + (long long)br * rt.cap;
+    const float* rbias = rt.bias + (long long)br * rt.cap;
+    const int W = (s.T + 32) >> 5;
+    const int NH = s.B / kKT;
+
+    // ---- set-up: barriers, TMEM, union of the block's routed + diagonal chunks --------------
+    if (tid == 0) {
+        tc::mbar_init(bar.q_full, 1);
+        for (int k = 0; k < kNS; ++k) { tc::mbar_init(bar.kv_full[k], 1); tc::mbar_init(bar.kv_empty[k], 1); }
+        for (int k = 0; k < 2; ++k) {
+            tc::mbar_init(bar.s_full[k], 1);
+            tc::mbar_init(bar.s_free[k], 128);
+            tc::mbar_init(bar.p_full[k], 128);
+            tc::mbar_init(bar.pv_done[k], 1);
+        }
+        tc::mbar_init(bar.drain, 1);
+        *abort = 0;
+        tc::mbar_fence_init();
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_alloc(tc::smem_addr(tmem_slot), kTmemCols);
+    }
+    for (int w = tid; w < W; w += blockDim.x) umask[w] = 0u;
+    __syncthreads();
+    for (int p = 0; p < P; ++p) {
+        const int i = i0 + p;
+        if (i >= s.n) break;
+        const int cnt = counts[i];
+        const int* li = ridx + tri_offset(i, s.B);
+        for (int k = tid; k < cnt; k += blockDim.x) atomicOr(&umask[li[k] >> 5], 1u << (li[k] & 31));
+        if (tid == 0) atomicOr(&umask[(i / s.B) >> 5], 1u << ((i / s.B) & 31));
+    }
+    __syncthreads();
+    if (warp == 0) {   // ordered bitmask -> list of chunk ids
+        int basec = 0;
+        for (int w0 = 0; w0 < W; w0 += 32) {
+            const uint32_t bits = w0 + lane < W ? umask[w0 + lane] : 0u;
+            const int pc = __popc(bits);
+            int incl = pc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int at = basec + incl - pc;
+            uint32_t bb = bits;
+            while (bb) {
+                const int bit = __ffs(bb) - 1;
+                jobs[at++] = ((w0 + lane) << 5) + bit;
+                bb &= bb - 1u;
+            }
+            basec += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) *njobs_s = basec * NH;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int njobs = *njobs_s;
+
+    if (warp == 0) {
+        // ---- TMA producer ------------------------------------------------------------------
+        if (lane == 0 && njobs > 0) {
+            tc::prefetch_tmap(&tmQ);
+            tc::prefetch_tmap(&tmK);
+            tc::prefetch_tmap(&tmV);
+            tc::mbar_expect_tx(bar.q_full, kQBytes);
+            tc::tma_load_4d(base + kOffQ, &tmQ, bar.q_full, 0, r * G, i0, b);
+            tc::tma_load_4d(base + kOffQ + kQBytes / 2, &tmQ, bar.q_full, 64, r * G, i0, b);
+            int last[kNS];
+            for (int k = 0; k < kNS; ++k) last[k] = -1;
+            for (int k = 0; k < njobs; ++k) {
+                const int slot = k % kNS;
+                if (k >= kNS && !tc::mbar_wait(bar.kv_empty[slot], ((k / kNS) - 1) & 1, abort, err, 1)) break;
+                last[slot] = k;
+                const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
+                const uint32_t dst = base + kOffSlots + slot * kSlot;
+                tc::mbar_expect_tx(bar.kv_full[slot], kSlot);
+                tc::tma_load_4d(dst, &tmK, bar.kv_full[slot], 0, r, key0, b);
+                tc::tma_load_4d(dst + kKVHalf, &tmK, bar.kv_full[slot], 64, r, key0, b);
+                tc::tma_load_4d(dst + 2 * kKVHalf, &tmV, bar.kv_full[slot], 0, r, key0, b);
+                tc::tma_load_4d(dst + 3 * kKVHalf, &tmV, bar.kv_full[slot], 64, r, key0, b);
+            }
+            if (*abort) {
+                // let this block's TMA copies still in flight land before its shared memory goes away
+                for (int k = 0; k < kNS; ++k)
+                    if (last[k] >= 0)
+                        for (long long it = 0; it < (1ll << 22); ++it)
+                            if (tc::mbar_try(bar.kv_full[k], (last[k] / kNS) & 1)) break;
+                for (long long it = 0; it < (1ll << 22); ++it)
+                    if (tc::mbar_try(bar.q_full, 0)) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer --------------------------------------------------------------------
+        if (lane == 0 && njobs > 0) {
+            const uint32_t sQ = base + kOffQ, sP = base + kOffP;
+            auto issue_pv = [&](int j) -> bool {
+                const int pbuf = j & 1;
+                if (!tc::mbar_wait(bar.p_full[pbuf], (j >> 1) & 1, abort, err, 2)) return false;
+                tc::fence_after_sync();
+                const uint32_t sV = base + kOffSlots + (j % kNS) * kSlot + 2 * kKVHalf;
+#pragma unroll
+                for (int kk = 0; kk < kKT / 16; ++kk) {
+                    const uint64_t ad = tc::sw128_desc(sP + pbuf * kPBytes + kk * 32, 16, 1024);
+                    const uint64_t bd = tc::sw128_desc(sV + kk * 2048, kKVHalf, 1024);
+                    tc::mma_f16_ss(tmem + 128, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(bar.kv_empty[j % kNS]);
+                tc::mma_commit(bar.pv_done[pbuf]);
+                return true;
+            };
+            bool ok = tc::mbar_wait(bar.q_full, 0, abort, err, 3);
+            for (int k = 0; ok && k < njobs; ++k) {
+                const int slot = k % kNS, sb = k & 1;
+                if (!tc::mbar_wait(bar.kv_full[slot], (k / kNS) & 1, abort, err, 4)) { ok = false; break; }
+                if (k >= 2 && !tc::mbar_wait(bar.s_free[sb], ((k - 2) >> 1) & 1, abort, err, 5)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t sK = base + kOffSlots + slot * kSlot;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t ad = tc::sw128_desc(sQ + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = tc::sw128_desc(sK + (kk >> 2) * kKVHalf + (kk & 3) * 32, 16, 1024);
+                    tc::mma_f16_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(bar.s_full[sb]);
+                if (k >= 1 && !issue_pv(k - 1)) { ok = false; break; }
+            }
+            if (ok) ok = issue_pv(njobs - 1);
+            if (!ok) {
+                // drain the MMAs already issued before TMEM is released
+                tc::mma_commit(bar.drain);
+                for (long long it = 0; it < (1ll << 22); ++it)
+                    if (tc::mbar_try(bar.drain, 0)) break;
+            }
+        }
+    } else {
+        // ---- softmax: one thread per row ---------------------------------------------------
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;
+        const int pl = row / G, h = row % G;
+        const int i = i0 + pl;
+        const bool valid = i < s.n;
+        const int diag = i / s.B;
+        const int* li = ridx + (valid ? tri_offset(i, s.B) : 0);
+        const float* lb = rbias + (valid ? tri_offset(i, s.B) : 0);
+        const int cnt = valid ? counts[i] : 0;
+        int cur = 0;
+        int nxt = cnt > 0 ? li[0] : INT_MAX;
+        float nbias = cnt > 0 ? lb[0] : 0.f;
+        const float scale2 = kLog2e * rsqrtf((float)kD);
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        char* prow = sm + kOffP + (row >> 3) * 1024 + (row & 7) * 128;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int k = 0; k < njobs; ++k) {
+            const int sb = k & 1;
+            // waits are made warp-uniform: the tcgen05 loads and stores below are .sync.aligned
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.s_full[sb], (k >> 1) & 1, abort, err, 6))) { ok = false; break; }
+            tc::fence_after_sync();
+            float v[64];
+            tc::tmem_ld32(lane_base + sb * 64, v);
+            tc::tmem_ld32(lane_base + sb * 64 + 32, v + 32);
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar.s_free[sb]);
+            const int c = jobs[k / NH];
+            const int j0 = c * s.B + (k % NH) * kKT;
+            float bias2 = -INFINITY;
+            int jmax = INT_MAX;
+            if (valid) {
+                if (nxt == c) bias2 = nbias * kLog2e;
+                else if (c == diag) { bias2 = 0.f; jmax = i; }
+            }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+                float x = v[e] * scale2 + bias2;
+                if (j0 + e > jmax) x = -INFINITY;
+                v[e] = x;
+                mt = fmaxf(mt, x);
+            }
+            const bool need = (m != -INFINITY) && (mt > m + 8.f);
+            if (m == -INFINITY) m = mt;
+            if (__any_sync(0xffffffffu, need)) {
+                // rescale O: wait until the previous P V has landed
+                if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort, err, 7))) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const float f = need ? exp2f(m - mt) : 1.f;
+                if (need) { l *= f; m = mt; }
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float o[32];
+                    tc::tmem_ld32(lane_base + 128 + cb * 32, o);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= f;
+                    tc::tmem_st32(lane_base + 128 + cb * 32, o);
+                }
+                tc::tmem_wait_st();
+            }
+            const float mref = m == -INFINITY ? 0.f : m;
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const float p0 = exp2f(v[2 * e] - mref), p1 = exp2f(v[2 * e + 1] - mref);
+                l += p0 + p1;
+                __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
+                pk[e] = *reinterpret_cast<uint32_t*>(&t2);
+            }
+            if (k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[sb], ((k - 2) >> 1) & 1, abort, err, 8))) {
+                ok = false;
+                break;
+            }
+            char* pdst = prow + sb * kPBytes;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(pdst + ((ch ^ (row & 7)) << 4)) =
+                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar.p_full[sb]);
+            if (k % NH == NH - 1 && nxt == c) {
+                ++cur;
+                nxt = cur < cnt ? li[cur] : INT_MAX;
+                nbias = cur < cnt ? lb[cur] : 0.f;
+            }
+        }
+        // ---- epilogue: O / l -> bf16 --------------------------------------------------------
+        if (ok && njobs > 0 &&
+            __all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[(njobs - 1) & 1], ((njobs - 1) >> 1) & 1, abort, err, 9))) {
+            tc::fence_after_sync();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = valid ? O + (long long)b * s.os[0] + (long long)i * s.os[1] +
+                                              (long long)(r * G + h) * s.os[2]
+                                        : nullptr;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                float o[32];
+                tc::tmem_ld32(lane_base + 128 + cb * 32, o);
+                tc::tmem_wait_ld();
+                if (orow) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 w4;
+                        __nv_bfloat162 a0 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
+                        __nv_bfloat162 a1 = __floats2bfloat162_rn(o[e + 2] * inv, o[e + 3] * inv);
+                        __nv_bfloat162 a2 = __floats2bfloat162_rn(o[e + 4] * inv, o[e + 5] * inv);
+                        __nv_bfloat162 a3 = __floats2bfloat162_rn(o[e + 6] * inv, o[e + 7] * inv);
+                        w4.x = *reinterpret_cast<uint32_t*>(&a0);
+                        w4.y = *reinterpret_cast<uint32_t*>(&a1);
+                        w4.z = *reinterpret_cast<uint32_t*>(&a2);
+                        w4.w = *reinterpret_cast<uint32_t*>(&a3);
+                        *reinterpret_cast<uint4*>(orow + cb * 32 + e) = w4;
+                    }
+                }
+            }
+        }
+    }
+    // ---- teardown -----------------------------------------------------------------------------
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 4-D map over a [batch, n, heads, 128] bf16 tensor (element strides st), box (64 d, bh heads,
+// bp positions, 1), 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* ptr, int batch, int n, int heads, const long long st[3], int bh,
+              int bp)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {128, (cuuint64_t)heads, (cuuint64_t)n, (cuuint64_t)batch};
+    cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
+    if (batch == 1) strides[2] = strides[1] * (cuuint64_t)n;   // unused dimension: any legal stride
+    cuuint32_t box[4] = {64, (cuuint32_t)bh, (cuuint32_t)bp, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult rc = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return rc == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attend_tc_supported(const Shape& s, int dtype)
+{
+    return dtype == DASH_BF16 && s.d == 128 && (s.B == 64 || s.B == 128) && s.g >= 1 && s.g <= 16 &&
+           (kRows % s.g) == 0 && encode_fn() != nullptr && (s.T + 2) * 4 <= 16 * 1024;
+}
+
+size_t attend_tc_smem(const Shape& s)
+{
+    return 1024 + kOffJobs + (size_t)(s.T + 2) * 4;
+}
+
+cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
+                                     const Routes& rt, int* err, cudaStream_t st)
+{
+    CUtensorMap mq, mk, mv;
+    const int P = kRows / s.g;
+    if (!make_map(&mq, Q, s.batch, s.n, s.hq, s.qs, s.g, P) || !make_map(&mk, K, s.batch, s.n, s.hkv, s.ks, 1, kKT) ||
+        !make_map(&mv, V, s.batch, s.n, s.hkv, s.vs, 1, kKT))
+        return cudaErrorInvalidValue;
+    const size_t smem = attend_tc_smem(s);
+    cudaError_t e = cudaFuncSetAttribute(attend_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long nblk = (s.n + P - 1) / P;
+    const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
+    if (grid == 0) return cudaSuccess;
+    attend_prefill_tc_kernel<<<grid, 192, smem, st>>>(mq, mk, mv, s, rt, (__nv_bfloat16*)O, err);
+    return cudaGetLastError();
+}
+
+}  // namespace dash

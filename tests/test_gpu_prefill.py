@@ -24,6 +24,7 @@ def run_prefill(x, *, chunk, alpha, gamma, inv_sigma=1.0, dtype="bf16", bitmask=
                    bitmask=bitmask)
     O = pf()
     torch.cuda.synchronize()
+    assert pf.error_word() == 0
     return O, pf
 
 
