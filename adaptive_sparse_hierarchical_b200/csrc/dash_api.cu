@@ -224,6 +224,7 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
     // the routing step keeps every head's logits of one (sequence, KV head) in shared memory
     if ((size_t)(p->h_q / p->h_kv) * (size_t)(p->seqlen / p->chunk) * 4 > 225 * 1024) return DASH_EUNSUPPORTED;
     const DecodeLayout L = decode_layout(p);
+    if (L.splits > 1024) return DASH_EUNSUPPORTED;   // the merge step holds at most 1024 split weights
     if (!workspace || ws_bytes < L.total) return DASH_EWORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DASH_EALIGN;
     const Shape s = make_shape(p);

@@ -261,36 +261,43 @@ __global__ void __launch_bounds__(32) dec_attend_mma_kernel(Shape s, const __nv_
     }
 }
 
-// Log-sum-exp merge of the split partials; one block per (sequence, KV head).
+// Log-sum-exp merge of the split partials; one block per (sequence, query head): the split
+// weights 2^(m_k - M) / L are computed once into shared memory, then each thread merges one
+// output column.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) dec_combine_kernel(Shape s, const float* __restrict__ part, int splits,
                                                           Routes rt, T* __restrict__ O)
 {
-    __shared__ float sm[16], sinv[16];
-    const int br = blockIdx.x, b = br / s.hkv, r = br % s.hkv, G = s.g;
-    const int nsp = (rt.counts[br] + 1 + kDecCPS - 1) / kDecCPS;
-    const float* base = part + (long long)br * splits * G * (D + 2);
-    if (threadIdx.x < G) {
-        const int row = threadIdx.x;
-        float M = -INFINITY;
-        for (int k = 0; k < nsp; ++k) M = fmaxf(M, base[((long long)k * G + row) * (D + 2) + D]);
-        float Lsum = 0.f;
-        for (int k = 0; k < nsp; ++k) {
-            const float* pr = base + ((long long)k * G + row) * (D + 2);
-            Lsum += pr[D + 1] * exp2f(pr[D] - M);
-        }
-        sm[row] = M;
-        sinv[row] = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    }
+    __shared__ float wk[1024];
+    __shared__ float red[4];
+    const int br = blockIdx.x / s.g, row = blockIdx.x % s.g, G = s.g;
+    const int b = br / s.hkv, r = br % s.hkv;
+    const int nsp = min((rt.counts[br] + 1 + kDecCPS - 1) / kDecCPS, 1024);
+    const float* base = part + (long long)br * splits * G * (D + 2) + (long long)row * (D + 2);
+    const long long sstride = (long long)G * (D + 2);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float M = -INFINITY;
+    for (int k = tid; k < nsp; k += blockDim.x) M = fmaxf(M, base[k * sstride + D]);
+    M = warp_max(M);
+    if (lane == 0) red[warp] = M;
     __syncthreads();
-    for (int v = threadIdx.x; v < G * D; v += blockDim.x) {
-        const int row = v / D, col = v % D;
+    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    float Lsum = 0.f;
+    for (int k = tid; k < nsp; k += blockDim.x) {
+        const float w = exp2f(base[k * sstride + D] - M);
+        wk[k] = w;
+        Lsum += base[k * sstride + D + 1] * w;
+    }
+    Lsum = warp_sum(Lsum);
+    if (lane == 0) red[warp] = Lsum;
+    __syncthreads();
+    Lsum = red[0] + red[1] + red[2] + red[3];
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    for (int col = tid; col < D; col += blockDim.x) {
         float o = 0.f;
-        for (int k = 0; k < nsp; ++k) {
-            const float* pr = base + ((long long)k * G + row) * (D + 2);
-            o += pr[col] * exp2f(pr[D] - sm[row]);
-        }
-        O[((long long)b * s.hq + r * G + row) * D + col] = from_f<T>(o * sinv[row]);
+        for (int k = 0; k < nsp; ++k) o += base[k * sstride + col] * wk[k];
+        O[((long long)b * s.hq + r * G + row) * D + col] = from_f<T>(o * inv);
     }
 }
 
@@ -416,8 +423,8 @@ cudaError_t dec_mma_t(const Shape& s, const void* q, const void* Kc, const void*
     dim3 grid(ws.splits, s.batch * s.hkv);
     k<<<grid, 32, smem, st>>>(s, (const __nv_bfloat16*)q, (const __nv_bfloat16*)Kc, (const __nv_bfloat16*)Vc,
                               seqlens, rt, ws.part, ws.splits);
-    dec_combine_kernel<__nv_bfloat16, D><<<s.batch * s.hkv, 128, 0, st>>>(s, ws.part, ws.splits, rt,
-                                                                           (__nv_bfloat16*)O);
+    dec_combine_kernel<__nv_bfloat16, D><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, ws.part, ws.splits, rt,
+                                                                                 (__nv_bfloat16*)O);
     return cudaGetLastError();
 }
 
