@@ -138,6 +138,23 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
                 const float* kbar_cache, const int* seqlens, void* O, const dash_route_out* route,
                 void* workspace, size_t ws_bytes, void* stream);
 
+/* dash_decode without a workspace, for callers that cannot obtain device memory of their own
+ * (for example a plugin inside a runtime that owns every device allocation and gives it no
+ * allocator, or a service that must not grow its device footprint once running).  The paper has
+ * no counterpart; this is a deployment variant of dash_decode with the same arguments minus
+ * route/workspace, and the same results.
+ *   Scratch: a fixed 16 MiB device array inside the library (one per GPU that loads it, held
+ *   until the process exits).  A request whose scratch (per-head logits, route lists, split
+ *   partials) exceeds 16 MiB returns DASH_EWORKSPACE before anything is enqueued.
+ *   The array is shared by every call on a GPU and keeps the last call's contents (each call
+ *   writes every scratch value before reading it): calls whose kernels overlap on the GPU race
+ *   and must be serialised by the caller.
+ *   The first call on each device looks up the array's device address with that device current
+ *   and caches it; make that first call before any stream capture.
+ *   Allocates nothing (no cudaMalloc / cudaFree / allocating library routine). */
+int dash_decode_noalloc(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
+                        const float* kbar_cache, const int* seqlens, void* O, void* stream);
+
 /* Static text for a status code. */
 const char* dash_status_string(int status);
 
