@@ -77,7 +77,7 @@ PrefillLayout prefill_layout(const dash_params* p)
     return L;
 }
 
-struct DecodeLayout { size_t x, part, counts, idx, bias, total; int splits; };
+struct DecodeLayout { size_t x, part, counts, idx, bias, err, total; int splits; };
 DecodeLayout decode_layout(const dash_params* p)
 {
     DecodeLayout L;
@@ -90,7 +90,8 @@ DecodeLayout decode_layout(const dash_params* p)
     L.counts = L.part + up(bh * (size_t)L.splits * s.g * (p->d_h + 2) * 4);
     L.idx = L.counts + up(bh * 4);
     L.bias = L.idx + up(bh * (T > 0 ? T : 1) * 4);
-    L.total = L.bias + up(bh * (T > 0 ? T : 1) * 4);
+    L.err = L.bias + up(bh * (T > 0 ? T : 1) * 4);
+    L.total = L.err + kAlign;
     return L;
 }
 
@@ -110,8 +111,10 @@ size_t dash_workspace_size(const dash_params* p, int op)
 
 long long dash_error_word_offset(const dash_params* p, int op)
 {
-    if (check_params(p) != DASH_OK || op != DASH_OP_PREFILL) return -1;
-    return (long long)prefill_layout(p).err;
+    if (check_params(p) != DASH_OK) return -1;
+    if (op == DASH_OP_PREFILL) return (long long)prefill_layout(p).err;
+    if (op == DASH_OP_DECODE) return (long long)decode_layout(p).err;
+    return -1;
 }
 
 long long dash_route_capacity(const dash_params* p)
@@ -240,6 +243,8 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
     dw.x = reinterpret_cast<float*>(ws + L.x);
     dw.part = reinterpret_cast<float*>(ws + L.part);
     dw.splits = L.splits;
+    dw.err = reinterpret_cast<int*>(ws + L.err);
+    if (cudaMemsetAsync(dw.err, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess) return DASH_ELAUNCH;
     return launch_status(launch_decode(s, p->dtype, q, K_cache, V_cache, kbar_cache, s.T, seqlens, O, rt, dw,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -69,7 +69,7 @@ extern "C" int dash_decode_noalloc(const dash_params* p, const void* q, const vo
     const size_t off_counts = off_part + upna(bh * splits * g * ((size_t)p->d_h + 2) * 4);
     const size_t off_idx = off_counts + upna(bh * 4);
     const size_t off_bias = off_idx + upna(bh * Tn * 4);
-    const size_t total = off_bias + upna(bh * Tn * 4);
+    const size_t total = off_bias + upna(bh * Tn * 4) + kAlignNA;   // + status word
     if (total > kNoAllocScratchBytes) return DASH_EWORKSPACE;
     void* scratch = scratch_for_current_device();
     if (!scratch) return DASH_ELAUNCH;

@@ -266,13 +266,13 @@ __global__ void __launch_bounds__(32) dec_attend_mma_kernel(Shape s, const __nv_
 // output column.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) dec_combine_kernel(Shape s, const float* __restrict__ part, int splits,
-                                                          Routes rt, T* __restrict__ O)
+                                                          int cps, Routes rt, T* __restrict__ O)
 {
     __shared__ float wk[1024];
     __shared__ float red[4];
     const int br = blockIdx.x / s.g, row = blockIdx.x % s.g, G = s.g;
     const int b = br / s.hkv, r = br % s.hkv;
-    const int nsp = min((rt.counts[br] + 1 + kDecCPS - 1) / kDecCPS, 1024);
+    const int nsp = min((rt.counts[br] + 1 + cps - 1) / cps, 1024);
     const float* base = part + (long long)br * splits * G * (D + 2) + (long long)row * (D + 2);
     const long long sstride = (long long)G * (D + 2);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -423,8 +423,8 @@ cudaError_t dec_mma_t(const Shape& s, const void* q, const void* Kc, const void*
     dim3 grid(ws.splits, s.batch * s.hkv);
     k<<<grid, 32, smem, st>>>(s, (const __nv_bfloat16*)q, (const __nv_bfloat16*)Kc, (const __nv_bfloat16*)Vc,
                               seqlens, rt, ws.part, ws.splits);
-    dec_combine_kernel<__nv_bfloat16, D><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, ws.part, ws.splits, rt,
-                                                                                 (__nv_bfloat16*)O);
+    dec_combine_kernel<__nv_bfloat16, D><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, ws.part, ws.splits, kDecCPS,
+                                                                                 rt, (__nv_bfloat16*)O);
     return cudaGetLastError();
 }
 
@@ -485,6 +485,15 @@ cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* 
 {
     cudaError_t e = launch_route_decode(s, dtype, q, kbar, kbar_T, seqlens, rt, ws.x, st);
     if (e != cudaSuccess) return e;
+    if (dec_tma_supported(s, dtype) && !legacy_stage2()) {
+        const int splits = dec_tma_splits(s, kbar_T);
+        e = launch_dec_attend_tma(s, q, Kc, Vc, seqlens, rt, ws.part, splits, ws.err, st);
+        if (e != cudaSuccess) return e;
+        dec_combine_kernel<__nv_bfloat16, 128><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, ws.part, splits,
+                                                                                      dec_tma_cps(), rt,
+                                                                                      (__nv_bfloat16*)O);
+        return cudaGetLastError();
+    }
     if (dtype == DASH_BF16)
         return s.d == 128 ? dec_bf16_d<128>(s, q, Kc, Vc, seqlens, rt, ws, O, st)
                           : dec_bf16_d<64>(s, q, Kc, Vc, seqlens, rt, ws, O, st);

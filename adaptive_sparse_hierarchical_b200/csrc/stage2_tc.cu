@@ -19,6 +19,7 @@
 //               is kept (values stay <= 2^8, exact in the final normalisation).
 // Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
 #include <climits>
+#include <cstdlib>
 #include <cudaTypedefs.h>
 
 #include "dash_common.cuh"
@@ -27,20 +28,29 @@
 namespace dash {
 namespace {
 
-constexpr int kRows = 128, kKT = 64, kD = 128, kNS = 4;
+constexpr int kRows = 128, kKT = 64, kD = 128, kNS = 2;
 constexpr int kQBytes = kRows * kD * 2;           // 32 KB, two 16 KB d-halves
 constexpr int kKVHalf = kKT * 64 * 2;             // 8 KB: [64 keys][64 d]
 constexpr int kSlot = 4 * kKVHalf;                // K (2 halves) + V (2 halves) = 32 KB
-constexpr int kPBytes = kRows * kKT * 2;          // 16 KB
-constexpr int kTmemCols = 256;                    // S0 [0,64), S1 [64,128), O [128,256)
-constexpr int kOffQ = 0, kOffSlots = kQBytes, kOffP = kOffSlots + kNS * kSlot;
-constexpr int kOffBar = kOffP + 2 * kPBytes;      // 196608
+constexpr int kTmemCols = 256;                    // S0 [0,64), S1 [64,128), O [128,256); P_k over S_k
+constexpr int kOffQ = 0, kOffSlots = kQBytes;
+constexpr int kOffScratch = kOffSlots;            // set-up scratch (chunk bitmask, sort keys) in the ring
+constexpr int kOffBar = kOffSlots + kNS * kSlot;  // 98304: two blocks fit on one SM
 constexpr int kNumBars = 1 + 2 * kNS + 2 + 2 + 2 + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, njobs
-constexpr int kOffJobs = kOffMisc + 32;
+constexpr int kOffPos = kOffMisc + 32;             // the block's positions (<= 16 when clustered)
+constexpr int kOffJobs = kOffPos + 4 * kRows;
 
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = tc::idesc_bf16(128, 128, false, true);
+
+// 2^x on the special-function unit (flush-to-zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 struct Bars {
     uint32_t q_full, kv_full[kNS], kv_empty[kNS], s_full[2], s_free[2], p_full[2], pv_done[2], drain;
@@ -61,11 +71,13 @@ __device__ __forceinline__ Bars make_bars(uint32_t base)
     return b;
 }
 
-__global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                   const __grid_constant__ CUtensorMap tmQ1,
                                                                    const __grid_constant__ CUtensorMap tmK,
                                                                    const __grid_constant__ CUtensorMap tmV,
                                                                    Shape s, Routes rt,
-                                                                   __nv_bfloat16* __restrict__ O, int* err)
+                                                                   __nv_bfloat16* __restrict__ O, int* err,
+                                                                   int cluster)
 {
     extern __shared__ char smem_raw[];
     char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -75,7 +87,8 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
     volatile int* abort = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
     int* njobs_s = reinterpret_cast<int*>(sm + kOffMisc + 8);
     int* jobs = reinterpret_cast<int*>(sm + kOffJobs);
-    uint32_t* umask = reinterpret_cast<uint32_t*>(sm + kOffP);   // scratch until P is used
+    int* spos = reinterpret_cast<int*>(sm + kOffPos);
+    uint32_t* umask = reinterpret_cast<uint32_t*>(sm + kOffScratch);   // scratch until the first TMA
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = s.g, P = kRows / G;
@@ -109,10 +122,30 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
         tc::tmem_alloc(tc::smem_addr(tmem_slot), kTmemCols);
     }
     for (int w = tid; w < W; w += blockDim.x) umask[w] = 0u;
+    if (cluster) {
+        // Rows of one tile share its union of routed chunks.  The window of 8 consecutive tiles
+        // is re-grouped by routed-chunk count (a stable order), so positions with small routes
+        // (here: queries matching the planted chunks) share tiles with small unions.
+        int* key = reinterpret_cast<int*>(sm + kOffScratch + 16384);
+        const int Wn = 8 * P, w0 = (pb / 8) * Wn, t8 = pb % 8;
+        for (int j = tid; j < Wn; j += blockDim.x) {
+            const int ii = w0 + j;
+            key[j] = ii < s.n ? ((counts[ii] << 8) | j) : INT_MAX - Wn + j;
+        }
+        __syncthreads();
+        for (int j = tid; j < Wn; j += blockDim.x) {
+            const int kj = key[j];
+            int rank = 0;
+            for (int q = 0; q < Wn; ++q) rank += key[q] < kj;
+            if (rank / P == t8) spos[rank % P] = w0 + j;
+        }
+    } else {
+        for (int p = tid; p < P; p += blockDim.x) spos[p] = i0 + p;
+    }
     __syncthreads();
     for (int p = 0; p < P; ++p) {
-        const int i = i0 + p;
-        if (i >= s.n) break;
+        const int i = spos[p];
+        if (i >= s.n) continue;
         const int cnt = counts[i];
         const int* li = ridx + tri_offset(i, s.B);
         for (int k = tid; k < cnt; k += blockDim.x) atomicOr(&umask[li[k] >> 5], 1u << (li[k] & 31));
@@ -154,8 +187,17 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
             tc::prefetch_tmap(&tmK);
             tc::prefetch_tmap(&tmV);
             tc::mbar_expect_tx(bar.q_full, kQBytes);
-            tc::tma_load_4d(base + kOffQ, &tmQ, bar.q_full, 0, r * G, i0, b);
-            tc::tma_load_4d(base + kOffQ + kQBytes / 2, &tmQ, bar.q_full, 64, r * G, i0, b);
+            if (cluster) {
+                // one box of g rows per position (g = 8 or 16 keeps every box 1024-byte aligned)
+                tc::prefetch_tmap(&tmQ1);
+                for (int p = 0; p < P; ++p) {
+                    tc::tma_load_4d(base + kOffQ + p * G * 128, &tmQ1, bar.q_full, 0, r * G, spos[p], b);
+                    tc::tma_load_4d(base + kOffQ + kQBytes / 2 + p * G * 128, &tmQ1, bar.q_full, 64, r * G, spos[p], b);
+                }
+            } else {
+                tc::tma_load_4d(base + kOffQ, &tmQ, bar.q_full, 0, r * G, i0, b);
+                tc::tma_load_4d(base + kOffQ + kQBytes / 2, &tmQ, bar.q_full, 64, r * G, i0, b);
+            }
             int last[kNS];
             for (int k = 0; k < kNS; ++k) last[k] = -1;
             for (int k = 0; k < njobs; ++k) {
@@ -183,7 +225,7 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
     } else if (warp == 1) {
         // ---- MMA issuer --------------------------------------------------------------------
         if (lane == 0 && njobs > 0) {
-            const uint32_t sQ = base + kOffQ, sP = base + kOffP;
+            const uint32_t sQ = base + kOffQ;
             auto issue_pv = [&](int j) -> bool {
                 const int pbuf = j & 1;
                 if (!tc::mbar_wait(bar.p_full[pbuf], (j >> 1) & 1, abort, err, 2)) return false;
@@ -191,9 +233,9 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
                 const uint32_t sV = base + kOffSlots + (j % kNS) * kSlot + 2 * kKVHalf;
 #pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk) {
-                    const uint64_t ad = tc::sw128_desc(sP + pbuf * kPBytes + kk * 32, 16, 1024);
+                    // P_j (bf16, 2 per column) sits in the first 32 columns of S buffer pbuf
                     const uint64_t bd = tc::sw128_desc(sV + kk * 2048, kKVHalf, 1024);
-                    tc::mma_f16_ss(tmem + 128, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_f16_ts(tmem + 128, tmem + pbuf * 64 + kk * 8, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(bar.kv_empty[j % kNS]);
                 tc::mma_commit(bar.pv_done[pbuf]);
@@ -228,7 +270,7 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int pl = row / G, h = row % G;
-        const int i = i0 + pl;
+        const int i = spos[pl];
         const bool valid = i < s.n;
         const int diag = i / s.B;
         const int* li = ridx + (valid ? tri_offset(i, s.B) : 0);
@@ -239,7 +281,6 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
         float nbias = cnt > 0 ? lb[0] : 0.f;
         const float scale2 = kLog2e * rsqrtf((float)kD);
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-        char* prow = sm + kOffP + (row >> 3) * 1024 + (row & 7) * 128;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int k = 0; k < njobs; ++k) {
@@ -256,19 +297,28 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
             const int c = jobs[k / NH];
             const int j0 = c * s.B + (k % NH) * kKT;
             float bias2 = -INFINITY;
-            int jmax = INT_MAX;
+            bool causal = false;
             if (valid) {
                 if (nxt == c) bias2 = nbias * kLog2e;
-                else if (c == diag) { bias2 = 0.f; jmax = i; }
+                else if (c == diag) { bias2 = 0.f; causal = j0 + kKT - 1 > i; }
             }
-            float mt = -INFINITY;
+            if (causal) {
+                // diagonal tile: keys past the query are masked
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                float x = v[e] * scale2 + bias2;
-                if (j0 + e > jmax) x = -INFINITY;
-                v[e] = x;
-                mt = fmaxf(mt, x);
+                for (int e = 0; e < 64; ++e)
+                    if (j0 + e > i) v[e] = -INFINITY;
             }
+            // tile maximum of the biased logits: max over raw scores (tree), then scale (scale2 > 0)
+            float mx8[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(v[a], v[a + 8]);
+#pragma unroll
+            for (int e = 16; e < 64; e += 8)
+#pragma unroll
+                for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], v[e + a]);
+            const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float mt = bias2 == -INFINITY ? -INFINITY : fmaf(smax, scale2, bias2);
             const bool need = (m != -INFINITY) && (mt > m + 8.f);
             if (m == -INFINITY) m = mt;
             if (__any_sync(0xffffffffu, need)) {
@@ -278,7 +328,7 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
                     break;
                 }
                 tc::fence_after_sync();
-                const float f = need ? exp2f(m - mt) : 1.f;
+                const float f = need ? ex2_approx(m - mt) : 1.f;
                 if (need) { l *= f; m = mt; }
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
@@ -289,27 +339,36 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
                     for (int e = 0; e < 32; ++e) o[e] *= f;
                     tc::tmem_st32(lane_base + 128 + cb * 32, o);
                 }
-                tc::tmem_wait_st();
             }
-            const float mref = m == -INFINITY ? 0.f : m;
-            uint32_t pk[32];
+            // p = 2^(s*scale2 + bias2 - m): one FMA and one ex2 per element; P (bf16 pairs) goes to
+            // the first 32 columns of this job's S buffer.  A warp whose rows all skip the tile
+            // writes zeros without computing.
+            const uint32_t pdst = lane_base + sb * 64;
+            if (__all_sync(0xffffffffu, bias2 == -INFINITY)) {
+                uint32_t z[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const float p0 = exp2f(v[2 * e] - mref), p1 = exp2f(v[2 * e + 1] - mref);
-                l += p0 + p1;
-                __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
-                pk[e] = *reinterpret_cast<uint32_t*>(&t2);
-            }
-            if (k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[sb], ((k - 2) >> 1) & 1, abort, err, 8))) {
-                ok = false;
-                break;
-            }
-            char* pdst = prow + sb * kPBytes;
+                for (int e = 0; e < 16; ++e) z[e] = 0u;
+                tc::tmem_st16(pdst, z);
+                tc::tmem_st16(pdst + 16, z);
+            } else {
+                const float off = bias2 - (m == -INFINITY ? 0.f : m);
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(pdst + ((ch ^ (row & 7)) << 4)) =
-                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            tc::fence_proxy_async_smem();
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2_approx(fmaf(v[32 * half + 2 * e], scale2, off));
+                        const float p1 = ex2_approx(fmaf(v[32 * half + 2 * e + 1], scale2, off));
+                        ls[e & 3] += p0 + p1;
+                        __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
+                        pk[e] = *reinterpret_cast<uint32_t*>(&t2);
+                    }
+                    tc::tmem_st16(pdst + 16 * half, pk);
+                }
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            }
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(bar.p_full[sb]);
             if (k % NH == NH - 1 && nxt == c) {
@@ -357,6 +416,17 @@ __global__ void __launch_bounds__(192, 1) attend_prefill_tc_kernel(const __grid_
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+bool cluster_disabled()
+{
+    // DASH_CLUSTER=0 keeps positions in sequence order inside each tile (comparison runs)
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("DASH_CLUSTER");
+        v = (e && e[0] == '0') ? 1 : 0;
+    }
+    return v == 1;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -407,10 +477,11 @@ size_t attend_tc_smem(const Shape& s)
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
                                      const Routes& rt, int* err, cudaStream_t st)
 {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mq1, mk, mv;
     const int P = kRows / s.g;
-    if (!make_map(&mq, Q, s.batch, s.n, s.hq, s.qs, s.g, P) || !make_map(&mk, K, s.batch, s.n, s.hkv, s.ks, 1, kKT) ||
-        !make_map(&mv, V, s.batch, s.n, s.hkv, s.vs, 1, kKT))
+    const int cluster = (s.g == 8 || s.g == 16) && !cluster_disabled() ? 1 : 0;
+    if (!make_map(&mq, Q, s.batch, s.n, s.hq, s.qs, s.g, P) || !make_map(&mq1, Q, s.batch, s.n, s.hq, s.qs, s.g, 1) ||
+        !make_map(&mk, K, s.batch, s.n, s.hkv, s.ks, 1, kKT) || !make_map(&mv, V, s.batch, s.n, s.hkv, s.vs, 1, kKT))
         return cudaErrorInvalidValue;
     const size_t smem = attend_tc_smem(s);
     cudaError_t e = cudaFuncSetAttribute(attend_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -418,7 +489,7 @@ cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* 
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    attend_prefill_tc_kernel<<<grid, 192, smem, st>>>(mq, mk, mv, s, rt, (__nv_bfloat16*)O, err);
+    attend_prefill_tc_kernel<<<grid, 192, smem, st>>>(mq, mq1, mk, mv, s, rt, (__nv_bfloat16*)O, err, cluster);
     return cudaGetLastError();
 }
 

@@ -48,7 +48,7 @@ def args_():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--cpu-rows", type=int, default=16384)
     return ap.parse_args()
 
 
@@ -201,7 +201,8 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind):
         "ms_per_step": ms, "value": ranks.world * tokens / (ms / 1e3) / 1e6,
         "stages_ms": {"stage0_summary": stage_ms[0], "stage1_route": stage_ms[1], "stage2_attend": stage_ms[2]},
         "routed_fraction": float(counts.sum()) / (wl.batch * wl.h_kv * sum(i // wl.chunk for i in range(wl.n))),
-        "roofline": {"kernel": "stage2 attend_prefill_mma_kernel", "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": ("attend_prefill_mma_kernel (mma.sync)" if os.environ.get("DASH_STAGE2", "").startswith("m")
+                               else "attend_prefill_tc_kernel (tcgen05)"), "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                      "peak_kind": f"bf16 dense burst, of {pk_kind}",
                      "flops_per_launch": flops, "launch_ms": stage_ms[2]},
@@ -303,7 +304,7 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
     achieved = bps / (statistics.mean(dec_ms) / 1e3) / 1e9
     res = {"workload": "decode_128k: b=8, 131072-token caches (+1 per step), 32/2 heads, d=128, B=64, alpha 1.5, "
                        f"gamma {wl.gamma} (~25% routed)",
-           "us_per_step": ms * 1e3, "us_per_token": ms * 1e3 / (wl.batch * ranks.world) * ranks.world / ranks.world,
+           "us_per_step": ms * 1e3,
            "steps": nst, "append_us": statistics.mean(a.elapsed_time(b) for a, b, c in evs) * 1e3,
            "decode_us": statistics.mean(dec_ms) * 1e3,
            "routed_fraction": float(routed[-1][1].sum()) / (wl.batch * wl.h_kv * ((prefix + routed[-1][0]) // wl.chunk)),
@@ -312,7 +313,7 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
                         "peak_kind": f"hbm copy, of {pk_kind}", "bytes_per_step": bps},
            "clocks": clk.summary(), "gpu_launches": 6 * nst,
            "l2": "KV caches (1.07 GB) larger than L2"}
-    res["us_per_token"] = res["us_per_step"] / wl.batch
+    res["us_per_token"] = res["us_per_step"] / wl.batch   # per sequence-token, one GPU
     return res
 
 

@@ -126,3 +126,32 @@ def test_decode_128k_full_size_sampled():
             print("decode_128k step", s, stt)
     frac = st.rt[0].sum().item() / (wl.batch * 2 * ((prefix + 31) // 64))
     assert 0.15 < frac < 0.35, frac
+
+
+def test_decode_long_run_is_deterministic():
+    """300 append+decode steps, run twice from the same saved state: the outputs must agree bit for
+    bit at every step (a race between the producer and consumer warps of a K/V ring would show up
+    here), and the last step must match the oracle.  Saving / restoring the caller-owned tensors is
+    also how a decode session is checkpointed."""
+    b, cap, hq, hkv, d, B = 4, 4096, 16, 2, 128, 64
+    x = inputs.planted(23, b, cap, hq, hkv, d, B, dtype="bf16", chunk_frac=0.1)
+    lengths = np.array([3000, 2500, 1999, 3300])
+    st = _state(x, lengths, cap, chunk=B, alpha=1.5, gamma=5.0, dtype="bf16")
+    saved = [t.clone() for t in (st.K, st.V, st.kbar, st.state, st.seqlens)]
+    dev = {k: torch.from_numpy(x[k]).to("cuda", torch.bfloat16) for k in ("Q", "K", "V")}
+    runs = []
+    for rep in range(2):
+        for t, sv in zip((st.K, st.V, st.kbar, st.state, st.seqlens), saved):
+            t.copy_(sv)
+        outs = []
+        for step in range(300):
+            pos = torch.from_numpy(lengths + step).long().cuda()
+            rows = torch.arange(b, device="cuda")
+            o = st.step(dev["Q"][rows, pos].contiguous(), dev["K"][rows, pos].contiguous(),
+                        dev["V"][rows, pos].contiguous())
+            outs.append(o.clone())
+        torch.cuda.synchronize()
+        runs.append(torch.stack(outs))
+    assert torch.equal(runs[0], runs[1])
+    last = lengths + 300
+    _check_step(st, x, x["Q"][np.arange(b), last - 1], last, chunk=B, alpha=1.5, gamma=5.0, dtype="bf16")

@@ -143,6 +143,11 @@ def test_prefill_32k_full_size_sampled():
     O, pf = run_prefill(x, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma)
     pos = _sample_positions(wl.n, wl.chunk, 192, 0)
     st = compare(x, pf, O, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, positions=pos)
+    # a second launch on the same buffers must reproduce the output bit for bit
+    O1 = O.clone()
+    pf()
+    torch.cuda.synchronize()
+    assert torch.equal(O1, pf.O) and pf.error_word() == 0
     frac = pf.counts.sum().item() / (2 * sum(i // 64 for i in range(wl.n)))
     assert 0.2 < frac < 0.3, frac
     print("prefill_32k", st, "routed fraction", frac)
