@@ -20,17 +20,15 @@ import numpy as np
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    """Round finite float32 values to the nearest bf16 (ties to even); returns float32."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    u = (u + 0x7FFF + lsb) >> 16 << 16
-    out = (u & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
-    nan = np.isnan(a)
-    if nan.any():
-        out = out.copy()
-        out[nan] = np.nan
-    return out
+    try:   # torch's float32 -> bf16 conversion rounds to nearest even, multi-threaded
+        import torch
+        return torch.from_numpy(a).to(torch.bfloat16).to(torch.float32).numpy()
+    except ImportError:  # pragma: no cover
+        u = a.view(np.uint32)
+        r = (u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) & np.uint32(0xFFFF0000)
+        return r.view(np.float32)
 
 
 def _streams(seed: int, k: int):
@@ -40,6 +38,23 @@ def _streams(seed: int, k: int):
 def _finish(a: np.ndarray, dtype: str) -> np.ndarray:
     a = a.astype(np.float32)
     return round_bf16(a) if dtype == "bf16" else a
+
+
+def _draw(rng, shape, dtype, scale=1.0, add=None, block=4096):
+    """Standard normals of `shape` = [b, n, ...] drawn in C order, position block by position block
+    (consecutive draws continue one stream, so the values equal a single draw), times `scale`,
+    plus add(b, n0, n1, block) applied in float64, then rounded to float32 (and bf16)."""
+    out = np.empty(shape, dtype=np.float32)
+    for b in range(shape[0]):
+        for n0 in range(0, shape[1], block):
+            n1 = min(n0 + block, shape[1])
+            x = rng.standard_normal((n1 - n0,) + tuple(shape[2:]))
+            if scale != 1.0:
+                x *= scale
+            if add is not None:
+                add(b, n0, n1, x)
+            out[b, n0:n1] = round_bf16(x.astype(np.float32)) if dtype == "bf16" else x
+    return out
 
 
 def _unit(rng, hkv, d):
@@ -59,23 +74,37 @@ def planted(seed: int, batch: int, n: int, h_q: int, h_kv: int, d: int, chunk: i
     g = h_q // h_kv
     T = n // chunk
     nrow = n if q_rows is None else int(q_rows[1])
-    Q = rq.standard_normal((batch, nrow, h_q, d))
-    K = rk.standard_normal((batch, n, h_kv, d))
-    V = rv.standard_normal((batch, n, h_kv, d))
-    qbar = rb.standard_normal((h_kv, d)) * qbar_std
-    u = _unit(ru, h_kv, d)
     nc = int(round(chunk_frac * T))
     nq = int(round(query_frac * nrow))
+    # the planted sets, drawn in the recipe's order: per (sequence, KV head) chunks, then rows
+    kplant = np.zeros((batch, h_kv, max(T, 1)), dtype=bool)
+    qplant = np.zeros((batch, h_kv, nrow), dtype=bool)
     for b in range(batch):
         for r in range(h_kv):
             if nc > 0:
-                for c in rp.choice(T, nc, replace=False):
-                    K[b, c * chunk:(c + 1) * chunk, r] += strength * u[r]
+                kplant[b, r, rp.choice(T, nc, replace=False)] = True
             if nq > 0:
-                pos = rp.choice(nrow, nq, replace=False)
-                Q[b, pos, r * g:(r + 1) * g] += strength * u[r]
-    return {"Q": _finish(Q, dtype), "K": _finish(K, dtype), "V": _finish(V, dtype),
-            "qbar": qbar.astype(np.float32)}
+                qplant[b, r, rp.choice(nrow, nq, replace=False)] = True
+    # the draws of qbar and u come from their own streams, so their order does not matter
+    qbar = rb.standard_normal((h_kv, d)) * qbar_std
+    u = _unit(ru, h_kv, d)
+
+    def add_q(b, n0, n1, x):
+        for r in range(h_kv):
+            rows = np.nonzero(qplant[b, r, n0:n1])[0]
+            x[rows, r * g:(r + 1) * g] += strength * u[r]
+
+    def add_k(b, n0, n1, x):
+        pos = np.arange(n0, n1)
+        c = pos // chunk
+        for r in range(h_kv):
+            sel = (c < T) & kplant[b, r, np.minimum(c, max(T, 1) - 1)]
+            x[sel, r] += strength * u[r]
+
+    Q = _draw(rq, (batch, nrow, h_q, d), dtype, add=add_q)
+    K = _draw(rk, (batch, n, h_kv, d), dtype, add=add_k)
+    V = _draw(rv, (batch, n, h_kv, d), dtype)
+    return {"Q": Q, "K": K, "V": V, "qbar": qbar.astype(np.float32)}
 
 
 def tiny(seed: int = 0, *, n: int = 512, h_q: int = 4, h_kv: int = 1, d: int = 64,
@@ -107,15 +136,24 @@ def mixture(seed: int, batch: int, n: int, h_q: int, h_kv: int, d: int, *, compo
     g = h_q // h_kv
     cen = rc.standard_normal((h_kv, components, d))
     nseg = (n + segment - 1) // segment
-    K = rk.standard_normal((batch, n, h_kv, d)) * spread
-    Q = rq.standard_normal((batch, n, h_q, d)) * spread
+    comp = np.zeros((batch, h_kv, nseg), dtype=np.int64)
+    qc = np.zeros((batch, h_kv, n), dtype=np.int64)
     for b in range(batch):
         for r in range(h_kv):
-            comp = ra.integers(0, components, nseg)
-            K[b, :, r] += np.repeat(cen[r, comp], segment, axis=0)[:n]
-            qc = ra.integers(0, components, n)
-            Q[b, :, r * g:(r + 1) * g] += cen[r, qc][:, None, :]
-    V = rv.standard_normal((batch, n, h_kv, d))
+            comp[b, r] = ra.integers(0, components, nseg)
+            qc[b, r] = ra.integers(0, components, n)
+
+    def add_k(b, n0, n1, x):
+        seg = np.arange(n0, n1) // segment
+        for r in range(h_kv):
+            x[:, r] += cen[r, comp[b, r, seg]]
+
+    def add_q(b, n0, n1, x):
+        for r in range(h_kv):
+            x[:, r * g:(r + 1) * g] += cen[r, qc[b, r, n0:n1]][:, None, :]
+
+    K = _draw(rk, (batch, n, h_kv, d), dtype, scale=spread, add=add_k)
+    Q = _draw(rq, (batch, n, h_q, d), dtype, scale=spread, add=add_q)
+    V = _draw(rv, (batch, n, h_kv, d), dtype)
     qbar = rb.standard_normal((h_kv, d)) * qbar_std
-    return {"Q": _finish(Q, dtype), "K": _finish(K, dtype), "V": _finish(V, dtype),
-            "qbar": qbar.astype(np.float32)}
+    return {"Q": Q, "K": K, "V": V, "qbar": qbar.astype(np.float32)}

@@ -151,3 +151,40 @@ def test_prefill_32k_full_size_sampled():
     frac = pf.counts.sum().item() / (2 * sum(i // 64 for i in range(wl.n)))
     assert 0.2 < frac < 0.3, frac
     print("prefill_32k", st, "routed fraction", frac)
+
+
+_SWEEP_X = {}
+
+
+@pytest.mark.parametrize("name", W.PREFILL_64K)
+def test_prefill_64k_full_size_sampled(name):
+    """8B-class layer shape at full size (b=2, n=65536, 32/2 heads, B=128) at 50 / 25 / 12.5% routed;
+    outputs checked on sampled rows of both sequences."""
+    wl = W.get(name)
+    if "x64" not in _SWEEP_X:
+        _SWEEP_X["x64"] = wl.make()   # the three sparsity levels share the inputs (only gamma differs)
+    x = _SWEEP_X["x64"]
+    O, pf = run_prefill(x, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma)
+    pos = _sample_positions(wl.n, wl.chunk, 96, 1)
+    st = compare(x, pf, O, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, positions=pos)
+    frac = pf.counts.sum().item() / (wl.batch * 2 * sum(i // wl.chunk for i in range(wl.n)))
+    assert abs(frac - wl.extra["target"]) < 0.25 * wl.extra["target"], frac
+    print(name, st, "routed fraction", frac)
+
+
+@pytest.mark.parametrize("name", W.SWEEP_128K)
+def test_sweep_128k_full_size_sampled(name):
+    """alpha x chunk-size sweep at n=131072 (16/2 heads) on Gaussian-mixture keys/queries; sampled
+    rows checked; the per-row support sizes span a wide range."""
+    wl = W.get(name)
+    if "x" not in _SWEEP_X:
+        _SWEEP_X["x"] = wl.make()   # the inputs do not depend on alpha or B
+    x = _SWEEP_X["x"]
+    O, pf = run_prefill(x, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma)
+    pos = _sample_positions(wl.n, wl.chunk, 48, 2)
+    st = compare(x, pf, O, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, positions=pos)
+    cnt = pf.counts[0].float()
+    vis = (torch.arange(wl.n, device=cnt.device) // wl.chunk).clamp(min=1).float()
+    frac_rows = (cnt / vis)[:, wl.chunk:]
+    print(name, st, "support fraction p10/p50/p90",
+          [round(v, 3) for v in torch.quantile(frac_rows.flatten()[::97], torch.tensor([0.1, 0.5, 0.9], device=cnt.device)).tolist()])
