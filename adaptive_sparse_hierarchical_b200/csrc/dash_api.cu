@@ -61,7 +61,7 @@ long long route_cap(const dash_params* p)
     return tri_offset(p->seqlen, p->chunk);
 }
 
-struct PrefillLayout { size_t kbar, counts, idx, bias, err, total; };
+struct PrefillLayout { size_t kbar, counts, idx, bias, err, planes, total; };
 PrefillLayout prefill_layout(const dash_params* p)
 {
     PrefillLayout L;
@@ -73,7 +73,8 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.idx = L.counts + up(bh * (size_t)p->seqlen * 4);
     L.bias = L.idx + up(bh * cap * 4);
     L.err = L.bias + up(bh * cap * 4);
-    L.total = L.err + kAlign;
+    L.planes = L.err + kAlign;
+    L.total = L.planes + up(bh * 3 * T * p->d_h * 2);
     return L;
 }
 
@@ -166,12 +167,14 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     if (!aligned4(rt.counts) || !aligned4(rt.idx) || !aligned4(rt.bias) || (rt.bitmask && !aligned4(rt.bitmask)))
         return DASH_EALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // bf16: Stage 0 also writes the summaries as three exact bf16 planes for Stage 1's MMAs
+    __nv_bfloat16* planes = p->dtype == DASH_BF16 ? reinterpret_cast<__nv_bfloat16*>(ws + L.planes) : nullptr;
     if (stage == -1 || stage == DASH_STAGE0) {
-        rc = launch_status(launch_stage0(s, p->dtype, K, qbar, nullptr, kbar, s.T, nullptr, st));
+        rc = launch_status(launch_stage0(s, p->dtype, K, qbar, nullptr, kbar, s.T, nullptr, st, planes));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE1) {
-        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, rt, st));
+        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, rt, st));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE2) {

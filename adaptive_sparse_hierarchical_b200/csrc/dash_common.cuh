@@ -89,14 +89,16 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // ---- launchers (each returns cudaGetLastError() of its launches) -------------------------
 // Stage 0: summaries of complete chunks of positions [0, len_b) and, if state != null, the
 // running state of the incomplete chunk.  len == null means every sequence has length s.n.
+// planes (optional, bf16 [b][hkv][3][T][d]): each summary split exactly into hi + mid + lo.
 cudaError_t launch_stage0(const Shape& s, int dtype, const void* K, const float* qbar,
-                          const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st);
+                          const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st,
+                          __nv_bfloat16* planes = nullptr);
 cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const void* v_new,
                           const float* qbar, void* Kc, void* Vc, float* kbar, int kbar_T,
                           float* state, int* seqlens, cudaStream_t st);
 // Stage 1 for prefill: routes of every position.
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const Routes& rt, cudaStream_t st);
+                                 const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st);
 size_t route_prefill_smem(const Shape& s, int* positions_per_block);
 // Stage 2 for prefill.
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,

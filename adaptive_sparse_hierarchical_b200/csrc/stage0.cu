@@ -48,7 +48,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restrict__ K,
                                                      const float* __restrict__ qbar,
                                                      const int* __restrict__ len, float* kbar,
-                                                     int kbar_T, float* state)
+                                                     int kbar_T, float* state, __nv_bfloat16* planes)
 {
     using L = KeyLanes<T, D>;
     const int lane = threadIdx.x & 31;
@@ -107,6 +107,20 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
         float* out = kbar + (((long long)b * s.hkv + r) * kbar_T + c) * D + sub * L::EPL;
         const float inv = 1.f / run.l;
         for (int e = 0; e < L::EPL; ++e) out[e] = run.acc[e] * inv;
+        if (planes) {
+            // the summary split exactly into three bf16 planes (hi + mid + lo), [b][r][3][T][D]
+            __nv_bfloat16* pl = planes + ((long long)(b * s.hkv + r) * 3 * kbar_T + c) * D + sub * L::EPL;
+            const long long ps = (long long)kbar_T * D;
+            for (int e = 0; e < L::EPL; ++e) {
+                const float v = run.acc[e] * inv;
+                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+                const float rem = v - __bfloat162float(hi);
+                const __nv_bfloat16 mid = __float2bfloat16_rn(rem);
+                pl[e] = hi;
+                pl[ps + e] = mid;
+                pl[2 * ps + e] = __float2bfloat16_rn(rem - __bfloat162float(mid));
+            }
+        }
     } else {
         float* st = state + ((long long)b * s.hkv + r) * (D + 2);
         for (int e = 0; e < L::EPL; ++e) st[sub * L::EPL + e] = run.acc[e];
@@ -164,15 +178,15 @@ __global__ void append_kernel(Shape s, const T* __restrict__ k_new, const T* __r
 
 template <typename T>
 cudaError_t stage0_t(const Shape& s, const void* K, const float* qbar, const int* len, float* kbar,
-                     int kbar_T, float* state, cudaStream_t st)
+                     int kbar_T, float* state, __nv_bfloat16* planes, cudaStream_t st)
 {
     const long long items = (long long)s.batch * s.hkv * (kbar_T + 1);
     const unsigned grid = (unsigned)((items + 3) / 4);
     if (grid == 0) return cudaSuccess;
     if (s.d == 128)
-        stage0_kernel<T, 128><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state);
+        stage0_kernel<T, 128><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes);
     else
-        stage0_kernel<T, 64><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state);
+        stage0_kernel<T, 64><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes);
     return cudaGetLastError();
 }
 
@@ -193,10 +207,11 @@ cudaError_t append_t(const Shape& s, const void* kn, const void* vn, const float
 }  // namespace
 
 cudaError_t launch_stage0(const Shape& s, int dtype, const void* K, const float* qbar,
-                          const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st)
+                          const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st,
+                          __nv_bfloat16* planes)
 {
-    return dtype == DASH_BF16 ? stage0_t<__nv_bfloat16>(s, K, qbar, len, kbar, kbar_T, state, st)
-                              : stage0_t<float>(s, K, qbar, len, kbar, kbar_T, state, st);
+    return dtype == DASH_BF16 ? stage0_t<__nv_bfloat16>(s, K, qbar, len, kbar, kbar_T, state, planes, st)
+                              : stage0_t<float>(s, K, qbar, len, kbar, kbar_T, state, planes, st);
 }
 
 cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const void* v_new,

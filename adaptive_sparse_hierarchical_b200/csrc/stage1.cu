@@ -231,19 +231,39 @@ __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __
     }
 }
 
+// Register-resident threshold: row x[0..nv) with nv <= 32*NPL, NPL values per lane (-inf pads).
+template <int NPL>
+__device__ float warp_threshold_reg(const float (&xr)[NPL], int nv, float alpha)
+{
+    float mx = xr[0];
+#pragma unroll
+    for (int k = 1; k < NPL; ++k) mx = fmaxf(mx, xr[k]);
+    mx = warp_max(mx);
+    return entmax_threshold(
+        [&](auto fn) {
+#pragma unroll
+            for (int k = 0; k < NPL; ++k) fn(xr[k]);
+        },
+        [](float& a, float& b) { a = warp_sum(a); b = warp_sum(b); }, mx, nv, alpha);
+}
+
 // ------------------------------------------------------------------------------------------
 // Prefill, bf16 queries: the chunk logits run on the tensor cores.  A query is exact in bf16;
 // each fp32 summary is split exactly into three bf16 planes (hi + mid + lo = kbar, 8 mantissa
-// bits each), so three bf16 MMAs with fp32 accumulation reproduce the fp32 dot product.
-// Block = 8 warps, ROWS = 16*RG query rows = ROWS/g positions of one (sequence, KV head).
-// Shared memory: one 64-chunk summary tile as three swizzled bf16 planes, logits [ROWS][Ts].
+// bits each; written by Stage 0), so three bf16 MMAs with fp32 accumulation reproduce the fp32
+// dot product.  Block = 8 warps, ROWS = 16*RG query rows = ROWS/g positions of one (sequence,
+// KV head); 32-chunk plane tiles are staged with cp.async.  Shared memory: one tile (three
+// swizzled bf16 planes) and the logits [ROWS][Ts].  Rows of up to 512 visible chunks solve the
+// threshold from registers.
 // ------------------------------------------------------------------------------------------
 template <int D, int RG>
 __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __nv_bfloat16* __restrict__ Q,
-                                                               const float* __restrict__ kbar, Routes rt, int Ts)
+                                                               const __nv_bfloat16* __restrict__ planes,
+                                                               Routes rt, int Ts)
 {
     constexpr int ROWS = 16 * RG;
-    constexpr int PLANE = 64 * D * 2;
+    constexpr int TCH = 32;                    // chunks per staged tile
+    constexpr int PLANE = TCH * D * 2;
     extern __shared__ __align__(128) char smem[];
     char* kt = smem;
     float* S = reinterpret_cast<float*>(smem + 3 * PLANE);
@@ -275,30 +295,21 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
         return Q + (long long)b * s.qs[0] + (long long)i * s.qs[1] + (long long)(r * G + R % G) * s.qs[2];
     });
     const float xs = (s.alpha - 1.f) * s.gamma * rsqrtf((float)D);
-    const float* kb = kbar + (long long)br * s.T * D;
+    const __nv_bfloat16* pg = planes + (long long)br * 3 * s.T * D;
     const int mi = lane >> 3, rr8 = lane & 7, t4 = lane & 3;
-    for (int c0 = 0; c0 < nvmax; c0 += 64) {
+    for (int c0 = 0; c0 < nvmax; c0 += TCH) {
         __syncthreads();
-        for (int v = tid; v < 64 * (D / 4); v += 256) {
-            const int cc = v / (D / 4), e = (v % (D / 4)) * 4;
-            float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (c0 + cc < nvmax) val = *reinterpret_cast<const float4*>(kb + (long long)(c0 + cc) * D + e);
-            const float xv[4] = {val.x, val.y, val.z, val.w};
-            __nv_bfloat16 hb[4], mb[4], lb[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                hb[k] = __float2bfloat16_rn(xv[k]);
-                const float rem = xv[k] - __bfloat162float(hb[k]);
-                mb[k] = __float2bfloat16_rn(rem);
-                lb[k] = __float2bfloat16_rn(rem - __bfloat162float(mb[k]));
-            }
-            const uint32_t off = swz<D>(cc, e);
-            *reinterpret_cast<uint2*>(kt + off) = *reinterpret_cast<uint2*>(hb);
-            *reinterpret_cast<uint2*>(kt + PLANE + off) = *reinterpret_cast<uint2*>(mb);
-            *reinterpret_cast<uint2*>(kt + 2 * PLANE + off) = *reinterpret_cast<uint2*>(lb);
+        for (int v = tid; v < 3 * TCH * (D / 8); v += 256) {
+            const int pl = v / (TCH * (D / 8)), rem = v % (TCH * (D / 8));
+            const int cc = rem / (D / 8), col = (rem % (D / 8)) * 8;
+            const bool ok = c0 + cc < s.T;
+            cp_async16_zfill(kt + pl * PLANE + swz<D>(cc, col),
+                             ok ? pg + ((long long)pl * s.T + c0 + cc) * D + col : pg, ok);
         }
+        cp_async_commit();
+        cp_async_wait<0>();
         __syncthreads();
-        for (int u = warp; u < RG * 4; u += 8) {
+        for (int u = warp; u < RG * (TCH / 16); u += 8) {
             const int slice = u / RG;
             float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -322,26 +333,38 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
         }
     }
     __syncthreads();
+    const float p = 1.f / (s.alpha - 1.f);
+    const int mode = ent_mode(s.alpha);
     for (int row = warp; row < ROWS; row += 8) {
         const int i = i0 + row / G;
         if (i >= s.n) continue;
         const int nv = min(i / s.B, s.T);
         if (nv == 0) continue;
         float* x = S + row * Ts;
-        const float tau = warp_threshold(x, nv, s.alpha);
-        const float p = 1.f / (s.alpha - 1.f);
-        const int mode = ent_mode(s.alpha);
-        for (int c = lane; c < nv; c += 32) {
-            const float u = x[c] - tau;
-            x[c] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
+        if (nv <= 512) {
+            float xr[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) xr[k] = lane + 32 * k < nv ? x[lane + 32 * k] : -INFINITY;
+            const float tau = warp_threshold_reg<16>(xr, nv, s.alpha);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float u = xr[k] - tau;
+                if (lane + 32 * k < nv) x[lane + 32 * k] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
+            }
+        } else {
+            const float tau = warp_threshold(x, nv, s.alpha);
+            for (int c = lane; c < nv; c += 32) {
+                const float u = x[c] - tau;
+                x[c] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
+            }
         }
     }
     __syncthreads();
-    for (int p = warp; p < P; p += 8) {
-        const int i = i0 + p;
+    for (int pp = warp; pp < P; pp += 8) {
+        const int i = i0 + pp;
         if (i >= s.n) continue;
         const int nv = min(i / s.B, s.T);
-        const float* W = S + p * G * Ts;
+        const float* W = S + pp * G * Ts;
         auto wsum = [&](int c) {
             float a = 0.f;
             for (int h = 0; h < G; ++h) a += W[h * Ts + c];
@@ -494,15 +517,15 @@ cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, co
 // Shared memory of the tensor-core routing kernel for RG row groups.
 size_t route_tc_smem(const Shape& s, int RG)
 {
-    const int Ts = (s.T + 63) / 64 * 64 + 8;
-    return 3 * (size_t)64 * s.d * 2 + (size_t)16 * RG * Ts * 4;
+    const int Ts = (s.T + 31) / 32 * 32 + 8;
+    return 3 * (size_t)32 * s.d * 2 + (size_t)16 * RG * Ts * 4;
 }
 
 template <int D, int RG>
-cudaError_t route_tc_t(const Shape& s, const void* Q, const float* kbar, const Routes& rt, cudaStream_t st)
+cudaError_t route_tc_t(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st)
 {
     const size_t smem = route_tc_smem(s, RG);
-    const int Ts = (s.T + 63) / 64 * 64 + 8;
+    const int Ts = (s.T + 31) / 32 * 32 + 8;
     auto k = route_prefill_tc_kernel<D, RG>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -510,21 +533,137 @@ cudaError_t route_tc_t(const Shape& s, const void* Q, const float* kbar, const R
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, kbar, rt, Ts);
+    k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, planes, rt, Ts);
     return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t route_tc_d(const Shape& s, const void* Q, const float* kbar, const Routes& rt, cudaStream_t st,
-                       bool* used)
+cudaError_t route_tc_d(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
+                       cudaStream_t st, bool* used)
 {
     constexpr size_t kLimit = 225 * 1024;
     *used = true;
-    if (16 * 4 >= s.g && route_tc_smem(s, 4) <= kLimit) return route_tc_t<D, 4>(s, Q, kbar, rt, st);
-    if (16 * 2 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, kbar, rt, st);
-    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, kbar, rt, st);
+    if (32 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, planes, rt, st);
+    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, planes, rt, st);
     *used = false;
     return cudaSuccess;
+}
+
+// (b') threshold of one head's row, one block of 256 threads per (head, sequence, KV head); the
+// row stays in registers (up to 16 values per thread) and each Newton step reduces over the block.
+__global__ void __launch_bounds__(256) dec_tau_block_kernel(Shape s, int kbar_T, const int* __restrict__ seqlens,
+                                                            float* X)
+{
+    __shared__ float red[2][8][2];
+    const int h = blockIdx.x, br = blockIdx.y, b = br / s.hkv;
+    const int nv = min((seqlens[b] - 1) / s.B, kbar_T);
+    if (nv <= 0) return;
+    float* x = X + ((long long)br * s.g + h) * kbar_T;
+    constexpr int NPL = 16;
+    float xr[NPL];
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+        const int c = threadIdx.x + 256 * k;
+        xr[k] = c < nv ? x[c] : -INFINITY;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int phase = 0;
+    auto bsum2 = [&](float& a, float& bb) {
+        a = warp_sum(a);
+        bb = warp_sum(bb);
+        if (lane == 0) { red[phase][warp][0] = a; red[phase][warp][1] = bb; }
+        __syncthreads();
+        a = 0.f;
+        bb = 0.f;
+        for (int w = 0; w < 8; ++w) { a += red[phase][w][0]; bb += red[phase][w][1]; }
+        phase ^= 1;   // alternate buffers: the next reduction cannot overwrite values still being read
+    };
+    float mx = xr[0];
+#pragma unroll
+    for (int k = 1; k < NPL; ++k) mx = fmaxf(mx, xr[k]);
+    {
+        const float m2 = warp_max(mx);
+        if (lane == 0) red[phase][warp][0] = m2;
+        __syncthreads();
+        mx = -INFINITY;
+        for (int w = 0; w < 8; ++w) mx = fmaxf(mx, red[phase][w][0]);
+        phase ^= 1;
+    }
+    const float tau = entmax_threshold(
+        [&](auto fn) {
+#pragma unroll
+            for (int k = 0; k < NPL; ++k) fn(xr[k]);
+        },
+        bsum2, mx, nv, s.alpha);
+    const float p = 1.f / (s.alpha - 1.f);
+    const int mode = ent_mode(s.alpha);
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+        const int c = threadIdx.x + 256 * k;
+        const float u = xr[k] - tau;
+        if (c < nv) x[c] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
+    }
+}
+
+// (c') GQA average, bias and ordered compaction from the head weights in global memory: one
+// block of 1024 threads per (sequence, KV head).
+__global__ void __launch_bounds__(1024) dec_emit_block_kernel(Shape s, int kbar_T, const int* __restrict__ seqlens,
+                                                              const float* __restrict__ X, Routes rt)
+{
+    __shared__ float red_f[32];
+    __shared__ int red_i[32], wpos[33];
+    const int br = blockIdx.x, b = br / s.hkv, G = s.g;
+    const int nv = max(0, min((seqlens[b] - 1) / s.B, kbar_T));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+    const float* Xb = X + (long long)br * G * kbar_T;
+    const float inv_g = 1.f / G;
+    auto wof = [&](int c) {
+        float a = 0.f;
+        for (int h = 0; h < G; ++h) a += Xb[(long long)h * kbar_T + c];
+        return a * inv_g;
+    };
+    float sl = 0.f;
+    int cnt = 0;
+    for (int c = tid; c < nv; c += blockDim.x) {
+        const float w = wof(c);
+        if (w > 0.f) { sl += __logf(w); ++cnt; }
+    }
+    sl = warp_sum(sl);
+    cnt = warp_isum(cnt);
+    if (lane == 0) { red_f[warp] = sl; red_i[warp] = cnt; }
+    __syncthreads();
+    float tot = 0.f;
+    int tcnt = 0;
+    for (int k = 0; k < nw; ++k) { tot += red_f[k]; tcnt += red_i[k]; }
+    const float mu = tcnt > 0 ? tot / tcnt : 0.f;
+    int* idx = rt.idx + (long long)br * rt.cap;
+    float* bias = rt.bias + (long long)br * rt.cap;
+    uint32_t* mrow = rt.bitmask ? rt.bitmask + (long long)br * rt.words : nullptr;
+    int base = 0;
+    for (int c0 = 0; c0 < nv; c0 += blockDim.x) {
+        const int c = c0 + tid;
+        const float w = c < nv ? wof(c) : 0.f;
+        const bool on = w > 0.f;
+        const uint32_t m = __ballot_sync(0xffffffffu, on);
+        __syncthreads();
+        if (lane == 0) red_i[warp] = __popc(m);
+        __syncthreads();
+        if (tid == 0) {
+            wpos[0] = 0;
+            for (int k = 0; k < nw; ++k) wpos[k + 1] = wpos[k] + red_i[k];
+        }
+        __syncthreads();
+        if (on) {
+            const int k = base + wpos[warp] + __popc(m & ((1u << lane) - 1u));
+            idx[k] = c;
+            bias[k] = (__logf(w) - mu) * s.inv_sigma;
+        }
+        if (mrow && lane == 0 && c0 + 32 * warp < nv) mrow[(c0 + 32 * warp) >> 5] = m;
+        base += wpos[nw];
+    }
+    if (mrow)
+        for (int wd = ((nv + 31) >> 5) + tid; wd < rt.words; wd += blockDim.x) mrow[wd] = 0u;
+    if (tid == 0) rt.counts[br] = base;
 }
 
 template <typename T, int D>
@@ -534,6 +673,11 @@ cudaError_t dec_route_t(const Shape& s, const void* q, const float* kbar, int kb
     if (kbar_T > 0) {
         dim3 g1((kbar_T + 31) / 32, s.batch * s.hkv);
         dec_logits_kernel<T, D><<<g1, 256, 0, st>>>(s, (const T*)q, kbar, kbar_T, seqlens, X);
+    }
+    if (kbar_T <= 16 * 256) {
+        if (kbar_T > 0) dec_tau_block_kernel<<<dim3(s.g, s.batch * s.hkv), 256, 0, st>>>(s, kbar_T, seqlens, X);
+        dec_emit_block_kernel<<<s.batch * s.hkv, 1024, 0, st>>>(s, kbar_T, seqlens, X, rt);
+        return cudaGetLastError();
     }
     const size_t smem = (size_t)s.g * (kbar_T > 0 ? kbar_T : 1) * 4;
     cudaError_t e = cudaFuncSetAttribute(dec_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -561,11 +705,12 @@ size_t route_prefill_smem(const Shape& s, int* positions_per_block)
 }
 
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const Routes& rt, cudaStream_t st)
+                                 const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st)
 {
-    if (dtype == DASH_BF16) {
+    if (dtype == DASH_BF16 && planes) {
         bool used = false;
-        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, kbar, rt, st, &used) : route_tc_d<64>(s, Q, kbar, rt, st, &used);
+        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, planes, rt, st, &used)
+                                   : route_tc_d<64>(s, Q, planes, rt, st, &used);
         if (used) return e;
         // very long rows (T * 16 rows of logits beyond shared memory): CUDA-core variant
         return s.d == 128 ? route_prefill_t<__nv_bfloat16, 128>(s, Q, kbar, rt, st)

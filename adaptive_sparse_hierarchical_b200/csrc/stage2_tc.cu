@@ -276,9 +276,13 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         const int* li = ridx + (valid ? tri_offset(i, s.B) : 0);
         const float* lb = rbias + (valid ? tri_offset(i, s.B) : 0);
         const int cnt = valid ? counts[i] : 0;
+        // the row's next two routed chunks stay in registers, so the global load of an entry is
+        // issued at least one tile before the entry is compared
         int cur = 0;
         int nxt = cnt > 0 ? li[0] : INT_MAX;
         float nbias = cnt > 0 ? lb[0] : 0.f;
+        int nxt2 = cnt > 1 ? li[1] : INT_MAX;
+        float nbias2 = cnt > 1 ? lb[1] : 0.f;
         const float scale2 = kLog2e * rsqrtf((float)kD);
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
         float m = -INFINITY, l = 0.f;
@@ -373,8 +377,10 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             tc::mbar_arrive(bar.p_full[sb]);
             if (k % NH == NH - 1 && nxt == c) {
                 ++cur;
-                nxt = cur < cnt ? li[cur] : INT_MAX;
-                nbias = cur < cnt ? lb[cur] : 0.f;
+                nxt = nxt2;
+                nbias = nbias2;
+                nxt2 = cur + 1 < cnt ? li[cur + 1] : INT_MAX;
+                nbias2 = cur + 1 < cnt ? lb[cur + 1] : 0.f;
             }
         }
         // ---- epilogue: O / l -> bf16 --------------------------------------------------------
