@@ -116,3 +116,22 @@ class DecodeState:
     def step(self, q, k_new, v_new, stream=None):
         self.append(k_new, v_new, stream)
         return self.decode(q, stream)
+
+    def graph_step(self, q, k_new, v_new):
+        """step() through a CUDA graph: the first call runs eagerly (one-time set-up stays out of
+        the capture) and records append + decode on static input buffers; later calls copy the
+        inputs in and replay.  The kernels read the lengths from device memory, so one graph
+        serves every step."""
+        if getattr(self, "_graph", None) is None:
+            out = self.step(q, k_new, v_new)
+            self._qs, self._ks, self._vs = q.clone(), k_new.clone(), v_new.clone()
+            self._graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self._graph):
+                self.append(self._ks, self._vs)
+                self.decode(self._qs)
+            return out
+        self._qs.copy_(q)
+        self._ks.copy_(k_new)
+        self._vs.copy_(v_new)
+        self._graph.replay()
+        return self.O

@@ -85,7 +85,9 @@ DecodeLayout decode_layout(const dash_params* p)
     const Shape s = make_shape(p);
     const size_t bh = (size_t)p->batch * p->h_kv;
     const size_t T = (size_t)s.T;
+    // partial slots per (sequence, KV head): the split kernel's splits, or one per persistent block
     L.splits = decode_splits(s, s.T);
+    if (dec_tma_blocks() > L.splits) L.splits = dec_tma_blocks();
     L.x = 0;
     L.part = L.x + up(bh * s.g * (T > 0 ? T : 1) * 4);
     L.counts = L.part + up(bh * (size_t)L.splits * s.g * (p->d_h + 2) * 4);

@@ -118,10 +118,9 @@ struct DecodeWs {
 };
 // Decode Stage 2 with TMA-fed K/V rings (bf16, d = 128, chunk 64 or 128).
 bool dec_tma_supported(const Shape& s, int dtype);
-int dec_tma_splits(const Shape& s, int kbar_T);
-int dec_tma_cps();
+int dec_tma_blocks();   // persistent blocks (the SM count); partial slots per pair
 cudaError_t launch_dec_attend_tma(const Shape& s, const void* q, const void* Kc, const void* Vc, const int* seqlens,
-                                  const Routes& rt, float* part, int splits, int* err, cudaStream_t st);
+                                  const Routes& rt, float* part, void* O, int* err, cudaStream_t st);
 cudaError_t launch_route_decode(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
                                 const int* seqlens, const Routes& rt, float* X, cudaStream_t st);
 cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* Kc, const void* Vc,

@@ -64,7 +64,8 @@ extern "C" int dash_decode_noalloc(const dash_params* p, const void* q, const vo
     const size_t T = (size_t)(p->seqlen / (p->chunk > 0 ? p->chunk : 1));
     const size_t Tn = T > 0 ? T : 1;
     const size_t bh = (size_t)p->batch * p->h_kv;
-    const size_t splits = (T + 1 + 7) / 8;
+    size_t splits = (T + 1 + 7) / 8;
+    if ((size_t)dec_tma_blocks() > splits) splits = (size_t)dec_tma_blocks();
     const size_t off_part = upna(bh * g * Tn * 4);
     const size_t off_counts = off_part + upna(bh * splits * g * ((size_t)p->d_h + 2) * 4);
     const size_t off_idx = off_counts + upna(bh * 4);

@@ -486,12 +486,8 @@ cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* 
     cudaError_t e = launch_route_decode(s, dtype, q, kbar, kbar_T, seqlens, rt, ws.x, st);
     if (e != cudaSuccess) return e;
     if (dec_tma_supported(s, dtype) && !legacy_stage2()) {
-        const int splits = dec_tma_splits(s, kbar_T);
-        e = launch_dec_attend_tma(s, q, Kc, Vc, seqlens, rt, ws.part, splits, ws.err, st);
+        e = launch_dec_attend_tma(s, q, Kc, Vc, seqlens, rt, ws.part, O, ws.err, st);
         if (e != cudaSuccess) return e;
-        dec_combine_kernel<__nv_bfloat16, 128><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, ws.part, splits,
-                                                                                      dec_tma_cps(), rt,
-                                                                                      (__nv_bfloat16*)O);
         return cudaGetLastError();
     }
     if (dtype == DASH_BF16)

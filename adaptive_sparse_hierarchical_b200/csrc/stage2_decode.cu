@@ -18,7 +18,6 @@
 namespace dash {
 namespace {
 
-constexpr int kCPS = 16;          // route entries (chunks) per split
 constexpr int kNSd = 6;           // ring slots
 constexpr int kHalf = 64 * 64 * 2;
 constexpr int kSlotB = 4 * kHalf; // K halves + V halves = 32 KB
@@ -35,10 +34,17 @@ __device__ __forceinline__ uint32_t sw_off(int row, int col)
     return (uint32_t)(half * kHalf + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) + (c & 7) * 2);
 }
 
+// Persistent: gridDim.x blocks (one per SM) split the concatenated tile list of all (sequence,
+// KV head) pairs evenly.  Pair br owns tiles [P[br], P[br+1]) with P the prefix sum of
+// (count + 1) * B/64 (the +1 is the diagonal chunk).  A block walks its range segment by segment;
+// for each pair it touches it writes one partial (o, m, l) per head at part[br][block].
+constexpr int kMaxBR = 64;
+constexpr int kMaxJobs = 2048;   // per-block tile table in shared memory
+
 __global__ void __launch_bounds__(32 * (1 + kCons), 1)
 dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Shape s,
                       const __nv_bfloat16* __restrict__ q, const int* __restrict__ seqlens, Routes rt,
-                      float* __restrict__ part, int splits, int* err)
+                      float* __restrict__ part, int* err)
 {
     extern __shared__ char smem_raw[];
     char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -46,25 +52,59 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     const uint32_t bar_full = base + kNSd * kSlotB, bar_empty = bar_full + 8 * kNSd;
     volatile int* abort = reinterpret_cast<volatile int*>(sm + kNSd * kSlotB + 16 * kNSd);
     float* mrg = reinterpret_cast<float*>(sm + kNSd * kSlotB + 16 * kNSd + 16);   // [kCons][16][2]
+    int* pre = reinterpret_cast<int*>(mrg + kCons * 16 * 2);                         // [kMaxBR + 1]
+    float* osm = reinterpret_cast<float*>(pre + kMaxBR + 1);                         // [16][128]
+    int* jkey = reinterpret_cast<int*>(osm + 16 * 128);                              // [kMaxJobs] first key
+    float* jbias = reinterpret_cast<float*>(jkey + kMaxJobs);                        // [kMaxJobs] bias, NaN = diagonal
 
-    const int br = blockIdx.y, sp = blockIdx.x, b = br / s.hkv, r = br % s.hkv;
-    const int L = seqlens[b], i = L - 1, G = s.g;
-    const int cnt = rt.counts[br];
-    const int e0 = sp * kCPS, e1 = min(e0 + kCPS, cnt + 1);
-    if (e0 >= e1 || L <= 0) return;
-    const int NH = s.B / 64;
-    const int njobs = (e1 - e0) * NH;
-    const int* li = rt.idx + (long long)br * rt.cap;
-    const float* lb = rt.bias + (long long)br * rt.cap;
+    const int BR = s.batch * s.hkv, G = s.g, NH = s.B / 64;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
     if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int x = 0; x < BR; ++x) {
+            pre[x] = acc;
+            acc += (rt.counts[x] + 1) * NH;
+        }
+        pre[BR] = acc;
         for (int k = 0; k < kNSd; ++k) { tc::mbar_init(bar_full + 8 * k, 1); tc::mbar_init(bar_empty + 8 * k, 1); }
         *abort = 0;
         tc::mbar_fence_init();
     }
     __syncthreads();
-    auto chunk_of = [&](int e) { return e < cnt ? li[e] : i / s.B; };
+    const long long total = pre[BR];
+    const int j_lo = (int)(total * blockIdx.x / gridDim.x), j_hi = (int)(total * (blockIdx.x + 1) / gridDim.x);
+    if (j_lo >= j_hi) return;
+    auto seg_of = [&](int j) {
+        int x = 0;
+        while (pre[x + 1] <= j) ++x;
+        return x;
+    };
+    // first key and bias of every tile of this block's range, looked up once (NaN bias marks the
+    // pair's diagonal chunk); ranges beyond the table fall back to looking tiles up on the fly
+    const int njobs = j_hi - j_lo;
+    const bool table = njobs <= kMaxJobs;
+    auto lookup = [&](int j, int x, int* key0, float* bias) {
+        const int t = j - pre[x], e = t / NH;
+        const int cnt = rt.counts[x];
+        if (e < cnt) {
+            *key0 = rt.idx[(long long)x * rt.cap + e] * s.B + (t % NH) * 64;
+            *bias = rt.bias[(long long)x * rt.cap + e];
+        } else {
+            *key0 = ((seqlens[x / s.hkv] - 1) / s.B) * s.B + (t % NH) * 64;
+            *bias = __int_as_float(0x7fc00000);
+        }
+    };
+    if (table) {
+        for (int k = threadIdx.x; k < njobs; k += blockDim.x) {
+            const int j = j_lo + k;
+            lookup(j, seg_of(j), &jkey[k], &jbias[k]);
+        }
+        __syncthreads();
+    }
+    auto job = [&](int k, int x, int* key0, float* bias) {
+        if (table) { *key0 = jkey[k]; *bias = jbias[k]; }
+        else lookup(j_lo + k, x, key0, bias);
+    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -72,17 +112,23 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             tc::prefetch_tmap(&tmV);
             int last[kNSd];
             for (int k = 0; k < kNSd; ++k) last[k] = -1;
-            for (int k = 0; k < njobs; ++k) {
+            int x = seg_of(j_lo);
+            for (int k = 0; k < j_hi - j_lo; ++k) {
+                const int j = j_lo + k;
+                while (pre[x + 1] <= j) ++x;
                 const int slot = k % kNSd;
                 if (k >= kNSd && !tc::mbar_wait(bar_empty + 8 * slot, ((k / kNSd) - 1) & 1, abort, err, 11)) break;
                 last[slot] = k;
-                const int key0 = chunk_of(e0 + k / NH) * s.B + (k % NH) * 64;
+                int key0;
+                float bdummy;
+                job(k, x, &key0, &bdummy);
+                const int bb = x / s.hkv, r = x % s.hkv;
                 const uint32_t dst = base + slot * kSlotB, fb = bar_full + 8 * slot;
                 tc::mbar_expect_tx(fb, kSlotB);
-                tc::tma_load_4d(dst, &tmK, fb, 0, r, key0, b);
-                tc::tma_load_4d(dst + kHalf, &tmK, fb, 64, r, key0, b);
-                tc::tma_load_4d(dst + 2 * kHalf, &tmV, fb, 0, r, key0, b);
-                tc::tma_load_4d(dst + 3 * kHalf, &tmV, fb, 64, r, key0, b);
+                tc::tma_load_4d(dst, &tmK, fb, 0, r, key0, bb);
+                tc::tma_load_4d(dst + kHalf, &tmK, fb, 64, r, key0, bb);
+                tc::tma_load_4d(dst + 2 * kHalf, &tmV, fb, 0, r, key0, bb);
+                tc::tma_load_4d(dst + 3 * kHalf, &tmV, fb, 64, r, key0, bb);
             }
             if (*abort)   // let copies still in flight land before the block's shared memory goes away
                 for (int k = 0; k < kNSd; ++k)
@@ -90,25 +136,36 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                         for (long long it = 0; it < (1ll << 22); ++it)
                             if (tc::mbar_try(bar_full + 8 * k, (last[k] / kNSd) & 1)) break;
         }
-    } else {
-        const int cw = warp - 1;
-        const int ra = lane >> 2, rb = ra + 8, t4 = lane & 3;
+        return;
+    }
+    // ---- consumers ------------------------------------------------------------------------------
+    const int cw = warp - 1;
+    const int ra = lane >> 2, rb = ra + 8, t4 = lane & 3;
+    const float scale2 = kLog2e * rsqrtf(128.f);
+    const int mi = lane >> 3, rr8 = lane & 7;
+    // a segment is the part of one pair's tiles inside this block's range
+    for (int x = seg_of(j_lo); x < BR && pre[x] < j_hi; ++x) {
+        const int s_lo = max(j_lo, pre[x]), s_hi = min(j_hi, pre[x + 1]);
+        const int bb = x / s.hkv, r = x % s.hkv;
+        const int L = seqlens[bb], i = L - 1;
         uint32_t qf[8][4];
         load_q_frags<128>(qf, [&](int rr) -> const __nv_bfloat16* {
-            return rr < G ? q + ((long long)b * s.hq + r * G + rr) * 128 : nullptr;
+            return rr < G ? q + ((long long)bb * s.hq + r * G + rr) * 128 : nullptr;
         });
         WarpAcc<128> acc;
         acc.init();
-        const float scale2 = kLog2e * rsqrtf(128.f);
-        const int mi = lane >> 3, rr8 = lane & 7;
-        for (int k = cw; k < njobs; k += kCons) {
+        // job index k counts tiles from j_lo: warp k % kCons, slot k % kNSd
+        int k0 = s_lo - j_lo;
+        k0 += ((cw - k0) % kCons + kCons) % kCons;
+        for (int k = k0; k < s_hi - j_lo; k += kCons) {
             const int slot = k % kNSd;
             if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_full + 8 * slot, (k / kNSd) & 1, abort, err, 12))) break;
             char* tile = sm + slot * kSlotB;
-            const int e = e0 + k / NH, c = chunk_of(e);
-            const int j0 = c * s.B + (k % NH) * 64;
+            int j0;
+            float jb;
+            job(k, x, &j0, &jb);
             RowMode md;
-            if (e < cnt) { md.bias2 = lb[e] * kLog2e; md.jmax = INT_MAX; }
+            if (jb == jb) { md.bias2 = jb * kLog2e; md.jmax = INT_MAX; }
             else {
                 md.bias2 = 0.f;
                 md.jmax = i;
@@ -123,7 +180,6 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             off.bias2 = -INFINITY;
             off.jmax = INT_MAX;
             const RowMode mA = ra < G ? md : off, mB = rb < G ? md : off;
-            // S = Q K^T over 64 keys
             float sv[8][4];
 #pragma unroll
             for (int j = 0; j < 8; ++j) sv[j][0] = sv[j][1] = sv[j][2] = sv[j][3] = 0.f;
@@ -144,10 +200,10 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
                     const RowMode& m = q2 < 2 ? mA : mB;
-                    float x = sv[j][q2] * scale2 + m.bias2;
-                    if (j0 + j * 8 + 2 * t4 + (q2 & 1) > m.jmax) x = -INFINITY;
-                    sv[j][q2] = x;
-                    mx[q2 >> 1] = fmaxf(mx[q2 >> 1], x);
+                    float xv = sv[j][q2] * scale2 + m.bias2;
+                    if (j0 + j * 8 + 2 * t4 + (q2 & 1) > m.jmax) xv = -INFINITY;
+                    sv[j][q2] = xv;
+                    mx[q2 >> 1] = fmaxf(mx[q2 >> 1], xv);
                 }
             float corr[2];
 #pragma unroll
@@ -170,11 +226,10 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             for (int j = 0; j < 8; ++j)
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
-                    const float p = exp2f(sv[j][q2] - mx[q2 >> 1]);
-                    sv[j][q2] = p;
-                    acc.l[q2 >> 1] += p;
+                    const float pv = exp2f(sv[j][q2] - mx[q2 >> 1]);
+                    sv[j][q2] = pv;
+                    acc.l[q2 >> 1] += pv;
                 }
-            // O += P V
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t a[4];
@@ -193,7 +248,7 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar_empty + 8 * slot);
         }
-        // merge the consumer warps: max and sum per row, then the rescaled outputs
+        // ---- merge the consumer warps' states of this segment (fixed order: deterministic) ----
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             acc.l[h] += __shfl_xor_sync(0xffffffffu, acc.l[h], 1);
@@ -202,51 +257,125 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         if (t4 == 0) {
             mrg[(cw * 16 + ra) * 2] = acc.m[0];
             mrg[(cw * 16 + rb) * 2] = acc.m[1];
+            mrg[(cw * 16 + ra) * 2 + 1] = acc.l[0];
+            mrg[(cw * 16 + rb) * 2 + 1] = acc.l[1];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons));
-        float M[2], sc[2];
+        // common maximum per row, then the warps add their rescaled sums one after another
+        float sc[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int row = h ? rb : ra;
-            M[h] = -INFINITY;
-            for (int w = 0; w < kCons; ++w) M[h] = fmaxf(M[h], mrg[(w * 16 + row) * 2]);
-            sc[h] = M[h] == -INFINITY ? 0.f : exp2f(acc.m[h] - M[h]);
+            float M = -INFINITY;
+            for (int w = 0; w < kCons; ++w) M = fmaxf(M, mrg[(w * 16 + row) * 2]);
+            sc[h] = acc.m[h] == -INFINITY ? 0.f : exp2f(acc.m[h] - M);
         }
-        float* osm = reinterpret_cast<float*>(sm);   // ring is idle now: [16][128] output sums
-        // one snapshot of the abort flag for all consumer threads: the branch below holds barriers
-        volatile int* snap = reinterpret_cast<volatile int*>(sm + kNSd * kSlotB + 16 * kNSd + 8);
-        if (threadIdx.x == 32) *snap = *abort;
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons));
-        if (!*snap) {
-            for (int v = threadIdx.x - 32; v < 16 * 128; v += 32 * kCons) osm[v] = 0.f;
-            if (t4 == 0) {
-                mrg[(cw * 16 + ra) * 2 + 1] = acc.l[0] * sc[0];
-                mrg[(cw * 16 + rb) * 2 + 1] = acc.l[1] * sc[1];
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons));
+        for (int w = 0; w < kCons; ++w) {
+            if (cw == w) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int col = j * 8 + 2 * t4;
-                atomicAdd(&osm[ra * 128 + col], acc.o[j][0] * sc[0]);
-                atomicAdd(&osm[ra * 128 + col + 1], acc.o[j][1] * sc[0]);
-                atomicAdd(&osm[rb * 128 + col], acc.o[j][2] * sc[1]);
-                atomicAdd(&osm[rb * 128 + col + 1], acc.o[j][3] * sc[1]);
+                for (int j = 0; j < 16; ++j) {
+                    const int col = j * 8 + 2 * t4;
+                    float* oa = osm + ra * 128 + col;
+                    float* ob = osm + rb * 128 + col;
+                    if (w == 0) {
+                        oa[0] = acc.o[j][0] * sc[0]; oa[1] = acc.o[j][1] * sc[0];
+                        ob[0] = acc.o[j][2] * sc[1]; ob[1] = acc.o[j][3] * sc[1];
+                    } else {
+                        oa[0] += acc.o[j][0] * sc[0]; oa[1] += acc.o[j][1] * sc[0];
+                        ob[0] += acc.o[j][2] * sc[1]; ob[1] += acc.o[j][3] * sc[1];
+                    }
+                }
             }
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons));
-            float* pb = part + ((long long)br * splits + sp) * G * 130;
-            for (int v = threadIdx.x - 32; v < G * 128; v += 32 * kCons) {
-                const int row = v >> 7, col = v & 127;
-                pb[row * 130 + col] = osm[row * 128 + col];
-            }
-            if (threadIdx.x - 32 < G) {
-                const int row = threadIdx.x - 32;
-                float Mr = -INFINITY, Lr = 0.f;
-                for (int w = 0; w < kCons; ++w) Mr = fmaxf(Mr, mrg[(w * 16 + row) * 2]);
-                for (int w = 0; w < kCons; ++w) Lr += mrg[(w * 16 + row) * 2 + 1];
-                pb[row * 130 + 128] = Mr;
-                pb[row * 130 + 129] = Lr;
-            }
         }
+        float* pb = part + ((long long)x * gridDim.x + blockIdx.x) * G * 130;
+        for (int v = threadIdx.x - 32; v < G * 128; v += 32 * kCons) {
+            const int row = v >> 7, col = v & 127;
+            pb[row * 130 + col] = osm[row * 128 + col];
+        }
+        if (threadIdx.x - 32 < G) {
+            const int row = threadIdx.x - 32;
+            float M = -INFINITY, Lr = 0.f;
+            for (int w = 0; w < kCons; ++w) M = fmaxf(M, mrg[(w * 16 + row) * 2]);
+            for (int w = 0; w < kCons; ++w) {
+                const float mw = mrg[(w * 16 + row) * 2];
+                if (mw != -INFINITY) Lr += mrg[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
+            }
+            pb[row * 130 + 128] = M;
+            pb[row * 130 + 129] = Lr;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons));   // osm / mrg are reused by the next segment
+    }
+}
+
+// Merge of the per-block partials of each pair: one block per (pair, head).  The blocks that
+// touched pair br are those whose tile range meets [P[br], P[br+1]).
+template <int D>
+__global__ void __launch_bounds__(128) dec_merge_kernel(Shape s, const float* __restrict__ part, int nblocks,
+                                                        Routes rt, __nv_bfloat16* __restrict__ O)
+{
+    __shared__ float wk[1024];
+    __shared__ float red[4];
+    __shared__ int range[2];
+    __shared__ long long span[3];   // total tiles, this pair's first and one-past-last tile
+    const int x = blockIdx.x / s.g, row = blockIdx.x % s.g, G = s.g, NH = s.B / 64;
+    const int b = x / s.hkv, r = x % s.hkv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        long long acc = 0, lo = 0, hi = 0;
+        for (int y = 0; y < s.batch * s.hkv; ++y) {
+            if (y == x) lo = acc;
+            acc += (long long)(rt.counts[y] + 1) * NH;
+            if (y == x) hi = acc;
+        }
+        // blocks c with [acc*c/n, acc*(c+1)/n) meeting [lo, hi)
+        int c0 = (int)((lo * nblocks) / acc), c1 = (int)(((hi - 1) * nblocks) / acc);
+        while (c0 > 0 && acc * c0 / nblocks > lo) --c0;
+        while (c0 < nblocks - 1 && acc * (c0 + 1) / nblocks <= lo) ++c0;
+        while (c1 < nblocks - 1 && acc * (c1 + 1) / nblocks <= hi - 1) ++c1;
+        while (c1 > 0 && acc * c1 / nblocks > hi - 1) --c1;
+        range[0] = c0;
+        range[1] = c1;
+        span[0] = acc;
+        span[1] = lo;
+        span[2] = hi;
+    }
+    __syncthreads();
+    // a block wrote a partial for this pair iff its tile range meets the pair's tiles
+    auto valid_block = [&](int c) {
+        const long long a = span[0] * c / nblocks, e = span[0] * (c + 1) / nblocks;
+        return (a > span[1] ? a : span[1]) < (e < span[2] ? e : span[2]);
+    };
+    const int c0 = range[0], nsp = range[1] - range[0] + 1;
+    const float* basep = part + ((long long)x * nblocks + c0) * G * 130 + (long long)row * 130;
+    const long long sstride = (long long)G * 130;
+    float M = -INFINITY;
+    for (int k = tid; k < nsp; k += blockDim.x) if (valid_block(c0 + k)) M = fmaxf(M, basep[k * sstride + 128]);
+    M = warp_max(M);
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    float Lsum = 0.f;
+    for (int k = tid; k < nsp; k += blockDim.x) {
+        float w = 0.f;
+        if (valid_block(c0 + k)) {
+            const float mk = basep[k * sstride + 128];
+            w = mk == -INFINITY ? 0.f : exp2f(mk - M);
+            Lsum += basep[k * sstride + 129] * w;
+        }
+        wk[k] = w;
+    }
+    Lsum = warp_sum(Lsum);
+    if (lane == 0) red[warp] = Lsum;
+    __syncthreads();
+    Lsum = red[0] + red[1] + red[2] + red[3];
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    for (int col = tid; col < D; col += blockDim.x) {
+        float o = 0.f;
+        for (int k = 0; k < nsp; ++k)
+            if (wk[k] != 0.f) o += basep[k * sstride + col] * wk[k];
+        O[((long long)b * s.hq + r * G + row) * D + col] = __float2bfloat16_rn(o * inv);
     }
 }
 
@@ -282,28 +411,34 @@ bool map_kv(CUtensorMap* map, const void* ptr, const Shape& s, const long long s
 
 bool dec_tma_supported(const Shape& s, int dtype)
 {
-    return dtype == DASH_BF16 && s.d == 128 && (s.B == 64 || s.B == 128) && s.g <= 16 && encode_fn_d() != nullptr;
+    return dtype == DASH_BF16 && s.d == 128 && (s.B == 64 || s.B == 128) && s.g <= 16 &&
+           s.batch * s.hkv <= kMaxBR && encode_fn_d() != nullptr;
 }
 
-int dec_tma_splits(const Shape& s, int kbar_T)
+int dec_tma_blocks()
 {
-    (void)s;
-    return (kbar_T + 1 + kCPS - 1) / kCPS;
+    static int n = 0;
+    if (!n) {
+        int dev = 0, sms = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        n = sms > 0 ? (sms > 1024 ? 1024 : sms) : 148;
+    }
+    return n;
 }
-
-int dec_tma_cps() { return kCPS; }
 
 cudaError_t launch_dec_attend_tma(const Shape& s, const void* q, const void* Kc, const void* Vc, const int* seqlens,
-                                  const Routes& rt, float* part, int splits, int* err, cudaStream_t st)
+                                  const Routes& rt, float* part, void* O, int* err, cudaStream_t st)
 {
     CUtensorMap mk, mv;
     if (!map_kv(&mk, Kc, s, s.ks) || !map_kv(&mv, Vc, s, s.vs)) return cudaErrorInvalidValue;
-    const size_t smem = 1024 + kNSd * kSlotB + 16 * kNSd + 16 + kCons * 16 * 2 * 4;
+    const size_t smem = 1024 + kNSd * kSlotB + 16 * kNSd + 16 + kCons * 16 * 2 * 4 + (kMaxBR + 1) * 4 +
+                        16 * 128 * 4 + 2 * kMaxJobs * 4;
     cudaError_t e = cudaFuncSetAttribute(dec_attend_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(splits, s.batch * s.hkv);
-    dec_attend_tma_kernel<<<grid, 32 * (1 + kCons), smem, st>>>(mk, mv, s, (const __nv_bfloat16*)q, seqlens, rt, part,
-                                                              splits, err);
+    const int nb = dec_tma_blocks();
+    dec_attend_tma_kernel<<<nb, 32 * (1 + kCons), smem, st>>>(mk, mv, s, (const __nv_bfloat16*)q, seqlens, rt, part, err);
+    dec_merge_kernel<128><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, part, nb, rt, (__nv_bfloat16*)O);
     return cudaGetLastError();
 }
 

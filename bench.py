@@ -277,22 +277,34 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
         st.step(qn[s], kn[s], vn[s])
     reset()
     torch.cuda.synchronize(dev)
-    ranks.barrier()
+    # eager pass: per-kernel-group times (append / decode) and the routed counts
     evs = [(ev(), ev(), ev()) for _ in range(nst)]
     routed = []
+    for s in range(nst):
+        evs[s][0].record(stream)
+        st.append(kn[s], vn[s])
+        evs[s][1].record(stream)
+        st.decode(qn[s])
+        evs[s][2].record(stream)
+        if s % 50 == 0:
+            routed.append((s, counts.clone()))
+    torch.cuda.synchronize(dev)
+    eager_ms = statistics.mean(a.elapsed_time(c) for a, b, c in evs)
+    dec_ms = [b.elapsed_time(c) for a, b, c in evs]
+    # timed pass: each step = copy the step's q, k, v into the graph's inputs + one graph replay
+    reset()
+    st.graph_step(qn[0], kn[0], vn[0])   # eager first step, then capture
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    gevs = [(ev(), ev()) for _ in range(nst - 1)]
     with Clocks(ranks.local) as clk:
-        for s in range(nst):
-            evs[s][0].record(stream)
-            st.append(kn[s], vn[s])
-            evs[s][1].record(stream)
-            st.decode(qn[s])
-            evs[s][2].record(stream)
-            if s % 50 == 0:
-                routed.append((s, counts.clone()))
+        for s in range(1, nst):
+            gevs[s - 1][0].record(stream)
+            st.graph_step(qn[s], kn[s], vn[s])
+            gevs[s - 1][1].record(stream)
         torch.cuda.synchronize(dev)
     ranks.barrier()
-    step_ms = [a.elapsed_time(c) for a, b, c in evs]
-    dec_ms = [b.elapsed_time(c) for a, b, c in evs]
+    step_ms = [a.elapsed_time(b) for a, b in gevs]
     ms = ranks.max(statistics.mean(step_ms))
     # routed K+V bytes per step (numerator of the HBM roofline), from sampled steps' counts
     byts = []
@@ -301,17 +313,19 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
         diag = (L - 1) % wl.chunk + 1
         byts.append(2 * wl.d * 2 * (float(c.sum()) * wl.chunk + wl.batch * wl.h_kv * diag))
     bps = statistics.mean(byts)
-    achieved = bps / (statistics.mean(dec_ms) / 1e3) / 1e9
+    achieved = bps / (ms / 1e3) / 1e9   # whole graph step (append + route + attend + merge)
     res = {"workload": "decode_128k: b=8, 131072-token caches (+1 per step), 32/2 heads, d=128, B=64, alpha 1.5, "
                        f"gamma {wl.gamma} (~25% routed)",
-           "us_per_step": ms * 1e3,
+           "us_per_step": ms * 1e3, "us_per_step_eager": eager_ms * 1e3,
+           "timing": "per step: copy of q, k, v into the captured graph's inputs + graph replay (append + decode)",
            "steps": nst, "append_us": statistics.mean(a.elapsed_time(b) for a, b, c in evs) * 1e3,
            "decode_us": statistics.mean(dec_ms) * 1e3,
            "routed_fraction": float(routed[-1][1].sum()) / (wl.batch * wl.h_kv * ((prefix + routed[-1][0]) // wl.chunk)),
-           "roofline": {"kernel": "decode (route + split attend + merge)", "bound": "hbm", "achieved": achieved,
+           "roofline": {"kernel": "decode step (append, route, dec_attend_tma_kernel, merge)", "bound": "hbm",
+                        "achieved": achieved,
                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
                         "peak_kind": f"hbm copy, of {pk_kind}", "bytes_per_step": bps},
-           "clocks": clk.summary(), "gpu_launches": 6 * nst,
+           "clocks": clk.summary(), "gpu_launches": 6 * (nst - 1),
            "l2": "KV caches (1.07 GB) larger than L2"}
     res["us_per_token"] = res["us_per_step"] / wl.batch   # per sequence-token, one GPU
     return res
