@@ -36,7 +36,7 @@ constexpr int kTmemCols = 256;                    // S0 [0,64), S1 [64,128), O [
 constexpr int kOffQ = 0, kOffSlots = kQBytes;
 constexpr int kOffScratch = kOffSlots;            // set-up scratch (chunk bitmask, sort keys) in the ring
 constexpr int kOffBar = kOffSlots + kNS * kSlot;  // 98304: two blocks fit on one SM
-constexpr int kNumBars = 1 + 2 * kNS + 2 + 2 + 2 + 2 + 1;
+constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 2 + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, njobs
 constexpr int kOffPos = kOffMisc + 32;             // the block's positions (<= 16 when clustered)
 constexpr int kOffJobs = kOffPos + 4 * kRows;
@@ -53,7 +53,9 @@ __device__ __forceinline__ float ex2_approx(float x)
 }
 
 struct Bars {
-    uint32_t q_full, kv_full[kNS], kv_empty[kNS], s_full[2], s_free[2], p_full[2], pv_done[2], drain;
+    // K and V of a slot have their own barriers: K is free once S = Q K^T is done, V only after P V
+    uint32_t q_full, k_full[kNS], k_empty[kNS], v_full[kNS], v_empty[kNS], s_full[2], s_free[2], p_full[2],
+        pv_done[2], drain;
 };
 
 __device__ __forceinline__ Bars make_bars(uint32_t base)
@@ -61,8 +63,10 @@ __device__ __forceinline__ Bars make_bars(uint32_t base)
     Bars b;
     uint32_t a = base + kOffBar;
     b.q_full = a; a += 8;
-    for (int k = 0; k < kNS; ++k) { b.kv_full[k] = a; a += 8; }
-    for (int k = 0; k < kNS; ++k) { b.kv_empty[k] = a; a += 8; }
+    for (int k = 0; k < kNS; ++k) { b.k_full[k] = a; a += 8; }
+    for (int k = 0; k < kNS; ++k) { b.k_empty[k] = a; a += 8; }
+    for (int k = 0; k < kNS; ++k) { b.v_full[k] = a; a += 8; }
+    for (int k = 0; k < kNS; ++k) { b.v_empty[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.s_full[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.s_free[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.p_full[k] = a; a += 8; }
@@ -106,7 +110,12 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
     // ---- set-up: barriers, TMEM, union of the block's routed + diagonal chunks --------------
     if (tid == 0) {
         tc::mbar_init(bar.q_full, 1);
-        for (int k = 0; k < kNS; ++k) { tc::mbar_init(bar.kv_full[k], 1); tc::mbar_init(bar.kv_empty[k], 1); }
+        for (int k = 0; k < kNS; ++k) {
+            tc::mbar_init(bar.k_full[k], 1);
+            tc::mbar_init(bar.k_empty[k], 1);
+            tc::mbar_init(bar.v_full[k], 1);
+            tc::mbar_init(bar.v_empty[k], 1);
+        }
         for (int k = 0; k < 2; ++k) {
             tc::mbar_init(bar.s_full[k], 1);
             tc::mbar_init(bar.s_free[k], 128);
@@ -198,26 +207,48 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 tc::tma_load_4d(base + kOffQ, &tmQ, bar.q_full, 0, r * G, i0, b);
                 tc::tma_load_4d(base + kOffQ + kQBytes / 2, &tmQ, bar.q_full, 64, r * G, i0, b);
             }
-            int last[kNS];
-            for (int k = 0; k < kNS; ++k) last[k] = -1;
-            for (int k = 0; k < njobs; ++k) {
+            // issue order K_0, K_1, V_0, K_2, V_1, ...: K runs one job ahead of V.  K_{k+1} needs
+            // S_{k-1} done, V_k needs P V_{k-2} done, and P V_{k-2} is issued before S_k, so no
+            // wait in this order blocks a load that could already go.
+            int lastk[kNS], lastv[kNS];
+            for (int k = 0; k < kNS; ++k) lastk[k] = lastv[k] = -1;
+            auto load_k = [&](int k) -> bool {
                 const int slot = k % kNS;
-                if (k >= kNS && !tc::mbar_wait(bar.kv_empty[slot], ((k / kNS) - 1) & 1, abort, err, 1)) break;
-                last[slot] = k;
+                if (k >= kNS && !tc::mbar_wait(bar.k_empty[slot], ((k / kNS) - 1) & 1, abort, err, 1)) return false;
+                lastk[slot] = k;
                 const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot;
-                tc::mbar_expect_tx(bar.kv_full[slot], kSlot);
-                tc::tma_load_4d(dst, &tmK, bar.kv_full[slot], 0, r, key0, b);
-                tc::tma_load_4d(dst + kKVHalf, &tmK, bar.kv_full[slot], 64, r, key0, b);
-                tc::tma_load_4d(dst + 2 * kKVHalf, &tmV, bar.kv_full[slot], 0, r, key0, b);
-                tc::tma_load_4d(dst + 3 * kKVHalf, &tmV, bar.kv_full[slot], 64, r, key0, b);
+                tc::mbar_expect_tx(bar.k_full[slot], 2 * kKVHalf);
+                tc::tma_load_4d(dst, &tmK, bar.k_full[slot], 0, r, key0, b);
+                tc::tma_load_4d(dst + kKVHalf, &tmK, bar.k_full[slot], 64, r, key0, b);
+                return true;
+            };
+            auto load_v = [&](int k) -> bool {
+                const int slot = k % kNS;
+                if (k >= kNS && !tc::mbar_wait(bar.v_empty[slot], ((k / kNS) - 1) & 1, abort, err, 10)) return false;
+                lastv[slot] = k;
+                const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
+                const uint32_t dst = base + kOffSlots + slot * kSlot + 2 * kKVHalf;
+                tc::mbar_expect_tx(bar.v_full[slot], 2 * kKVHalf);
+                tc::tma_load_4d(dst, &tmV, bar.v_full[slot], 0, r, key0, b);
+                tc::tma_load_4d(dst + kKVHalf, &tmV, bar.v_full[slot], 64, r, key0, b);
+                return true;
+            };
+            bool pok = load_k(0);
+            for (int k = 0; pok && k < njobs; ++k) {
+                if (k + 1 < njobs && !load_k(k + 1)) break;
+                pok = load_v(k);
             }
             if (*abort) {
                 // let this block's TMA copies still in flight land before its shared memory goes away
-                for (int k = 0; k < kNS; ++k)
-                    if (last[k] >= 0)
+                for (int k = 0; k < kNS; ++k) {
+                    if (lastk[k] >= 0)
                         for (long long it = 0; it < (1ll << 22); ++it)
-                            if (tc::mbar_try(bar.kv_full[k], (last[k] / kNS) & 1)) break;
+                            if (tc::mbar_try(bar.k_full[k], (lastk[k] / kNS) & 1)) break;
+                    if (lastv[k] >= 0)
+                        for (long long it = 0; it < (1ll << 22); ++it)
+                            if (tc::mbar_try(bar.v_full[k], (lastv[k] / kNS) & 1)) break;
+                }
                 for (long long it = 0; it < (1ll << 22); ++it)
                     if (tc::mbar_try(bar.q_full, 0)) break;
             }
@@ -229,6 +260,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             auto issue_pv = [&](int j) -> bool {
                 const int pbuf = j & 1;
                 if (!tc::mbar_wait(bar.p_full[pbuf], (j >> 1) & 1, abort, err, 2)) return false;
+                if (!tc::mbar_wait(bar.v_full[j % kNS], (j / kNS) & 1, abort, err, 13)) return false;
                 tc::fence_after_sync();
                 const uint32_t sV = base + kOffSlots + (j % kNS) * kSlot + 2 * kKVHalf;
 #pragma unroll
@@ -237,14 +269,14 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                     const uint64_t bd = tc::sw128_desc(sV + kk * 2048, kKVHalf, 1024);
                     tc::mma_f16_ts(tmem + 128, tmem + pbuf * 64 + kk * 8, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc::mma_commit(bar.kv_empty[j % kNS]);
+                tc::mma_commit(bar.v_empty[j % kNS]);
                 tc::mma_commit(bar.pv_done[pbuf]);
                 return true;
             };
             bool ok = tc::mbar_wait(bar.q_full, 0, abort, err, 3);
             for (int k = 0; ok && k < njobs; ++k) {
                 const int slot = k % kNS, sb = k & 1;
-                if (!tc::mbar_wait(bar.kv_full[slot], (k / kNS) & 1, abort, err, 4)) { ok = false; break; }
+                if (!tc::mbar_wait(bar.k_full[slot], (k / kNS) & 1, abort, err, 4)) { ok = false; break; }
                 if (k >= 2 && !tc::mbar_wait(bar.s_free[sb], ((k - 2) >> 1) & 1, abort, err, 5)) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint32_t sK = base + kOffSlots + slot * kSlot;
@@ -255,6 +287,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                     tc::mma_f16_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(bar.s_full[sb]);
+                tc::mma_commit(bar.k_empty[slot]);
                 if (k >= 1 && !issue_pv(k - 1)) { ok = false; break; }
             }
             if (ok) ok = issue_pv(njobs - 1);
