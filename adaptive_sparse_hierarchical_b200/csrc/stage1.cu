@@ -231,6 +231,34 @@ __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __
     }
 }
 
+// Threshold from a compacted candidate list: tau >= max x - 1, so entries at or below max - 1
+// never enter the support and never contribute to the mass; the warp copies the others (about a
+// sixth of a typical row) to its scratch list once and takes the Newton passes over that list.
+template <int NPL>
+__device__ float warp_threshold_compact(const float (&xr)[NPL], int nv, float alpha, float* scratch)
+{
+    const int lane = threadIdx.x & 31;
+    float mx = xr[0];
+#pragma unroll
+    for (int k = 1; k < NPL; ++k) mx = fmaxf(mx, xr[k]);
+    mx = warp_max(mx);
+    const float lo = mx - 1.f;
+    int m = 0;
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+        const bool keep = xr[k] > lo;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) scratch[m + __popc(bal & ((1u << lane) - 1u))] = xr[k];
+        m += __popc(bal);
+    }
+    __syncwarp();
+    const float t = entmax_threshold(
+        [&](auto fn) { for (int c = lane; c < m; c += 32) fn(scratch[c]); },
+        [](float& a, float& b) { a = warp_sum(a); b = warp_sum(b); }, mx, nv, alpha);
+    __syncwarp();   // scratch is reused by the warp's next row
+    return t;
+}
+
 // Register-resident threshold: row x[0..nv) with nv <= 32*NPL, NPL values per lane (-inf pads).
 template <int NPL>
 __device__ float warp_threshold_reg(const float (&xr)[NPL], int nv, float alpha)
@@ -267,6 +295,7 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
     extern __shared__ __align__(128) char smem[];
     char* kt = smem;
     float* S = reinterpret_cast<float*>(smem + 3 * PLANE);
+    float* scratch = S + ROWS * Ts + (threadIdx.x >> 5) * 512;   // per-warp candidate list
     const int G = s.g, P = ROWS / G;
     const int nblk = (s.n + P - 1) / P;
     const int br = blockIdx.x % (s.batch * s.hkv);
@@ -345,7 +374,7 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
             float xr[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) xr[k] = lane + 32 * k < nv ? x[lane + 32 * k] : -INFINITY;
-            const float tau = warp_threshold_reg<16>(xr, nv, s.alpha);
+            const float tau = warp_threshold_compact<16>(xr, nv, s.alpha, scratch);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float u = xr[k] - tau;
@@ -518,7 +547,7 @@ cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, co
 size_t route_tc_smem(const Shape& s, int RG)
 {
     const int Ts = (s.T + 31) / 32 * 32 + 8;
-    return 3 * (size_t)32 * s.d * 2 + (size_t)16 * RG * Ts * 4;
+    return 3 * (size_t)32 * s.d * 2 + (size_t)16 * RG * Ts * 4 + 8 * 512 * 4;
 }
 
 template <int D, int RG>
