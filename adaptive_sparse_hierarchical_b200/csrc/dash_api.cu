@@ -171,19 +171,19 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // bf16: Stage 0 also writes the summaries as three exact bf16 planes for Stage 1's MMAs
     __nv_bfloat16* planes = p->dtype == DASH_BF16 ? reinterpret_cast<__nv_bfloat16*>(ws + L.planes) : nullptr;
+    int* err = reinterpret_cast<int*>(ws + L.err);
     if (stage == -1 || stage == DASH_STAGE0) {
+        // a prefill starts here: clear the status word of the bounded waits
+        if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return DASH_ELAUNCH;
         rc = launch_status(launch_stage0(s, p->dtype, K, qbar, nullptr, kbar, s.T, nullptr, st, planes));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE1) {
-        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, rt, st));
+        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, rt, err, st));
         if (rc != DASH_OK) return rc;
     }
-    if (stage == -1 || stage == DASH_STAGE2) {
-        int* err = reinterpret_cast<int*>(ws + L.err);
-        if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return DASH_ELAUNCH;
+    if (stage == -1 || stage == DASH_STAGE2)
         rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt, err, st));
-    }
     return rc;
 }
 

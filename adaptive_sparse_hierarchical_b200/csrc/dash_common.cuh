@@ -98,7 +98,11 @@ cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const vo
                           float* state, int* seqlens, cudaStream_t st);
 // Stage 1 for prefill: routes of every position.
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st);
+                                 const __nv_bfloat16* planes, const Routes& rt, int* err, cudaStream_t st);
+// tcgen05 / TMEM variant of Stage 1 (bf16, d = 128, at most 512 complete chunks)
+bool route_tcgen05_supported(const Shape& s, int dtype);
+cudaError_t launch_route_prefill_tcgen05(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
+                                         int* err, cudaStream_t st);
 size_t route_prefill_smem(const Shape& s, int* positions_per_block);
 // Stage 2 for prefill.
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,

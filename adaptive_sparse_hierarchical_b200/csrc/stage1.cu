@@ -734,8 +734,10 @@ size_t route_prefill_smem(const Shape& s, int* positions_per_block)
 }
 
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st)
+                                 const __nv_bfloat16* planes, const Routes& rt, int* err, cudaStream_t st)
 {
+    if (planes && route_tcgen05_supported(s, dtype) && !legacy_stage2())
+        return launch_route_prefill_tcgen05(s, Q, planes, rt, err, st);
     if (dtype == DASH_BF16 && planes) {
         bool used = false;
         cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, planes, rt, st, &used)

@@ -81,7 +81,8 @@ typedef struct {
  * 0 on invalid params.  The workspace must be 256-byte aligned. */
 size_t dash_workspace_size(const dash_params* p, int op);
 
-/* Byte offset inside the prefill or decode workspace (op) of an int32 status word: the call clears it, and
+/* Byte offset inside the prefill or decode workspace (op) of an int32 status word: a prefill (its
+ * Stage 0) or a decode call clears it, and
  * a kernel whose bounded wait on an on-chip barrier timed out writes a non-zero code there and
  * leaves instead of hanging (read it after the stream has finished).  -1 for invalid params or
  * an op without such a word. */
