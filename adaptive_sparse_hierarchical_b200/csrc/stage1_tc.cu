@@ -13,11 +13,13 @@
 //   warp 1     allocates TMEM and issues, from one thread, X[:, tile] += Q . plane^T for the
 //              three planes (M=128, N=64, K=16 steps), so X holds the fp32 logits of every
 //              visible chunk, one row per TMEM lane
-//   warps 2-5  one thread per row: max, Newton steps on f(t)^(alpha-1) and the head weights,
-//              reading the row from TMEM in 32-column pieces (the passes are warp-uniform because
-//              tcgen05.ld is a warp instruction); the g rows of a position are g neighbouring
-//              lanes, summed by a shuffle reduce-scatter into shared memory; then one warp per
-//              position writes the ascending route list (mean log weight, bias, bitmask).
+//   warps 2-17 four warps per TMEM lane quarter (32 rows), each reading every fourth 32-column
+//              piece of its rows: max, Newton steps on f(t)^(alpha-1) and the head weights, the
+//              partial sums of a row combined in shared memory in a fixed order (the passes are
+//              warp-uniform because tcgen05.ld is a warp instruction); the g rows of a position
+//              are g neighbouring lanes, summed by a shuffle reduce-scatter into shared memory;
+//              then one warp per position writes the ascending route list (mean log weight,
+//              bias, bitmask).
 // Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
 #include <climits>
 #include <cudaTypedefs.h>
@@ -34,6 +36,7 @@ constexpr int kQB = kR * kDd * 2;               // Q tile, two 16 KB d-halves
 constexpr int kPlaneHalf = kCT * 64 * 2;        // [64 chunks][64 d] bf16 = 8 KB
 constexpr int kStage = 3 * 2 * kPlaneHalf;      // three planes x two d-halves = 48 KB
 constexpr int kOffQ1 = 0, kOffRing = kQB, kOffW = kOffRing + 2 * kStage;
+constexpr int kMisc = 128 + 3 * 4 * kR * 8;     // barriers, TMEM slot, abort flag, reduction slots
 constexpr uint32_t kIdescX = tc::idesc_bf16(128, 64, false, false);
 
 __device__ __forceinline__ float pw(float u, float p, int mode)
@@ -71,7 +74,7 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane, i
 }
 
 template <int G>
-__global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                        const __grid_constant__ CUtensorMap tmP,
                                                                        Shape s, Routes rt, int Tw, int* err)
 {
@@ -81,6 +84,7 @@ __global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __g
     constexpr int P = kR / G;
     float* wbuf = reinterpret_cast<float*>(sm + kOffW);            // [P][Tw] group sums of the head weights
     char* misc = sm + kOffW + P * Tw * 4;
+    float2* red = reinterpret_cast<float2*>(misc + 128);          // [3][4][kR] partial (f, f') / max
     const uint32_t bar0 = tc::smem_addr(misc);
     const uint32_t q_full = bar0, x_ready = bar0 + 8;
     const uint32_t full0 = bar0 + 16, empty0 = bar0 + 32;          // [2] each
@@ -183,20 +187,26 @@ __global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __g
             }
         }
     } else {
-        // ---- one thread per row ----------------------------------------------------------------
-        const int q4 = warp & 3;
+        // ---- four warps per 32 rows: warp (2 + 4 cq + q) reads TMEM lanes 32 (warp % 4) .. +31
+        // and the column pieces pc with pc % 4 == cq; partial max / f / f' of a row are combined
+        // through shared memory in a fixed order, so the four warps take identical Newton steps
+        const int q4 = warp & 3, cq = (warp - 2) >> 2;
         const int row = q4 * 32 + lane;
         const int pl = row / G;
         const int i = i0 + pl;
         const int nv = i < s.n ? min(i / s.B, s.T) : 0;
-        int nvw = nv;   // warp-uniform column bound
+        int nvw = nv;   // column bound, uniform over the warp and over the four warps of the rows
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) nvw = max(nvw, __shfl_xor_sync(0xffffffffu, nvw, o));
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
         const float xs = (s.alpha - 1.f) * s.gamma * rsqrtf((float)kDd);
         const float p = 1.f / (s.alpha - 1.f);
         const int mode = s.alpha == 2.f ? 1 : s.alpha == 1.5f ? 2 : 0;
-        const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(x_ready, 0, abort, err, 24));
+        tc::mbar_wait(x_ready, 0, abort, err, 24);
+        asm volatile("bar.sync 1, 512;" ::: "memory");
+        const bool ok = *abort == 0;   // same value in every worker: all waits ended before the barrier
+        const uint32_t gbar = 2 + q4;
+        auto group_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(gbar) : "memory"); };
         if (ok) {
             tc::fence_after_sync();
             const int npieces = (nvw + 31) / 32;
@@ -208,21 +218,25 @@ __global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __g
             };
             // row maximum
             float mx = -INFINITY;
-            for (int pc = 0; pc < npieces; ++pc) {
+            for (int pc = cq; pc < npieces; pc += 4) {
                 float v[32];
                 load_piece(pc, v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
             }
-            // Newton on g(t) = f(t)^(alpha-1) from t = max - 1 (see stage1.cu), per thread; every
-            // lane keeps stepping until the whole warp has converged
+            red[(2 * 4 + cq) * kR + row].x = mx;
+            group_sync();
+            mx = fmaxf(fmaxf(red[(2 * 4 + 0) * kR + row].x, red[(2 * 4 + 1) * kR + row].x),
+                       fmaxf(red[(2 * 4 + 2) * kR + row].x, red[(2 * 4 + 3) * kR + row].x));
+            // Newton on g(t) = f(t)^(alpha-1) from t = max - 1 (see stage1.cu); every lane keeps
+            // stepping until the whole warp has converged
             float lo = mx - 1.f;
             float hi = nv > 0 ? mx - exp2f(-(s.alpha - 1.f) * __log2f((float)nv)) : 0.f;
             float t = lo;
             bool done = nv == 0;
             for (int it = 0; it < 32 && !__all_sync(0xffffffffu, done); ++it) {
                 float f = 0.f, fd = 0.f;
-                for (int pc = 0; pc < npieces; ++pc) {
+                for (int pc = cq; pc < npieces; pc += 4) {
                     float v[32];
                     load_piece(pc, v);
 #pragma unroll
@@ -231,6 +245,12 @@ __global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __g
                         if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
                     }
                 }
+                float2* slot = red + (it & 1) * 4 * kR;
+                slot[cq * kR + row] = make_float2(f, fd);
+                group_sync();
+                const float2 r0 = slot[row], r1 = slot[kR + row], r2 = slot[2 * kR + row], r3 = slot[3 * kR + row];
+                f = (r0.x + r1.x) + (r2.x + r3.x);
+                fd = (r0.y + r1.y) + (r2.y + r3.y);
                 if (!done) {
                     fd *= p;
                     if (f >= 1.f) lo = t; else hi = t;
@@ -246,8 +266,8 @@ __global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __g
                     }
                 }
             }
-            // head weights, summed over the position's g lanes, into wbuf[pl][*]
-            for (int pc = 0; pc < npieces; ++pc) {
+            // head weights of this warp's pieces, summed over the position's g lanes, into wbuf
+            for (int pc = cq; pc < npieces; pc += 4) {
                 float v[32];
                 load_piece(pc, v);
 #pragma unroll
@@ -261,10 +281,10 @@ __global__ void __launch_bounds__(192, 1) route_prefill_tcgen05_kernel(const __g
                 for (int j = 0; j < 32 / G; ++j) wbuf[pl * Tw + pc * 32 + off + j] = v[j];
             }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 512;" ::: "memory");
         if (ok) {
             // one warp per position: GQA average, bias and the ordered route list
-            for (int pp = q4; pp < P; pp += 4) {
+            for (int pp = warp - 2; pp < P; pp += 16) {
                 const int ip = i0 + pp;
                 if (ip >= s.n) continue;
                 const int nvp = min(ip / s.B, s.T);
@@ -355,14 +375,14 @@ cudaError_t launch_g(const Shape& s, const void* Q, const __nv_bfloat16* planes,
             return cudaErrorInvalidValue;
     }
     const int Tw = (s.T + 31) / 32 * 32;
-    const size_t smem = 1024 + kOffW + (size_t)P * Tw * 4 + 128;
+    const size_t smem = 1024 + kOffW + (size_t)P * Tw * 4 + kMisc;
     auto k = route_prefill_tcgen05_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 192, smem, st>>>(mq, mp, s, rt, Tw, err);
+    k<<<grid, 576, smem, st>>>(mq, mp, s, rt, Tw, err);
     return cudaGetLastError();
 }
 
@@ -373,7 +393,7 @@ bool route_tcgen05_supported(const Shape& s, int dtype)
     if (dtype != DASH_BF16 || s.d != 128 || s.T > 512 || s.T < 1) return false;
     if (!(s.g == 1 || s.g == 2 || s.g == 4 || s.g == 8 || s.g == 16)) return false;
     const int P = kR / s.g, Tw = (s.T + 31) / 32 * 32;
-    return 1024 + kOffW + (size_t)P * Tw * 4 + 128 <= 227 * 1024 && encode_fn_r() != nullptr;
+    return 1024 + kOffW + (size_t)P * Tw * 4 + kMisc <= 227 * 1024 && encode_fn_r() != nullptr;
 }
 
 cudaError_t launch_route_prefill_tcgen05(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
