@@ -36,6 +36,8 @@ constexpr int kQB = kR * kDd * 2;               // Q tile, two 16 KB d-halves
 constexpr int kPlaneHalf = kCT * 64 * 2;        // [64 chunks][64 d] bf16 = 8 KB
 constexpr int kStage = 3 * 2 * kPlaneHalf;      // three planes x two d-halves = 48 KB
 constexpr int kOffQ1 = 0, kOffRing = kQB, kOffW = kOffRing + 2 * kStage;
+constexpr int kCand = 48;   // candidate list length per row and warp: 16 x 32 x 48 floats fill the ring
+static_assert(16 * 32 * kCand * 4 <= 2 * kStage && kCand % 4 == 0, "candidate lists must fit the ring");
 constexpr int kMisc = 128 + 3 * 4 * kR * 8;     // barriers, TMEM slot, abort flag, reduction slots
 constexpr uint32_t kIdescX = tc::idesc_bf16(128, 64, false, false);
 
@@ -209,6 +211,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
         auto group_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(gbar) : "memory"); };
         if (ok) {
             tc::fence_after_sync();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             const int npieces = (nvw + 31) / 32;
             auto load_piece = [&](int pc, float (&v)[32]) {
                 tc::tmem_ld32(lane_base + pc * 32, v);
@@ -228,21 +231,58 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
             group_sync();
             mx = fmaxf(fmaxf(red[(2 * 4 + 0) * kR + row].x, red[(2 * 4 + 1) * kR + row].x),
                        fmaxf(red[(2 * 4 + 2) * kR + row].x, red[(2 * 4 + 3) * kR + row].x));
+            // entries at or below max - 1 never enter the support (tau >= max - 1): each thread
+            // copies the others of its pieces into a list in shared memory (over the Q / plane
+            // ring, idle once X is complete; entry k of lane l at [k][l]), padded with -inf to a
+            // multiple of four; a warp whose rows overflow kCand keeps reading TMEM instead
+            float lo = mx - 1.f;
+            float* cl = reinterpret_cast<float*>(sm + kOffRing) + (warp - 2) * kCand * 32 + lane;
+            int m = 0;
+            for (int pc = cq; pc < npieces; pc += 4) {
+                float v[32];
+                load_piece(pc, v);
+                uint32_t mask = 0u;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) mask |= (v[e] > lo ? 1u : 0u) << e;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int k = m + __popc(mask & ((1u << e) - 1u));
+                    if (((mask >> e) & 1u) && k < kCand) cl[k * 32] = v[e];
+                }
+                m += __popc(mask);
+            }
+            const bool listed = __all_sync(0xffffffffu, m <= kCand);
+            const int m4 = (m + 3) >> 2;
+            for (int k = m; k < 4 * m4 && k < kCand; ++k) cl[k * 32] = -INFINITY;
             // Newton on g(t) = f(t)^(alpha-1) from t = max - 1 (see stage1.cu); every lane keeps
             // stepping until the whole warp has converged
-            float lo = mx - 1.f;
             float hi = nv > 0 ? mx - exp2f(-(s.alpha - 1.f) * __log2f((float)nv)) : 0.f;
             float t = lo;
             bool done = nv == 0;
             for (int it = 0; it < 32 && !__all_sync(0xffffffffu, done); ++it) {
                 float f = 0.f, fd = 0.f;
-                for (int pc = cq; pc < npieces; pc += 4) {
-                    float v[32];
-                    load_piece(pc, v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float u = v[e] - t;
+                if (listed && mode == 2) {
+#pragma unroll 2
+                    for (int k = 0; k < m4; ++k) {
+                        const float u0 = fmaxf(cl[(4 * k) * 32] - t, 0.f), u1 = fmaxf(cl[(4 * k + 1) * 32] - t, 0.f);
+                        const float u2 = fmaxf(cl[(4 * k + 2) * 32] - t, 0.f), u3 = fmaxf(cl[(4 * k + 3) * 32] - t, 0.f);
+                        f += u0 * u0 + u1 * u1 + u2 * u2 + u3 * u3;
+                        fd += (u0 + u1) + (u2 + u3);
+                    }
+                } else if (listed) {
+                    for (int k = 0; k < 4 * m4; ++k) {
+                        const float u = cl[k * 32] - t;
                         if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
+                    }
+                } else {
+                    for (int pc = cq; pc < npieces; pc += 4) {
+                        float v[32];
+                        load_piece(pc, v);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float u = v[e] - t;
+                            if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
+                        }
                     }
                 }
                 float2* slot = red + (it & 1) * 4 * kR;
@@ -252,7 +292,8 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
                 f = (r0.x + r1.x) + (r2.x + r3.x);
                 fd = (r0.y + r1.y) + (r2.y + r3.y);
                 if (!done) {
-                    fd *= p;
+                    // g = f^(alpha-1) has g' = -(alpha-1) f^(alpha-2) p sum u^(p-1) = -f^(alpha-2) fd,
+                    // so the Newton step (g - 1) / -g' is (g - 1) f / (g fd)
                     if (f >= 1.f) lo = t; else hi = t;
                     float tn = 0.5f * (lo + hi);
                     if (fd > 0.f && f > 0.f) {
