@@ -165,20 +165,24 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            // descriptors of the Q tile and ring stage 0; a stage / K-step moves only the start
+            // address field (16-byte units, no carry), so each MMA is issued after one add
+            const uint64_t dQ = tc::sw128_desc(base + kOffQ1, 16, 1024);
+            const uint64_t dP0 = tc::sw128_desc(base + kOffRing, 16, 1024);
             bool ok = tc::mbar_wait(q_full, 0, abort, err, 22);
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int st = t & 1;
                 if (!tc::mbar_wait(full0 + 8 * st, (t >> 1) & 1, abort, err, 23)) { ok = false; break; }
                 tc::fence_after_sync();
-                const uint32_t ring = base + kOffRing + st * kStage;
+                const uint64_t dp = dP0 + (uint64_t)((st * kStage) >> 4);
+                const uint32_t xd = tmem + t * kCT;
 #pragma unroll
                 for (int pl = 0; pl < 3; ++pl)
 #pragma unroll
-                    for (int kk = 0; kk < kDd / 16; ++kk) {
-                        const uint64_t ad = tc::sw128_desc(base + kOffQ1 + (kk >> 2) * (kQB / 2) + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = tc::sw128_desc(ring + (2 * pl + (kk >> 2)) * kPlaneHalf + (kk & 3) * 32, 16, 1024);
-                        tc::mma_f16_ss(tmem + t * kCT, ad, bd, kIdescX, (pl > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < kDd / 16; ++kk)
+                        tc::mma_f16_ss(xd, dQ + (uint64_t)(((kk >> 2) * (kQB / 2) + (kk & 3) * 32) >> 4),
+                                       dp + (uint64_t)(((2 * pl + (kk >> 2)) * kPlaneHalf + (kk & 3) * 32) >> 4), kIdescX,
+                                       (pl > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(empty0 + 8 * st);
             }
             if (ok) tc::mma_commit(x_ready);
