@@ -36,7 +36,7 @@ constexpr int kTmemCols = 256;                    // S0 [0,64), S1 [64,128), O [
 constexpr int kOffQ = 0, kOffSlots = kQBytes;
 constexpr int kOffScratch = kOffSlots;            // set-up scratch (chunk bitmask, sort keys) in the ring
 constexpr int kOffBar = kOffSlots + kNS * kSlot;  // 98304: two blocks fit on one SM
-constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 2 + 2 + 1;
+constexpr int kNumBars = 1 + 2 * kNS + 2 + 2 + 2 + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, njobs
 constexpr int kOffPos = kOffMisc + 32;             // the block's positions (<= 16 when clustered)
 constexpr int kOffJobs = kOffPos + 4 * kRows;
@@ -52,10 +52,13 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// K and V of a slot have their own barriers.  With as many slots as S buffers (2), slot k % 2 holds
+// job k's K until S_k is done and its V until P V_k is done, so the producer waits on s_full and
+// pv_done themselves (two commits per job); neither can run a phase ahead of the producer's wait,
+// since the next phase needs the load it has yet to issue.
+static_assert(kNS == 2, "slot k % kNS must be S buffer k % 2");
 struct Bars {
-    // K and V of a slot have their own barriers: K is free once S = Q K^T is done, V only after P V
-    uint32_t q_full, k_full[kNS], k_empty[kNS], v_full[kNS], v_empty[kNS], s_full[2], s_free[2], p_full[2],
-        pv_done[2], drain;
+    uint32_t q_full, k_full[kNS], v_full[kNS], s_full[2], s_free[2], p_full[2], pv_done[2], drain;
 };
 
 __device__ __forceinline__ Bars make_bars(uint32_t base)
@@ -64,9 +67,7 @@ __device__ __forceinline__ Bars make_bars(uint32_t base)
     uint32_t a = base + kOffBar;
     b.q_full = a; a += 8;
     for (int k = 0; k < kNS; ++k) { b.k_full[k] = a; a += 8; }
-    for (int k = 0; k < kNS; ++k) { b.k_empty[k] = a; a += 8; }
     for (int k = 0; k < kNS; ++k) { b.v_full[k] = a; a += 8; }
-    for (int k = 0; k < kNS; ++k) { b.v_empty[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.s_full[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.s_free[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.p_full[k] = a; a += 8; }
@@ -112,9 +113,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         tc::mbar_init(bar.q_full, 1);
         for (int k = 0; k < kNS; ++k) {
             tc::mbar_init(bar.k_full[k], 1);
-            tc::mbar_init(bar.k_empty[k], 1);
             tc::mbar_init(bar.v_full[k], 1);
-            tc::mbar_init(bar.v_empty[k], 1);
         }
         for (int k = 0; k < 2; ++k) {
             tc::mbar_init(bar.s_full[k], 1);
@@ -214,7 +213,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             for (int k = 0; k < kNS; ++k) lastk[k] = lastv[k] = -1;
             auto load_k = [&](int k) -> bool {
                 const int slot = k % kNS;
-                if (k >= kNS && !tc::mbar_wait(bar.k_empty[slot], ((k / kNS) - 1) & 1, abort, err, 1)) return false;
+                if (k >= kNS && !tc::mbar_wait(bar.s_full[slot], ((k / kNS) - 1) & 1, abort, err, 1)) return false;
                 lastk[slot] = k;
                 const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot;
@@ -225,7 +224,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             };
             auto load_v = [&](int k) -> bool {
                 const int slot = k % kNS;
-                if (k >= kNS && !tc::mbar_wait(bar.v_empty[slot], ((k / kNS) - 1) & 1, abort, err, 10)) return false;
+                if (k >= kNS && !tc::mbar_wait(bar.pv_done[slot], ((k / kNS) - 1) & 1, abort, err, 10)) return false;
                 lastv[slot] = k;
                 const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot + 2 * kKVHalf;
@@ -256,20 +255,22 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
     } else if (warp == 1) {
         // ---- MMA issuer --------------------------------------------------------------------
         if (lane == 0 && njobs > 0) {
-            const uint32_t sQ = base + kOffQ;
+            // descriptors of Q and slot 0; a slot / K-step moves only the start-address field
+            // (16-byte units, no carry), so each MMA is issued after one add
+            const uint64_t dQ = tc::sw128_desc(base + kOffQ, 16, 1024);
+            const uint64_t dK0 = tc::sw128_desc(base + kOffSlots, 16, 1024);
+            const uint64_t dV0 = tc::sw128_desc(base + kOffSlots + 2 * kKVHalf, kKVHalf, 1024);
             auto issue_pv = [&](int j) -> bool {
                 const int pbuf = j & 1;
                 if (!tc::mbar_wait(bar.p_full[pbuf], (j >> 1) & 1, abort, err, 2)) return false;
                 if (!tc::mbar_wait(bar.v_full[j % kNS], (j / kNS) & 1, abort, err, 13)) return false;
                 tc::fence_after_sync();
-                const uint32_t sV = base + kOffSlots + (j % kNS) * kSlot + 2 * kKVHalf;
+                const uint64_t dv = dV0 + (uint64_t)(((j % kNS) * kSlot) >> 4);
+                // P_j (bf16, 2 per column) sits in the first 32 columns of S buffer pbuf
+                tc::mma_f16_ts(tmem + 128, tmem + pbuf * 64, dv, kIdescPV, j > 0 ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk) {
-                    // P_j (bf16, 2 per column) sits in the first 32 columns of S buffer pbuf
-                    const uint64_t bd = tc::sw128_desc(sV + kk * 2048, kKVHalf, 1024);
-                    tc::mma_f16_ts(tmem + 128, tmem + pbuf * 64 + kk * 8, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc::mma_commit(bar.v_empty[j % kNS]);
+                for (int kk = 1; kk < kKT / 16; ++kk)
+                    tc::mma_f16_ts(tmem + 128, tmem + pbuf * 64 + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV, 1u);
                 tc::mma_commit(bar.pv_done[pbuf]);
                 return true;
             };
@@ -279,15 +280,12 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 if (!tc::mbar_wait(bar.k_full[slot], (k / kNS) & 1, abort, err, 4)) { ok = false; break; }
                 if (k >= 2 && !tc::mbar_wait(bar.s_free[sb], ((k - 2) >> 1) & 1, abort, err, 5)) { ok = false; break; }
                 tc::fence_after_sync();
-                const uint32_t sK = base + kOffSlots + slot * kSlot;
+                const uint64_t dk = dK0 + (uint64_t)((slot * kSlot) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t ad = tc::sw128_desc(sQ + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = tc::sw128_desc(sK + (kk >> 2) * kKVHalf + (kk & 3) * 32, 16, 1024);
-                    tc::mma_f16_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    tc::mma_f16_ss(tmem + sb * 64, dQ + (uint64_t)(((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4),
+                                   dk + (uint64_t)(((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4), kIdescS, kk > 0 ? 1u : 0u);
                 tc::mma_commit(bar.s_full[sb]);
-                tc::mma_commit(bar.k_empty[slot]);
                 if (k >= 1 && !issue_pv(k - 1)) { ok = false; break; }
             }
             if (ok) ok = issue_pv(njobs - 1);
