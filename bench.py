@@ -29,6 +29,11 @@ METRIC = "prefill Mtok/s and decode µs/token at 32K–128K ctx; % of HBM / bf16
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes per launch of the Stage 2 tcgen05 kernel (dram__bytes_read.sum + dram__bytes_write.sum
+# from one ncu capture of the current kernel on that workload); reset to absent when the kernel
+# changes and the capture has not been repeated.
+STAGE2_TRAFFIC = {"prefill_32k": 313.6e6}
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -203,7 +208,9 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind):
         "routed_fraction": float(counts.sum()) / (wl.batch * wl.h_kv * sum(i // wl.chunk for i in range(wl.n))),
         "roofline": {"kernel": ("attend_prefill_mma_kernel (mma.sync)" if os.environ.get("DASH_STAGE2", "").startswith("m")
                                else "attend_prefill_tc_kernel (tcgen05)"), "bound": "tensor", "achieved": achieved,
-                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": (STAGE2_TRAFFIC.get(wl.name) if not os.environ.get("DASH_STAGE2", "").startswith("m")
+                                 else None),
                      "peak_kind": f"bf16 dense burst, of {pk_kind}",
                      "flops_per_launch": flops, "launch_ms": stage_ms[2]},
         "clocks": clk.summary(),
