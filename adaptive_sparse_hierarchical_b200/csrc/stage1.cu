@@ -14,6 +14,8 @@
 // number of bisection steps narrows that bracket to about 1e-6 of its width, then Newton steps
 // from the left end (the tangent of a convex decreasing function stays below it, so the steps
 // never pass the root) finish to float precision.
+#include <cstdlib>
+
 #include "dash_common.cuh"
 #include "stage2_mma.cuh"
 
@@ -754,6 +756,13 @@ cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const
 cudaError_t launch_route_decode(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
                                 const int* seqlens, const Routes& rt, float* X, cudaStream_t st)
 {
+    // DASH_DEC_ROUTE=heads keeps the per-head kernels below (the long-context path) for comparison
+    static const bool per_head = [] {
+        const char* e = getenv("DASH_DEC_ROUTE");
+        return e && e[0] == 'h';
+    }();
+    if (!per_head && dec_route_cluster_supported(s, kbar_T))
+        return launch_route_decode_cluster(s, dtype, q, kbar, kbar_T, seqlens, rt, st);
     if (dtype == DASH_BF16)
         return s.d == 128 ? dec_route_t<__nv_bfloat16, 128>(s, q, kbar, kbar_T, seqlens, rt, X, st)
                           : dec_route_t<__nv_bfloat16, 64>(s, q, kbar, kbar_T, seqlens, rt, X, st);

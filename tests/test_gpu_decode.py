@@ -1,6 +1,10 @@
 """GPU parity of incremental decoding (dash_summary_build / dash_summary_append / dash_decode
 through the C ABI) against the float64 oracle: summary cache, incomplete-chunk state, routes and
 outputs, step after step."""
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -29,9 +33,25 @@ def _state(x, lengths, capacity, *, chunk, alpha, gamma, dtype, inv_sigma=1.0):
     counts = torch.zeros((b, hkv), dtype=torch.int32, device="cuda")
     idx = torch.zeros((b, hkv, max(capacity // chunk, 1)), dtype=torch.int32, device="cuda")
     bias = torch.zeros((b, hkv, max(capacity // chunk, 1)), dtype=torch.float32, device="cuda")
-    st.route = D.route_out(counts, idx, bias)
+    words = (capacity // chunk + 31) // 32
+    bm = torch.full((b, hkv, max(words, 1)), -1, dtype=torch.int32, device="cuda")   # all bits set: must be rewritten
+    st.route = D.route_out(counts, idx, bias, bm)
     st.rt = (counts, idx, bias)
+    st.bm = bm
     return st
+
+
+def _check_bitmask(st):
+    """The bitmask output holds exactly the chunks of the route list (32 chunks per word)."""
+    counts, idx, _ = (t.cpu().numpy() for t in st.rt)
+    bm = st.bm.cpu().numpy().view(np.uint32)
+    b, hkv, words = bm.shape
+    for bb in range(b):
+        for r in range(hkv):
+            want = np.zeros(words * 32, dtype=bool)
+            want[idx[bb, r, :counts[bb, r]]] = True
+            got = ((bm[bb, r][:, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(bool).reshape(-1)
+            assert np.array_equal(got, want), (bb, r)
 
 
 def _check_summaries(st, x, chunk):
@@ -62,6 +82,7 @@ def _check_step(st, x, q, lengths, *, chunk, alpha, gamma, dtype, inv_sigma=1.0)
     pos = (np.asarray(lengths) - 1).reshape(b, 1)
     # oracle route arrays are [b, hkv, 1, T']; pad T' to the cache's chunk count
     mism, _ = check_routes(gs, rt, chunk, pos, T)
+    _check_bitmask(st)
     return check_outputs(O[:, None], oref[:, None], dtype, hq // hkv, mism, rt, chunk, pos, T)
 
 
@@ -155,3 +176,15 @@ def test_decode_long_run_is_deterministic():
     assert torch.equal(runs[0], runs[1])
     last = lengths + 300
     _check_step(st, x, x["Q"][np.arange(b), last - 1], last, chunk=B, alpha=1.5, gamma=5.0, dtype="bf16")
+
+
+def test_decode_per_head_routing_kernels():
+    """The per-head decode routing kernels (used when a group's logits do not fit the cluster
+    kernel's shared memory, i.e. very long contexts) selected by DASH_DEC_ROUTE=heads: the small
+    decode cases pass through them too."""
+    env = dict(os.environ, DASH_DEC_ROUTE="heads")
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-x",
+                        os.path.join(here, "test_gpu_decode.py"), "-k", "test_decode_steps_small"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
