@@ -52,6 +52,37 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions: one issue slot for two lanes of arithmetic) and
+// the three-input maximum: the softmax below is bound by instruction issue.
+__device__ __forceinline__ unsigned long long f2(float a, float b)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void unf2(unsigned long long r, float& a, float& b)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long fadd2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // K and V of a slot have their own barriers.  With as many slots as S buffers (2), slot k % 2 holds
 // job k's K until S_k is done and its V until P V_k is done, so the producer waits on s_full and
 // pv_done themselves (two commits per job); neither can run a phase ahead of the producer's wait,
@@ -343,16 +374,15 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 for (int e = 0; e < 64; ++e)
                     if (j0 + e > i) v[e] = -INFINITY;
             }
-            // tile maximum of the biased logits: max over raw scores (tree), then scale (scale2 > 0)
+            // tile maximum of the biased logits: max over raw scores (three-input tree), then scale
+            // (scale2 > 0)
             float mx8[8];
 #pragma unroll
-            for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(v[a], v[a + 8]);
-#pragma unroll
-            for (int e = 16; e < 64; e += 8)
-#pragma unroll
-                for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], v[e + a]);
-            const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int a = 0; a < 8; ++a) {
+                const float t1 = fmax3(v[a], v[a + 8], v[a + 16]), t2 = fmax3(v[a + 24], v[a + 32], v[a + 40]);
+                mx8[a] = fmax3(fmax3(v[a + 48], v[a + 56], t1), t2, t2);
+            }
+            const float smax = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
             const float mt = bias2 == -INFINITY ? -INFINITY : fmaf(smax, scale2, bias2);
             const bool need = (m != -INFINITY) && (mt > m + 8.f);
             if (m == -INFINITY) m = mt;
@@ -387,21 +417,28 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 tc::tmem_st16(pdst + 16, z);
             } else {
                 const float off = bias2 - (m == -INFINITY ? 0.f : m);
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                // pairs of columns in f32x2: x = s * scale2 + off, then 2^x per lane, the running
+                // sums in two packed accumulators
+                const unsigned long long sc2 = f2(scale2, scale2), off2 = f2(off, off);
+                unsigned long long ls2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(fmaf(v[32 * half + 2 * e], scale2, off));
-                        const float p1 = ex2_approx(fmaf(v[32 * half + 2 * e + 1], scale2, off));
-                        ls[e & 3] += p0 + p1;
+                        float x0, x1;
+                        unf2(ffma2(f2(v[32 * half + 2 * e], v[32 * half + 2 * e + 1]), sc2, off2), x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        ls2[e & 1] = fadd2(ls2[e & 1], f2(p0, p1));
                         __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t*>(&t2);
                     }
                     tc::tmem_st16(pdst + 16 * half, pk);
                 }
-                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                float a0, a1, b0, b1;
+                unf2(ls2[0], a0, a1);
+                unf2(ls2[1], b0, b1);
+                l += (a0 + a1) + (b0 + b1);
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
