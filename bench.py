@@ -240,8 +240,58 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind):
     nbytes = lambda t: t.numel() * t.element_size()
     out["e2e"] = {"value": ranks.world * tokens / (ems / 1e3) / 1e6, "unit": "Mtok/s", "ms_per_step": ems,
                   "h2d_bytes_per_step": sum(nbytes(hq[k]) for k in hq), "d2h_bytes_per_step": nbytes(ho)}
+    out["dense_causal"] = dense_denominators(wl, tq, qbar, pf, steps, flush, ms, dev)
     out["_inputs"] = x
     return out
+
+
+def dense_denominators(wl, tq, qbar, pf, steps, flush, sparse_ms, dev):
+    """Same-box dense causal attention on the same Q, K, V (context for the sparse step, not part
+    of `value`): (a) this library at gamma = 0, where every visible chunk is routed with bias 0 and
+    the method reduces to dense causal attention; (b) torch's scaled_dot_product_attention."""
+    import torch
+    import adaptive_sparse_hierarchical_b200 as D
+
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        tot = 0.0
+        for k in range(n):
+            flush.fill_(k & 0xff)
+            a, b = ev(), ev()
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            tot += a.elapsed_time(b)
+        return tot / n
+
+    res = {}
+    pfd = D.Prefill(tq["Q"], tq["K"], tq["V"], qbar, chunk=wl.chunk, alpha=wl.alpha, gamma=0.0,
+                    inv_sigma=wl.inv_sigma)
+    res["own_kernels_gamma0_ms"] = timed(pfd, steps)
+    res["own_stage2_gamma0_ms"] = timed(lambda: pfd.stage(2), steps)
+    del pfd
+    try:
+        import torch.nn.functional as F
+        q = tq["Q"].transpose(1, 2).contiguous()
+        k = tq["K"].transpose(1, 2).contiguous()
+        v = tq["V"].transpose(1, 2).contiguous()
+        res["torch_sdpa_ms"] = timed(lambda: F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True),
+                                     steps)
+        del q, k, v
+    except Exception as e:   # pragma: no cover - backend availability differs by build
+        res["torch_sdpa_ms"] = None
+        res["torch_sdpa_error"] = str(e)[:200]
+    res["sparse_step_ms"] = sparse_ms
+    res["speedup_vs_own_dense"] = res["own_kernels_gamma0_ms"] / sparse_ms
+    if res.get("torch_sdpa_ms"):
+        res["speedup_vs_torch_sdpa"] = res["torch_sdpa_ms"] / sparse_ms
+    return res
 
 
 # ---------------------------------------------------------------------------------------- decode
@@ -415,7 +465,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, planted chunks; see DESIGN.md)",
             "config": config_of(wl, args), "roofline": pre["roofline"], "e2e": pre["e2e"],
             "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "stages_ms": pre["stages_ms"],
-            "routed_fraction": pre["routed_fraction"]}
+            "routed_fraction": pre["routed_fraction"], "dense_causal": pre["dense_causal"]}
     if not args.no_decode:
         line["decode"] = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind)
         line["gpu_launches"] += line["decode"]["gpu_launches"]
