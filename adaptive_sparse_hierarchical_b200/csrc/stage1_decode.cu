@@ -55,15 +55,21 @@ __host__ __device__ inline size_t route_cluster_smem(int g, int per)
     return ((size_t)g * per + (size_t)slots * kRanks * per) * 4;
 }
 
-// (hi, mid, lo) bf16 pairs with hi + mid + lo == (x0, x1) exactly (8 + 8 + 8 significand bits)
+// (hi, mid, lo) bf16 pairs with hi + mid + lo == (x0, x1) exactly, by truncation: hi keeps the
+// top 8 significand bits of x, r = x - hi is exact and has at most 16, mid keeps r's top 8 and
+// lo = r - mid the remaining 8 (all exactly representable in bf16).  Integer masks, subtractions
+// and byte permutes only.
 __device__ __forceinline__ void split3(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo)
 {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-    const float r0 = x0 - __bfloat162float(h0), r1 = x1 - __bfloat162float(h1);
-    const __nv_bfloat16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
-    hi = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-    mid = pack_bf16(__bfloat162float(m0), __bfloat162float(m1));
-    lo = pack_bf16(r0 - __bfloat162float(m0), r1 - __bfloat162float(m1));
+    const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffff0000u);
+    const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffff0000u);
+    const float r0 = x0 - h0, r1 = x1 - h1;
+    const float m0 = __uint_as_float(__float_as_uint(r0) & 0xffff0000u);
+    const float m1 = __uint_as_float(__float_as_uint(r1) & 0xffff0000u);
+    const float l0 = r0 - m0, l1 = r1 - m1;
+    hi = __byte_perm(__float_as_uint(h0), __float_as_uint(h1), 0x7632);
+    mid = __byte_perm(__float_as_uint(m0), __float_as_uint(m1), 0x7632);
+    lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
 }
 
 template <typename T, int D>
