@@ -54,6 +54,8 @@ def args_():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=16384)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the 64K sparsity sweep and the 128K alpha x chunk-size sweep (one line each)")
     return ap.parse_args()
 
 
@@ -153,12 +155,12 @@ def stage2_routed_flops(counts, n, B, g, d, hq):
     return 4.0 * d * (float(counts.sum()) * B * g + counts.shape[0] * hq * diag)
 
 
-def run_prefill(wl, steps, warmup, ranks, pk, pk_kind):
+def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
     import torch
     import adaptive_sparse_hierarchical_b200 as D
 
     dev = torch.device("cuda", ranks.local)
-    x = wl.make()
+    x = wl.make() if x is None else x
     tq = {k: torch.from_numpy(x[k]).to(dev, torch.bfloat16) for k in ("Q", "K", "V")}
     qbar = torch.from_numpy(x["qbar"]).to(dev)
     pf = D.Prefill(tq["Q"], tq["K"], tq["V"], qbar, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
@@ -216,6 +218,14 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind):
         "clocks": clk.summary(),
         "gpu_launches": 3 * steps,
     }
+    if lite:   # sweep mode: the device-timed step and the per-row support only
+        c = counts.reshape(-1, wl.n)[:, wl.chunk:].astype("float64")
+        vis = (np.arange(wl.n) // wl.chunk)[wl.chunk:].astype("float64")
+        frac = (c / vis).reshape(-1)
+        out["support_fraction_deciles"] = [round(float(v), 4) for v in np.quantile(frac, np.linspace(0.1, 0.9, 9))]
+        out["support_chunks_deciles"] = [int(v) for v in np.quantile(c.reshape(-1), np.linspace(0.1, 0.9, 9))]
+        del pf
+        return out
     # e2e: host (pinned) inputs copied in, result copied out, every step, through the public API.
     # Two device buffer sets and three streams (copy in, compute, copy out): step k+1's inputs
     # cross PCIe while step k computes and step k-1's output comes back; every copy of every step
@@ -468,6 +478,34 @@ def config_of(wl, args):
             "l2": "flushed between steps (256 MB write, outside the per-step events)"}
 
 
+def run_sweep(args, ranks, pk, pk_kind):
+    """The 8B-class 64K prefill at 50 / 25 / 12.5% routed and the 128K alpha x chunk-size sweep on
+    Gaussian-mixture inputs: per workload the device-timed step, Mtok/s, Stage 2 roofline and the
+    per-row support (routed chunks / visible chunks) deciles.  Inputs shared by several workloads
+    are drawn once."""
+    import gc
+    from adaptive_sparse_hierarchical_b200 import workloads as W
+
+    cache = {}
+    for name in W.PREFILL_64K + W.SWEEP_128K:
+        wl = W.get(name)
+        key = (wl.recipe, wl.extra.get("seed"), wl.batch, wl.n, wl.h_q, wl.h_kv, wl.d)
+        if key not in cache:
+            cache.clear()
+            gc.collect()
+            cache[key] = wl.make()
+        r = run_prefill(wl, args.steps, args.warmup, ranks, pk, pk_kind, x=cache[key], lite=True)
+        line = {"sweep": name, "metric": "prefill Mtok/s", "value": r["value"], "unit": "Mtok/s",
+                "ms_per_step": r["ms_per_step"], "stages_ms": r["stages_ms"], "routed_fraction": r["routed_fraction"],
+                "stage2_roofline_frac": r["roofline"]["frac"], "stage2_routed_tflops": r["roofline"]["achieved"],
+                "support_fraction_deciles": r["support_fraction_deciles"],
+                "support_chunks_deciles": r["support_chunks_deciles"], "clocks": r["clocks"],
+                "config": {"batch": wl.batch, "seq_len": wl.n, "h_q": wl.h_q, "h_kv": wl.h_kv, "d_h": wl.d,
+                           "chunk": wl.chunk, "alpha": wl.alpha, "gamma": wl.gamma}}
+        if ranks.rank == 0:
+            print(json.dumps(line), flush=True)
+
+
 def main():
     args = args_()
     if args.impl == "reference":
@@ -484,6 +522,10 @@ def main():
     ranks = Ranks()
     torch.cuda.set_device(ranks.local)
     pk, pk_kind = peaks()
+    if args.sweep:
+        run_sweep(args, ranks, pk, pk_kind)
+        ranks.close()
+        return
     wl = W.get(args.workload)
     pre = run_prefill(wl, args.steps, args.warmup, ranks, pk, pk_kind)
     x = pre.pop("_inputs")
