@@ -110,15 +110,21 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
         const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(q) + ((long long)b * s.hq + r * G) * D;
         load_q_frags<D>(qf, [&](int h) -> const __nv_bfloat16* { return h < G ? qb + (long long)h * D : nullptr; });
         const int g8 = lane >> 2, t4 = lane & 3;
-        for (int nt = warp; nt * 8 < nloc; nt += kThr / 32) {
+        // the next tile's fragments are loaded while the current tile is computed
+        float2 u[D / 16][2], un[D / 16][2];
+        auto load_tile = [&](int nt, float2 (&dst)[D / 16][2]) {
             const int row = nt * 8 + g8;
+            const bool ok = nt * 8 < nloc && row < nloc;
             const float* kr = kb + (long long)row * D + 2 * t4;
-            float2 u[D / 16][2];
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                u[kk][0] = row < nloc ? __ldg(reinterpret_cast<const float2*>(kr + kk * 16)) : make_float2(0.f, 0.f);
-                u[kk][1] = row < nloc ? __ldg(reinterpret_cast<const float2*>(kr + kk * 16 + 8)) : make_float2(0.f, 0.f);
+                dst[kk][0] = ok ? __ldg(reinterpret_cast<const float2*>(kr + kk * 16)) : make_float2(0.f, 0.f);
+                dst[kk][1] = ok ? __ldg(reinterpret_cast<const float2*>(kr + kk * 16 + 8)) : make_float2(0.f, 0.f);
             }
+        };
+        load_tile(warp, u);
+        for (int nt = warp; nt * 8 < nloc; nt += kThr / 32) {
+            load_tile(nt + kThr / 32, un);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -135,6 +141,8 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
                 const int h = g8 + (e >> 1) * 8, cc = c + (e & 1);
                 if (h < G && cc < nloc) xsm[h * per + cc] = acc[e] * xs;
             }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) { u[kk][0] = un[kk][0]; u[kk][1] = un[kk][1]; }
         }
     } else {
         for (int v = tid; v < G * D; v += kThr) qs[v] = to_f(q[((long long)b * s.hq + r * G) * D + v]) * xs;
