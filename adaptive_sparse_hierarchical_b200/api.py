@@ -124,7 +124,15 @@ class DecodeState:
         serves every step."""
         if getattr(self, "_graph", None) is None:
             out = self.step(q, k_new, v_new)
-            self._qs, self._ks, self._vs = q.clone(), k_new.clone(), v_new.clone()
+            # one staging buffer holding q, k, v back to back (graph_step_packed fills it at once)
+            self._stage = torch.empty(q.numel() + k_new.numel() + v_new.numel(), dtype=q.dtype, device=q.device)
+            nq, nk = q.numel(), k_new.numel()
+            self._qs = self._stage[:nq].view(q.shape)
+            self._ks = self._stage[nq:nq + nk].view(k_new.shape)
+            self._vs = self._stage[nq + nk:].view(v_new.shape)
+            self._qs.copy_(q)
+            self._ks.copy_(k_new)
+            self._vs.copy_(v_new)
             self._graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(self._graph):
                 self.append(self._ks, self._vs)
@@ -133,5 +141,17 @@ class DecodeState:
         self._qs.copy_(q)
         self._ks.copy_(k_new)
         self._vs.copy_(v_new)
+        self._graph.replay()
+        return self.O
+
+    @staticmethod
+    def pack(q, k_new, v_new):
+        """q, k, v of one step in the layout graph_step_packed takes (flattened, back to back)."""
+        return torch.cat([q.reshape(-1), k_new.reshape(-1), v_new.reshape(-1)])
+
+    def graph_step_packed(self, qkv):
+        """graph_step with the step's q, k, v already packed (pack()): one copy in, then replay.
+        The graph must exist (one graph_step call first)."""
+        self._stage.copy_(qkv)
         self._graph.replay()
         return self.O

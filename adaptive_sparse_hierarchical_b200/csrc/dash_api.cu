@@ -248,8 +248,7 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
     dw.x = reinterpret_cast<float*>(ws + L.x);
     dw.part = reinterpret_cast<float*>(ws + L.part);
     dw.splits = L.splits;
-    dw.err = reinterpret_cast<int*>(ws + L.err);
-    if (cudaMemsetAsync(dw.err, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess) return DASH_ELAUNCH;
+    dw.err = reinterpret_cast<int*>(ws + L.err);   // cleared by the routing launch
     return launch_status(launch_decode(s, p->dtype, q, K_cache, V_cache, kbar_cache, s.T, seqlens, O, rt, dw,
                                        static_cast<cudaStream_t>(stream)));
 }

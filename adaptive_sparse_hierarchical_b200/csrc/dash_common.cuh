@@ -125,13 +125,14 @@ bool dec_tma_supported(const Shape& s, int dtype);
 int dec_tma_blocks();   // persistent blocks (the SM count); partial slots per pair
 cudaError_t launch_dec_attend_tma(const Shape& s, const void* q, const void* Kc, const void* Vc, const int* seqlens,
                                   const Routes& rt, float* part, void* O, int* err, cudaStream_t st);
+// status: the decode call's status word, set to 0 by the routing launch before later kernels run
 cudaError_t launch_route_decode(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
-                                const int* seqlens, const Routes& rt, float* X, cudaStream_t st);
+                                const int* seqlens, const Routes& rt, float* X, int* status, cudaStream_t st);
 // Decode Stage 1 in one launch (8-block clusters per (sequence, KV head); g <= 16, d = 64 / 128).
 int dec_route_cluster_per(int kbar_T);
 bool dec_route_cluster_supported(const Shape& s, int kbar_T);
 cudaError_t launch_route_decode_cluster(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
-                                        const int* seqlens, const Routes& rt, cudaStream_t st);
+                                        const int* seqlens, const Routes& rt, int* status, cudaStream_t st);
 cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* Kc, const void* Vc,
                           const float* kbar, int kbar_T, const int* seqlens, void* O,
                           const Routes& rt, const DecodeWs& ws, cudaStream_t st);

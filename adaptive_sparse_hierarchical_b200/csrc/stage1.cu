@@ -754,7 +754,7 @@ cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const
 }
 
 cudaError_t launch_route_decode(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
-                                const int* seqlens, const Routes& rt, float* X, cudaStream_t st)
+                                const int* seqlens, const Routes& rt, float* X, int* status, cudaStream_t st)
 {
     // DASH_DEC_ROUTE=heads keeps the per-head kernels below (the long-context path) for comparison
     static const bool per_head = [] {
@@ -762,7 +762,8 @@ cudaError_t launch_route_decode(const Shape& s, int dtype, const void* q, const 
         return e && e[0] == 'h';
     }();
     if (!per_head && dec_route_cluster_supported(s, kbar_T))
-        return launch_route_decode_cluster(s, dtype, q, kbar, kbar_T, seqlens, rt, st);
+        return launch_route_decode_cluster(s, dtype, q, kbar, kbar_T, seqlens, rt, status, st);
+    if (status && cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return cudaGetLastError();
     if (dtype == DASH_BF16)
         return s.d == 128 ? dec_route_t<__nv_bfloat16, 128>(s, q, kbar, kbar_T, seqlens, rt, X, st)
                           : dec_route_t<__nv_bfloat16, 64>(s, q, kbar, kbar_T, seqlens, rt, X, st);

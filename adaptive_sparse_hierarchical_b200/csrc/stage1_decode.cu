@@ -75,8 +75,10 @@ __device__ __forceinline__ void split3(float x0, float x1, uint32_t& hi, uint32_
 template <typename T, int D>
 __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
     dec_route_cluster_kernel(Shape s, const T* __restrict__ q, const float* __restrict__ kbar, int kbar_T,
-                             const int* __restrict__ seqlens, Routes rt, int per)
+                             const int* __restrict__ seqlens, Routes rt, int per, int* status)
 {
+    // the step's status word starts at 0 here (the later kernels of the step may set it)
+    if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
     extern __shared__ __align__(16) float dyn[];
     __shared__ __align__(16) float qs[kMaxG * D];
     __shared__ Cross cx;
@@ -333,7 +335,7 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
 
 template <typename T, int D>
 cudaError_t launch_t(const Shape& s, const void* q, const float* kbar, int kbar_T, const int* seqlens,
-                     const Routes& rt, cudaStream_t st)
+                     const Routes& rt, int* status, cudaStream_t st)
 {
     const int per = dec_route_cluster_per(kbar_T);
     const size_t smem = route_cluster_smem(s.g, per);
@@ -342,7 +344,7 @@ cudaError_t launch_t(const Shape& s, const void* q, const float* kbar, int kbar_
         const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k<<<kRanks * s.batch * s.hkv, kThr, smem, st>>>(s, (const T*)q, kbar, kbar_T, seqlens, rt, per);
+    k<<<kRanks * s.batch * s.hkv, kThr, smem, st>>>(s, (const T*)q, kbar, kbar_T, seqlens, rt, per, status);
     return cudaGetLastError();
 }
 
@@ -362,13 +364,13 @@ bool dec_route_cluster_supported(const Shape& s, int kbar_T)
 }
 
 cudaError_t launch_route_decode_cluster(const Shape& s, int dtype, const void* q, const float* kbar, int kbar_T,
-                                        const int* seqlens, const Routes& rt, cudaStream_t st)
+                                        const int* seqlens, const Routes& rt, int* status, cudaStream_t st)
 {
     if (dtype == DASH_BF16)
-        return s.d == 128 ? launch_t<__nv_bfloat16, 128>(s, q, kbar, kbar_T, seqlens, rt, st)
-                          : launch_t<__nv_bfloat16, 64>(s, q, kbar, kbar_T, seqlens, rt, st);
-    return s.d == 128 ? launch_t<float, 128>(s, q, kbar, kbar_T, seqlens, rt, st)
-                      : launch_t<float, 64>(s, q, kbar, kbar_T, seqlens, rt, st);
+        return s.d == 128 ? launch_t<__nv_bfloat16, 128>(s, q, kbar, kbar_T, seqlens, rt, status, st)
+                          : launch_t<__nv_bfloat16, 64>(s, q, kbar, kbar_T, seqlens, rt, status, st);
+    return s.d == 128 ? launch_t<float, 128>(s, q, kbar, kbar_T, seqlens, rt, status, st)
+                      : launch_t<float, 64>(s, q, kbar, kbar_T, seqlens, rt, status, st);
 }
 
 }  // namespace dash

@@ -483,7 +483,7 @@ cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* 
                           const float* kbar, int kbar_T, const int* seqlens, void* O, const Routes& rt,
                           const DecodeWs& ws, cudaStream_t st)
 {
-    cudaError_t e = launch_route_decode(s, dtype, q, kbar, kbar_T, seqlens, rt, ws.x, st);
+    cudaError_t e = launch_route_decode(s, dtype, q, kbar, kbar_T, seqlens, rt, ws.x, ws.err, st);
     if (e != cudaSuccess) return e;
     if (dec_tma_supported(s, dtype) && !legacy_stage2()) {
         e = launch_dec_attend_tma(s, q, Kc, Vc, seqlens, rt, ws.part, O, ws.err, st);

