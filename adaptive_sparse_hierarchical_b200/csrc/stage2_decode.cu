@@ -308,75 +308,46 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     }
 }
 
-// Merge of the per-block partials of each pair: one block per (pair, head).  The blocks that
-// touched pair br are those whose tile range meets [P[br], P[br+1]).
+// Merge of the per-block partials of each pair: one block per (pair, head), one thread per
+// column.  Every thread finds the pair's blocks and the common maximum / sum itself (the few
+// partial (m, l) values are broadcast loads), so the merge is one chain of loads, no barrier.
 template <int D>
-__global__ void __launch_bounds__(128) dec_merge_kernel(Shape s, const float* __restrict__ part, int nblocks,
-                                                        Routes rt, __nv_bfloat16* __restrict__ O)
+__global__ void __launch_bounds__(D) dec_merge_kernel(Shape s, const float* __restrict__ part, int nblocks,
+                                                      Routes rt, __nv_bfloat16* __restrict__ O)
 {
-    __shared__ float wk[1024];
-    __shared__ float red[4];
-    __shared__ int range[2];
-    __shared__ long long span[3];   // total tiles, this pair's first and one-past-last tile
     const int x = blockIdx.x / s.g, row = blockIdx.x % s.g, G = s.g, NH = s.B / 64;
-    const int b = x / s.hkv, r = x % s.hkv;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) {
-        long long acc = 0, lo = 0, hi = 0;
-        for (int y = 0; y < s.batch * s.hkv; ++y) {
-            if (y == x) lo = acc;
-            acc += (long long)(rt.counts[y] + 1) * NH;
-            if (y == x) hi = acc;
-        }
-        // blocks c with [acc*c/n, acc*(c+1)/n) meeting [lo, hi)
-        int c0 = (int)((lo * nblocks) / acc), c1 = (int)(((hi - 1) * nblocks) / acc);
-        while (c0 > 0 && acc * c0 / nblocks > lo) --c0;
-        while (c0 < nblocks - 1 && acc * (c0 + 1) / nblocks <= lo) ++c0;
-        while (c1 < nblocks - 1 && acc * (c1 + 1) / nblocks <= hi - 1) ++c1;
-        while (c1 > 0 && acc * c1 / nblocks > hi - 1) --c1;
-        range[0] = c0;
-        range[1] = c1;
-        span[0] = acc;
-        span[1] = lo;
-        span[2] = hi;
+    const int b = x / s.hkv, r = x % s.hkv, col = threadIdx.x;
+    long long lo = 0, total = 0;
+    for (int y = 0; y < s.batch * s.hkv; ++y) {
+        const long long c = (long long)(rt.counts[y] + 1) * NH;
+        if (y < x) lo += c;
+        total += c;
     }
-    __syncthreads();
-    // a block wrote a partial for this pair iff its tile range meets the pair's tiles
-    auto valid_block = [&](int c) {
-        const long long a = span[0] * c / nblocks, e = span[0] * (c + 1) / nblocks;
-        return (a > span[1] ? a : span[1]) < (e < span[2] ? e : span[2]);
-    };
-    const int c0 = range[0], nsp = range[1] - range[0] + 1;
-    const float* basep = part + ((long long)x * nblocks + c0) * G * 130 + (long long)row * 130;
+    const long long hi = lo + (long long)(rt.counts[x] + 1) * NH;
+    // block c covers tiles [total c / n, total (c+1) / n); it wrote a partial for this pair iff
+    // that range is nonempty and meets [lo, hi)
+    auto jlo = [&](int c) { return total * c / nblocks; };
+    int c0 = (int)(lo * nblocks / total), c1 = (int)((hi - 1) * nblocks / total);
+    while (c0 > 0 && jlo(c0) > lo) --c0;
+    while (c0 + 1 < nblocks && jlo(c0 + 1) <= lo) ++c0;
+    while (c1 + 1 < nblocks && jlo(c1 + 1) <= hi - 1) ++c1;
+    while (c1 > 0 && jlo(c1) > hi - 1) --c1;
+    const bool all_nonempty = total >= nblocks;
+    const float* basep = part + (long long)x * nblocks * G * 130 + (long long)row * 130;
     const long long sstride = (long long)G * 130;
     float M = -INFINITY;
-    for (int k = tid; k < nsp; k += blockDim.x) if (valid_block(c0 + k)) M = fmaxf(M, basep[k * sstride + 128]);
-    M = warp_max(M);
-    if (lane == 0) red[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    float Lsum = 0.f;
-    for (int k = tid; k < nsp; k += blockDim.x) {
-        float w = 0.f;
-        if (valid_block(c0 + k)) {
-            const float mk = basep[k * sstride + 128];
-            w = mk == -INFINITY ? 0.f : exp2f(mk - M);
-            Lsum += basep[k * sstride + 129] * w;
-        }
-        wk[k] = w;
+    for (int c = c0; c <= c1; ++c)
+        if (all_nonempty || jlo(c) < jlo(c + 1)) M = fmaxf(M, basep[c * sstride + 128]);
+    float Lsum = 0.f, o = 0.f;
+    for (int c = c0; c <= c1; ++c) {
+        if (!(all_nonempty || jlo(c) < jlo(c + 1))) continue;
+        const float mk = basep[c * sstride + 128];
+        if (mk == -INFINITY) continue;
+        const float w = exp2f(mk - M);
+        Lsum += basep[c * sstride + 129] * w;
+        o += basep[c * sstride + col] * w;
     }
-    Lsum = warp_sum(Lsum);
-    if (lane == 0) red[warp] = Lsum;
-    __syncthreads();
-    Lsum = red[0] + red[1] + red[2] + red[3];
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    for (int col = tid; col < D; col += blockDim.x) {
-        float o = 0.f;
-        for (int k = 0; k < nsp; ++k)
-            if (wk[k] != 0.f) o += basep[k * sstride + col] * wk[k];
-        O[((long long)b * s.hq + r * G + row) * D + col] = __float2bfloat16_rn(o * inv);
-    }
+    O[((long long)b * s.hq + r * G + row) * D + col] = __float2bfloat16_rn(Lsum > 0.f ? o / Lsum : 0.f);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn_d()
