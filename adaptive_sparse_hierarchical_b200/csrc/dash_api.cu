@@ -61,7 +61,7 @@ long long route_cap(const dash_params* p)
     return tri_offset(p->seqlen, p->chunk);
 }
 
-struct PrefillLayout { size_t kbar, counts, idx, bias, err, planes, total; };
+struct PrefillLayout { size_t kbar, counts, idx, bias, err, planes, redo, total; };
 PrefillLayout prefill_layout(const dash_params* p)
 {
     PrefillLayout L;
@@ -74,7 +74,8 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.bias = L.idx + up(bh * cap * 4);
     L.err = L.bias + up(bh * cap * 4);
     L.planes = L.err + kAlign;
-    L.total = L.planes + up(bh * 3 * T * p->d_h * 2);
+    L.redo = L.planes + up(bh * 3 * T * p->d_h * 2);
+    L.total = L.redo + up(bh * (size_t)p->seqlen);   // one flag per position block at most
     return L;
 }
 
@@ -179,7 +180,8 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE1) {
-        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, rt, err, st));
+        unsigned char* redo = reinterpret_cast<unsigned char*>(ws + L.redo);
+        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, rt, redo, err, st));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE2)

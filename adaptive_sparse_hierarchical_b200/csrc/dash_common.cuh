@@ -97,13 +97,22 @@ cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const vo
                           const float* qbar, void* Kc, void* Vc, float* kbar, int kbar_T,
                           float* state, int* seqlens, cudaStream_t st);
 // Stage 1 for prefill: routes of every position.
+// redo: one byte per (sequence, KV head, position block) for the long-row kernel's overflow flags
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const __nv_bfloat16* planes, const Routes& rt, int* err, cudaStream_t st);
+                                 const __nv_bfloat16* planes, const Routes& rt, unsigned char* redo, int* err,
+                                 cudaStream_t st);
 // tcgen05 / TMEM variant of Stage 1 (bf16, d = 128, at most 512 complete chunks)
 bool route_tcgen05_supported(const Shape& s, int dtype);
 cudaError_t launch_route_prefill_tcgen05(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
                                          int* err, cudaStream_t st);
 size_t route_prefill_smem(const Shape& s, int* positions_per_block);
+// tcgen05 variant for rows of more than 512 chunks (bf16, d = 128, g in {4, 8, 16}): blocks of
+// route_long_positions(s) positions; a block whose candidate lists overflow sets its redo byte
+// and writes nothing, and launch_route_prefill recomputes those blocks with the kernels above.
+bool route_long_supported(const Shape& s, int dtype);
+int route_long_positions(const Shape& s);
+cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
+                                      unsigned char* redo, int* err, cudaStream_t st);
 // Stage 2 for prefill.
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,
                                   const void* V, void* O, const Routes& rt, int* err, cudaStream_t st);

@@ -117,6 +117,18 @@ __device__ void warp_emit(WF wsum, int nv, float inv_g, float inv_sigma, int* id
     if (lane == 0) *count = base;
 }
 
+// A block of positions [i0, ilast] is recomputed only where the long-row kernel flagged one of
+// the position blocks (redo_p positions each) that it overlaps; redo == null runs every block.
+__device__ __forceinline__ bool redo_wanted(const unsigned char* redo, int redo_p, const Shape& s, int br, int i0,
+                                            int ilast)
+{
+    if (!redo) return true;
+    const unsigned char* rr = redo + (long long)br * ((s.n + redo_p - 1) / redo_p);
+    for (int tb = i0 / redo_p; tb <= ilast / redo_p; ++tb)
+        if (rr[tb]) return true;
+    return false;
+}
+
 // ------------------------------------------------------------------------------------------
 // Prefill: one block per (sequence, KV head, block of P positions); rows = P * g query rows.
 // Shared memory: scaled query rows [rows][D], one summary tile [32][D+4], logits [rows][Ts].
@@ -124,7 +136,8 @@ __device__ void warp_emit(WF wsum, int nv, float inv_g, float inv_sigma, int* id
 template <typename T, int D>
 __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __restrict__ Q,
                                                             const float* __restrict__ kbar,
-                                                            Routes rt, int P, int Ts)
+                                                            Routes rt, int P, int Ts,
+                                                            const unsigned char* redo, int redo_p)
 {
     extern __shared__ float4 smem4[];
     float* qsm = reinterpret_cast<float*>(smem4);
@@ -143,6 +156,7 @@ __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __
     int* idx = rt.idx + (long long)br * rt.cap;
     float* bias = rt.bias + (long long)br * rt.cap;
     uint32_t* bm = rt.bitmask ? rt.bitmask + (long long)br * s.n * rt.words : nullptr;
+    if (!redo_wanted(redo, redo_p, s, br, i0, ilast)) return;
 
     if (nvmax == 0) {
         for (int p = tid; p < P && i0 + p < s.n; p += blockDim.x) counts[i0 + p] = 0;
@@ -289,7 +303,8 @@ __device__ float warp_threshold_reg(const float (&xr)[NPL], int nv, float alpha)
 template <int D, int RG>
 __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __nv_bfloat16* __restrict__ Q,
                                                                const __nv_bfloat16* __restrict__ planes,
-                                                               Routes rt, int Ts)
+                                                               Routes rt, int Ts,
+                                                               const unsigned char* redo, int redo_p)
 {
     constexpr int ROWS = 16 * RG;
     constexpr int TCH = 32;                    // chunks per staged tile
@@ -311,6 +326,7 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
     int* idx = rt.idx + (long long)br * rt.cap;
     float* bias = rt.bias + (long long)br * rt.cap;
     uint32_t* bm = rt.bitmask ? rt.bitmask + (long long)br * s.n * rt.words : nullptr;
+    if (!redo_wanted(redo, redo_p, s, br, i0, ilast)) return;
     if (nvmax == 0) {
         for (int p = tid; p < P && i0 + p < s.n; p += blockDim.x) counts[i0 + p] = 0;
         if (bm)
@@ -529,7 +545,7 @@ __global__ void __launch_bounds__(512) dec_route_kernel(Shape s, int kbar_T, con
 
 template <typename T, int D>
 cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, const Routes& rt,
-                            cudaStream_t st)
+                            cudaStream_t st, const unsigned char* redo = nullptr, int redo_p = 1)
 {
     int P = 0;
     const size_t smem = route_prefill_smem(s, &P);
@@ -541,7 +557,7 @@ cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, co
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 256, smem, st>>>(s, (const T*)Q, kbar, rt, P, Ts);
+    k<<<grid, 256, smem, st>>>(s, (const T*)Q, kbar, rt, P, Ts, redo, redo_p);
     return cudaGetLastError();
 }
 
@@ -553,7 +569,8 @@ size_t route_tc_smem(const Shape& s, int RG)
 }
 
 template <int D, int RG>
-cudaError_t route_tc_t(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st)
+cudaError_t route_tc_t(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st,
+                       const unsigned char* redo, int redo_p)
 {
     const size_t smem = route_tc_smem(s, RG);
     const int Ts = (s.T + 31) / 32 * 32 + 8;
@@ -564,18 +581,18 @@ cudaError_t route_tc_t(const Shape& s, const void* Q, const __nv_bfloat16* plane
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, planes, rt, Ts);
+    k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, planes, rt, Ts, redo, redo_p);
     return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t route_tc_d(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
-                       cudaStream_t st, bool* used)
+                       cudaStream_t st, bool* used, const unsigned char* redo = nullptr, int redo_p = 1)
 {
     constexpr size_t kLimit = 225 * 1024;
     *used = true;
-    if (32 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, planes, rt, st);
-    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, planes, rt, st);
+    if (32 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, planes, rt, st, redo, redo_p);
+    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, planes, rt, st, redo, redo_p);
     *used = false;
     return cudaSuccess;
 }
@@ -735,19 +752,40 @@ size_t route_prefill_smem(const Shape& s, int* positions_per_block)
     return bytes;
 }
 
+// DASH_LONG_ROUTE=off keeps rows of more than 512 chunks on the per-shape kernels (for comparison)
+static bool long_route_off()
+{
+    static const bool off = [] {
+        const char* v = getenv("DASH_LONG_ROUTE");
+        return v && v[0] == 'o';
+    }();
+    return off;
+}
+
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const __nv_bfloat16* planes, const Routes& rt, int* err, cudaStream_t st)
+                                 const __nv_bfloat16* planes, const Routes& rt, unsigned char* redo, int* err,
+                                 cudaStream_t st)
 {
     if (planes && route_tcgen05_supported(s, dtype) && !legacy_stage2())
         return launch_route_prefill_tcgen05(s, Q, planes, rt, err, st);
+    // rows of more than 512 chunks: the long-row tcgen05 kernel, then the kernels below only for
+    // the position blocks whose candidate lists overflowed
+    const unsigned char* mask = nullptr;
+    int mask_p = 1;
+    if (planes && redo && route_long_supported(s, dtype) && !legacy_stage2() && !long_route_off()) {
+        cudaError_t e = launch_route_prefill_long(s, Q, planes, rt, redo, err, st);
+        if (e != cudaSuccess) return e;
+        mask = redo;
+        mask_p = route_long_positions(s);
+    }
     if (dtype == DASH_BF16 && planes) {
         bool used = false;
-        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, planes, rt, st, &used)
-                                   : route_tc_d<64>(s, Q, planes, rt, st, &used);
+        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, planes, rt, st, &used, mask, mask_p)
+                                   : route_tc_d<64>(s, Q, planes, rt, st, &used, mask, mask_p);
         if (used) return e;
         // very long rows (T * 16 rows of logits beyond shared memory): CUDA-core variant
-        return s.d == 128 ? route_prefill_t<__nv_bfloat16, 128>(s, Q, kbar, rt, st)
-                          : route_prefill_t<__nv_bfloat16, 64>(s, Q, kbar, rt, st);
+        return s.d == 128 ? route_prefill_t<__nv_bfloat16, 128>(s, Q, kbar, rt, st, mask, mask_p)
+                          : route_prefill_t<__nv_bfloat16, 64>(s, Q, kbar, rt, st, mask, mask_p);
     }
     return s.d == 128 ? route_prefill_t<float, 128>(s, Q, kbar, rt, st)
                       : route_prefill_t<float, 64>(s, Q, kbar, rt, st);

@@ -92,6 +92,38 @@ def test_ragged_shapes(case):
     compare(x, pf, O, chunk=B, alpha=alpha, gamma=gamma, inv_sigma=inv_sigma, dtype=dtype)
 
 
+LONG_CASES = [
+    # n, hq, hkv, B, gamma, alpha, batch: rows of more than 512 chunks (the long-row routing kernel
+    # with its overflow fallback); the last case has weak logits, so that many position blocks'
+    # candidate lists overflow and are recomputed by the per-shape kernels
+    (9000, 8, 2, 16, 6.0, 1.5, 1),
+    (12000, 16, 2, 16, 8.0, 2.0, 1),
+    (17000, 16, 1, 32, 6.0, 1.25, 1),
+    (10000, 8, 2, 16, 1.0, 1.5, 2),
+]
+
+
+@pytest.mark.parametrize("case", LONG_CASES, ids=[f"n{c[0]}_g{c[1] // c[2]}_B{c[3]}_a{c[5]}_gam{c[4]}" for c in LONG_CASES])
+def test_long_rows(case):
+    n, hq, hkv, B, gamma, alpha, batch = case
+    x = inputs.planted(21, batch, n, hq, hkv, 128, B, dtype="bf16", chunk_frac=0.1, strength=2.0)
+    O, pf = run_prefill(x, chunk=B, alpha=alpha, gamma=gamma)
+    pos = _sample_positions(n, B, 160, 3)
+    compare(x, pf, O, chunk=B, alpha=alpha, gamma=gamma, positions=pos)
+
+
+def test_long_rows_gamma_zero_routes_everything():
+    """gamma = 0 with 600 chunks: every row's candidate lists overflow, every position block is
+    recomputed by the fallback kernels, and every visible chunk is routed with zero bias."""
+    n, B = 9600, 16
+    x = inputs.planted(22, 1, n, 8, 2, 128, B, dtype="bf16")
+    O, pf = run_prefill(x, chunk=B, alpha=1.5, gamma=0.0)
+    cnt = pf.counts.cpu().numpy()[0]
+    assert np.array_equal(cnt, np.broadcast_to(np.arange(n) // B, cnt.shape))
+    # equal weights: log w - mean log w is zero up to the rounding of the mean
+    assert float(pf.bias.abs().max()) < 1e-5
+
+
 @pytest.mark.parametrize("n", [1, 2, 63, 64, 65])
 def test_degenerate_lengths(n):
     """Single token, sequences shorter than one chunk, exactly one chunk and one past it."""
