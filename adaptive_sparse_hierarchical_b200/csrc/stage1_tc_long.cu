@@ -63,15 +63,17 @@ __device__ __forceinline__ float dpw(float u, float p, int mode)
     return mode == 1 ? 1.f : mode == 2 ? u : exp2f((p - 1.f) * __log2f(u));
 }
 
-// Root of f_S(t) = sum_{x in S} [x - t]_+^p = 1 over a subset S of a row's logits: this thread's
-// list (entry k at cl[32 k], m entries) and three more values (the other column sets' maxima).  f_S <= f everywhere, so the root is a lower
-// bound on the row's tau.  Starts from t0 (a known lower bound); returns -inf when f_S(t0) < 1 (no
-// tighter bound from this subset).
-__device__ __noinline__ float subset_root(const float* cl, int m, float om0, float om1, float om2, float t0,
-                                          float t_hi, float p, int mode, float am1)
+// Lower bound on the root of f_S(t) = sum_{x in S} [x - t]_+^p = 1 over a subset S of a row's
+// logits: this thread's list (entry k at cl[32 k], m entries) and three more values (the other
+// column sets' maxima).  f_S <= f everywhere, so that root is itself a lower bound on the row's
+// tau.  g = f_S^(alpha-1) is convex and decreasing (a p-norm of the [x - t]_+), so Newton steps
+// on g taken from a point left of its root stay left of it: three steps from t0 (where f_S >= 1)
+// give a bound good enough to cut a list; -inf when f_S(t0) < 1 (nothing to gain).
+__device__ __noinline__ float subset_bound(const float* cl, int m, float om0, float om1, float om2, float t0,
+                                           float p, int mode, float am1)
 {
-    float lo = t0, hi = t_hi, t = t0;
-    for (int it = 0; it < 40; ++it) {
+    float t = t0;
+    for (int it = 0; it < 3; ++it) {
         float f = 0.f, fd = 0.f;
         for (int k = 0; k < m; ++k) {
             const float u = cl[32 * k] - t;
@@ -83,18 +85,14 @@ __device__ __noinline__ float subset_root(const float* cl, int m, float om0, flo
             const float u = om[j] - t;
             if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
         }
-        if (it == 0 && f < 1.f) return -INFINITY;
-        if (f >= 1.f) lo = t; else hi = t;
-        float tn = 0.5f * (lo + hi);
-        if (fd > 0.f && f > 0.f) {
-            const float gg = mode == 2 ? sqrtf(f) : mode == 1 ? f : exp2f(am1 * __log2f(f));
-            tn = t + (gg - 1.f) * f / (gg * fd);
-        }
-        if (fabsf(tn - t) <= 2e-7f * fmaxf(1.f, fabsf(t)) || fabsf(f - 1.f) <= 1e-6f) return tn;
-        if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+        if (f < 1.f) return it == 0 ? -INFINITY : t;
+        if (!(fd > 0.f)) break;
+        const float gg = mode == 2 ? sqrtf(f) : mode == 1 ? f : exp2f(am1 * __log2f(f));
+        const float tn = t + (gg - 1.f) * f / (gg * fd);
+        if (!(tn > t)) break;
         t = tn;
     }
-    return lo;   // f_S(lo) >= 1: still a lower bound
+    return t;
 }
 
 // Sum over the g neighbouring lanes of a position of 32 values, reduce-scattered: afterwards
@@ -347,7 +345,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                             if (m + __popc(mask) > cap && m <= cap) {
                                 // list full: raise the cut to this thread's subset bound on tau
                                 // (less the margin below) and drop the entries under it
-                                const float tb = subset_root(cl, m, om[0], om[1], om[2], lo_t, mx, p, mode, s.alpha - 1.f);
+                                const float tb = subset_bound(cl, m, om[0], om[1], om[2], lo_t, p, mode, s.alpha - 1.f);
                                 const float cut = tb - 1e-3f * fmaxf(1.f, fabsf(tb));
                                 if (cut > lo_t) {
                                     lo_t = cut;
@@ -362,12 +360,14 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                                     for (int e = 0; e < 32; ++e) mask |= (v[e] > lo_t ? 1u : 0u) << e;
                                 }
                             }
+                            if (mask) {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const int kk = m + __popc(mask & ((1u << e) - 1u));
-                                if (((mask >> e) & 1u) && kk < cap) cl[kk * 32] = v[e];
+                                for (int e = 0; e < 32; ++e) {
+                                    const int kk = m + __popc(mask & ((1u << e) - 1u));
+                                    if (((mask >> e) & 1u) && kk < cap) cl[kk * 32] = v[e];
+                                }
+                                m += __popc(mask);
                             }
-                            m += __popc(mask);
                         } else {
 #pragma unroll
                             for (int e = 0; e < 32; ++e) {
