@@ -107,6 +107,9 @@ __device__ __forceinline__ Bars make_bars(uint32_t base)
     return b;
 }
 
+// CPT = chunks per 64-key tile: 1 for chunks of 64 or 128 keys (a chunk is one or two jobs), 2 for
+// 32-key chunks (a job covers two neighbouring chunks, each row with its own bias per half).
+template <int CPT>
 __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                    const __grid_constant__ CUtensorMap tmQ1,
                                                                    const __grid_constant__ CUtensorMap tmK,
@@ -137,7 +140,8 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
     const int* ridx = rt.idx + (long long)br * rt.cap;
     const float* rbias = rt.bias + (long long)br * rt.cap;
     const int W = (s.T + 32) >> 5;
-    const int NH = s.B / kKT;
+    const int NH = CPT == 1 ? s.B / kKT : 1;   // jobs per union unit (chunk, or 64-key tile)
+    const int UB = CPT == 1 ? s.B : kKT;       // keys per union unit
 
     // ---- set-up: barriers, TMEM, union of the block's routed + diagonal chunks --------------
     if (tid == 0) {
@@ -187,8 +191,14 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         if (i >= s.n) continue;
         const int cnt = counts[i];
         const int* li = ridx + tri_offset(i, s.B);
-        for (int k = tid; k < cnt; k += blockDim.x) atomicOr(&umask[li[k] >> 5], 1u << (li[k] & 31));
-        if (tid == 0) atomicOr(&umask[(i / s.B) >> 5], 1u << ((i / s.B) & 31));
+        for (int k = tid; k < cnt; k += blockDim.x) {
+            const int u = li[k] / CPT;
+            atomicOr(&umask[u >> 5], 1u << (u & 31));
+        }
+        if (tid == 0) {
+            const int u = (i / s.B) / CPT;
+            atomicOr(&umask[u >> 5], 1u << (u & 31));
+        }
     }
     __syncthreads();
     if (warp == 0) {   // ordered bitmask -> list of chunk ids
@@ -246,7 +256,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 const int slot = k % kNS;
                 if (k >= kNS && !tc::mbar_wait(bar.s_full[slot], ((k / kNS) - 1) & 1, abort, err, 1)) return false;
                 lastk[slot] = k;
-                const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
+                const int key0 = jobs[k / NH] * UB + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot;
                 tc::mbar_expect_tx(bar.k_full[slot], 2 * kKVHalf);
                 tc::tma_load_4d(dst, &tmK, bar.k_full[slot], 0, r, key0, b);
@@ -257,7 +267,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 const int slot = k % kNS;
                 if (k >= kNS && !tc::mbar_wait(bar.pv_done[slot], ((k / kNS) - 1) & 1, abort, err, 10)) return false;
                 lastv[slot] = k;
-                const int key0 = jobs[k / NH] * s.B + (k % NH) * kKT;
+                const int key0 = jobs[k / NH] * UB + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot + 2 * kKVHalf;
                 tc::mbar_expect_tx(bar.v_full[slot], 2 * kKVHalf);
                 tc::tma_load_4d(dst, &tmV, bar.v_full[slot], 0, r, key0, b);
@@ -345,6 +355,12 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         float nbias = cnt > 0 ? lb[0] : 0.f;
         int nxt2 = cnt > 1 ? li[1] : INT_MAX;
         float nbias2 = cnt > 1 ? lb[1] : 0.f;
+        // two chunks per job: entries cur+2, cur+3 as well, and the queue only shifts at the end
+        // of a job, so no compare waits on a load issued in the same job
+        int nxt3 = CPT > 1 && cnt > 2 ? li[2] : INT_MAX;
+        float nbias3 = CPT > 1 && cnt > 2 ? lb[2] : 0.f;
+        int nxt4 = CPT > 1 && cnt > 3 ? li[3] : INT_MAX;
+        float nbias4 = CPT > 1 && cnt > 3 ? lb[3] : 0.f;
         const float scale2 = kLog2e * rsqrtf((float)kD);
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
         float m = -INFINITY, l = 0.f;
@@ -361,12 +377,26 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             tc::fence_before_sync();
             tc::mbar_arrive(bar.s_free[sb]);
             const int c = jobs[k / NH];
-            const int j0 = c * s.B + (k % NH) * kKT;
-            float bias2 = -INFINITY;
+            const int j0 = c * UB + (k % NH) * kKT;
+            float bias2 = -INFINITY, bias2b = -INFINITY;   // per 32-key half (equal when CPT == 1)
             bool causal = false;
-            if (valid) {
-                if (nxt == c) bias2 = nbias * kLog2e;
-                else if (c == diag) { bias2 = 0.f; causal = j0 + kKT - 1 > i; }
+            int adv = 0;   // entries of the row's list consumed by this job (CPT > 1)
+            if (CPT == 1) {
+                if (valid) {
+                    if (nxt == c) bias2 = nbias * kLog2e;
+                    else if (c == diag) { bias2 = 0.f; causal = j0 + kKT - 1 > i; }
+                }
+                bias2b = bias2;
+            } else if (valid) {
+                const int c0 = c * 2, c1 = c0 + 1;
+                const bool m0 = nxt == c0;
+                const int nn = m0 ? nxt2 : nxt;
+                const float nb = m0 ? nbias2 : nbias;
+                const bool m1 = nn == c1;
+                bias2 = m0 ? nbias * kLog2e : c0 == diag ? 0.f : -INFINITY;
+                bias2b = m1 ? nb * kLog2e : c1 == diag ? 0.f : -INFINITY;
+                causal = (c0 == diag || c1 == diag) && j0 + kKT - 1 > i;
+                adv = (m0 ? 1 : 0) + (m1 ? 1 : 0);
             }
             if (causal) {
                 // diagonal tile: keys past the query are masked
@@ -382,8 +412,22 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 const float t1 = fmax3(v[a], v[a + 8], v[a + 16]), t2 = fmax3(v[a + 24], v[a + 32], v[a + 40]);
                 mx8[a] = fmax3(fmax3(v[a + 48], v[a + 56], t1), t2, t2);
             }
-            const float smax = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-            const float mt = bias2 == -INFINITY ? -INFINITY : fmaf(smax, scale2, bias2);
+            float mt;
+            if (CPT == 1) {
+                const float smax = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+                mt = bias2 == -INFINITY ? -INFINITY : fmaf(smax, scale2, bias2);
+            } else {
+                // the two halves' maxima (columns 0-31 and 32-63), each with its own bias
+                float ha = -INFINITY, hb = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    ha = fmax3(ha, v[e], v[e + 1]);
+                    hb = fmax3(hb, v[32 + e], v[32 + e + 1]);
+                }
+                const float ma = bias2 == -INFINITY ? -INFINITY : fmaf(ha, scale2, bias2);
+                const float mb = bias2b == -INFINITY ? -INFINITY : fmaf(hb, scale2, bias2b);
+                mt = fmaxf(ma, mb);
+            }
             const bool need = (m != -INFINITY) && (mt > m + 8.f);
             if (m == -INFINITY) m = mt;
             if (__any_sync(0xffffffffu, need)) {
@@ -409,20 +453,22 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             // the first 32 columns of this job's S buffer.  A warp whose rows all skip the tile
             // writes zeros without computing.
             const uint32_t pdst = lane_base + sb * 64;
-            if (__all_sync(0xffffffffu, bias2 == -INFINITY)) {
+            if (__all_sync(0xffffffffu, bias2 == -INFINITY && bias2b == -INFINITY)) {
                 uint32_t z[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) z[e] = 0u;
                 tc::tmem_st16(pdst, z);
                 tc::tmem_st16(pdst + 16, z);
             } else {
-                const float off = bias2 - (m == -INFINITY ? 0.f : m);
+                const float mref = m == -INFINITY ? 0.f : m;
                 // pairs of columns in f32x2: x = s * scale2 + off, then 2^x per lane, the running
                 // sums in two packed accumulators
-                const unsigned long long sc2 = f2(scale2, scale2), off2 = f2(off, off);
+                const unsigned long long sc2 = f2(scale2, scale2);
                 unsigned long long ls2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
+                    const float off = (half == 0 ? bias2 : bias2b) - mref;
+                    const unsigned long long off2 = f2(off, off);
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -443,12 +489,29 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(bar.p_full[sb]);
-            if (k % NH == NH - 1 && nxt == c) {
+            if (CPT == 1) {
+                if (k % NH == NH - 1 && nxt == c) {
+                    ++cur;
+                    nxt = nxt2;
+                    nbias = nbias2;
+                    nxt2 = cur + 1 < cnt ? li[cur + 1] : INT_MAX;
+                    nbias2 = cur + 1 < cnt ? lb[cur + 1] : 0.f;
+                }
+            } else if (adv == 1) {
                 ++cur;
-                nxt = nxt2;
-                nbias = nbias2;
-                nxt2 = cur + 1 < cnt ? li[cur + 1] : INT_MAX;
-                nbias2 = cur + 1 < cnt ? lb[cur + 1] : 0.f;
+                nxt = nxt2; nbias = nbias2;
+                nxt2 = nxt3; nbias2 = nbias3;
+                nxt3 = nxt4; nbias3 = nbias4;
+                nxt4 = cur + 3 < cnt ? li[cur + 3] : INT_MAX;
+                nbias4 = cur + 3 < cnt ? lb[cur + 3] : 0.f;
+            } else if (adv == 2) {
+                cur += 2;
+                nxt = nxt3; nbias = nbias3;
+                nxt2 = nxt4; nbias2 = nbias4;
+                nxt3 = cur + 2 < cnt ? li[cur + 2] : INT_MAX;
+                nbias3 = cur + 2 < cnt ? lb[cur + 2] : 0.f;
+                nxt4 = cur + 3 < cnt ? li[cur + 3] : INT_MAX;
+                nbias4 = cur + 3 < cnt ? lb[cur + 3] : 0.f;
             }
         }
         // ---- epilogue: O / l -> bf16 --------------------------------------------------------
@@ -537,15 +600,18 @@ bool make_map(CUtensorMap* map, const void* ptr, int batch, int n, int heads, co
 
 }  // namespace
 
+// union units (chunks, or 64-key tiles of two 32-key chunks) a block's job list may hold
+int attend_units(const Shape& s) { return (s.B >= kKT ? s.T : s.T / 2) + 2; }
+
 bool attend_tc_supported(const Shape& s, int dtype)
 {
-    return dtype == DASH_BF16 && s.d == 128 && (s.B == 64 || s.B == 128) && s.g >= 1 && s.g <= 16 &&
-           (kRows % s.g) == 0 && encode_fn() != nullptr && (s.T + 2) * 4 <= 16 * 1024;
+    return dtype == DASH_BF16 && s.d == 128 && (s.B == 32 || s.B == 64 || s.B == 128) && s.g >= 1 && s.g <= 16 &&
+           (kRows % s.g) == 0 && encode_fn() != nullptr && attend_units(s) * 4 <= 16 * 1024;
 }
 
 size_t attend_tc_smem(const Shape& s)
 {
-    return 1024 + kOffJobs + (size_t)(s.T + 2) * 4;
+    return 1024 + kOffJobs + (size_t)attend_units(s) * 4;
 }
 
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
@@ -558,12 +624,13 @@ cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* 
         !make_map(&mk, K, s.batch, s.n, s.hkv, s.ks, 1, kKT) || !make_map(&mv, V, s.batch, s.n, s.hkv, s.vs, 1, kKT))
         return cudaErrorInvalidValue;
     const size_t smem = attend_tc_smem(s);
-    cudaError_t e = cudaFuncSetAttribute(attend_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = s.B >= kKT ? attend_prefill_tc_kernel<1> : attend_prefill_tc_kernel<2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    attend_prefill_tc_kernel<<<grid, 192, smem, st>>>(mq, mq1, mk, mv, s, rt, (__nv_bfloat16*)O, err, cluster);
+    kern<<<grid, 192, smem, st>>>(mq, mq1, mk, mv, s, rt, (__nv_bfloat16*)O, err, cluster);
     return cudaGetLastError();
 }
 

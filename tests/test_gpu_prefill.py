@@ -81,6 +81,10 @@ CASES = [
     (640, 16, 16, 128, 64, 7.0, 1.75, 1.0, "bf16"),
     (600, 8, 2, 128, 32, 6.0, 1.5, 1.0, "f32"),
     (300, 4, 1, 64, 16, 6.0, 2.0, 2.0, "f32"),
+    # 32-key chunks at d = 128: the tensor-core Stage 2 with two chunks per 64-key tile
+    (1000, 8, 2, 128, 32, 6.0, 1.5, 1.0, "bf16"),
+    (700, 16, 1, 128, 32, 7.0, 2.0, 0.5, "bf16"),
+    (1100, 4, 2, 128, 32, 3.0, 1.25, 1.0, "bf16"),
 ]
 
 
