@@ -37,6 +37,30 @@ __host__ __device__ inline long long tri_offset(int i, int B)
     return (long long)B * (c * (c - 1) / 2) + (long long)(i - c * B) * c;
 }
 
+// Programmatic dependent launch: a kernel launched with launch_after() may start while the
+// previous kernel of the stream still runs; it calls pdl_wait() (every thread, before any early
+// exit) ahead of its first access to that kernel's results, so completion stays transitive along
+// the stream.  pdl_launch_dependents() lets the next such kernel start early.  Both are no-ops
+// for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... P, typename... A>
+inline cudaError_t launch_after(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, A... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 __device__ __forceinline__ float warp_sum(float v)
 {
 #pragma unroll

@@ -134,6 +134,7 @@ __global__ void append_kernel(Shape s, const T* __restrict__ k_new, const T* __r
                               const float* __restrict__ qbar, T* Kc, T* Vc, float* kbar, int kbar_T,
                               float* state, int* seqlens)
 {
+    pdl_launch_dependents();   // the decode routing that follows waits for this grid itself
     const int b = blockIdx.x, r = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = seqlens[b];
     const bool ok = L < s.n;

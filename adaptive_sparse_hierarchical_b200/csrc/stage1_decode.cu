@@ -77,6 +77,10 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
     dec_route_cluster_kernel(Shape s, const T* __restrict__ q, const float* __restrict__ kbar, int kbar_T,
                              const int* __restrict__ seqlens, Routes rt, int per, int* status)
 {
+    // the append of this step (the previous kernel) may still run: seqlens and the caches are
+    // read after its completion
+    pdl_wait();
+    pdl_launch_dependents();
     // the step's status word starts at 0 here (the later kernels of the step may set it)
     if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
     extern __shared__ __align__(16) float dyn[];
@@ -344,8 +348,8 @@ cudaError_t launch_t(const Shape& s, const void* q, const float* kbar, int kbar_
         const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k<<<kRanks * s.batch * s.hkv, kThr, smem, st>>>(s, (const T*)q, kbar, kbar_T, seqlens, rt, per, status);
-    return cudaGetLastError();
+    return launch_after(k, dim3(kRanks * s.batch * s.hkv), dim3(kThr), smem, st, s, (const T*)q, kbar, kbar_T,
+                        seqlens, rt, per, status);
 }
 
 }  // namespace

@@ -59,6 +59,8 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 
     const int BR = s.batch * s.hkv, G = s.g, NH = s.B / 64;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();   // the routes of this step
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         int acc = 0;
         for (int x = 0; x < BR; ++x) {
@@ -315,6 +317,7 @@ template <int D>
 __global__ void __launch_bounds__(D) dec_merge_kernel(Shape s, const float* __restrict__ part, int nblocks,
                                                       Routes rt, __nv_bfloat16* __restrict__ O)
 {
+    pdl_wait();   // the partials of this step
     const int x = blockIdx.x / s.g, row = blockIdx.x % s.g, G = s.g, NH = s.B / 64;
     const int b = x / s.hkv, r = x % s.hkv, col = threadIdx.x;
     long long lo = 0, total = 0;
@@ -408,9 +411,11 @@ cudaError_t launch_dec_attend_tma(const Shape& s, const void* q, const void* Kc,
     cudaError_t e = cudaFuncSetAttribute(dec_attend_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int nb = dec_tma_blocks();
-    dec_attend_tma_kernel<<<nb, 32 * (1 + kCons), smem, st>>>(mk, mv, s, (const __nv_bfloat16*)q, seqlens, rt, part, err);
-    dec_merge_kernel<128><<<s.batch * s.hkv * s.g, 128, 0, st>>>(s, part, nb, rt, (__nv_bfloat16*)O);
-    return cudaGetLastError();
+    e = launch_after(dec_attend_tma_kernel, dim3(nb), dim3(32 * (1 + kCons)), smem, st, mk, mv, s,
+                     (const __nv_bfloat16*)q, seqlens, rt, part, err);
+    if (e != cudaSuccess) return e;
+    return launch_after(dec_merge_kernel<128>, dim3(s.batch * s.hkv * s.g), dim3(128), 0, st, s, (const float*)part,
+                        nb, rt, (__nv_bfloat16*)O);
 }
 
 }  // namespace dash
