@@ -61,7 +61,7 @@ long long route_cap(const dash_params* p)
     return tri_offset(p->seqlen, p->chunk);
 }
 
-struct PrefillLayout { size_t kbar, counts, idx, bias, err, planes, redo, total; };
+struct PrefillLayout { size_t kbar, counts, idx, bias, err, planes, redo, perm, total; };
 PrefillLayout prefill_layout(const dash_params* p)
 {
     PrefillLayout L;
@@ -75,7 +75,8 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.err = L.bias + up(bh * cap * 4);
     L.planes = L.err + kAlign;
     L.redo = L.planes + up(bh * 3 * T * p->d_h * 2);
-    L.total = L.redo + up(bh * (size_t)p->seqlen);   // one flag per position block at most
+    L.perm = L.redo + up(bh * (size_t)p->seqlen);   // one flag per position block at most
+    L.total = L.perm + up(bh * (size_t)p->seqlen * 4);
     return L;
 }
 
@@ -185,7 +186,8 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE2)
-        rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt, err, st));
+        rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt,
+                                                 reinterpret_cast<int*>(ws + L.perm), err, st));
     return rc;
 }
 

@@ -138,13 +138,15 @@ int route_long_positions(const Shape& s);
 cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
                                       unsigned char* redo, int* err, cudaStream_t st);
 // Stage 2 for prefill.
+// perm: workspace of batch * h_kv * n ints (the tensor-core path's grouped position order)
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,
-                                  const void* V, void* O, const Routes& rt, int* err, cudaStream_t st);
+                                  const void* V, void* O, const Routes& rt, int* perm, int* err, cudaStream_t st);
 // tcgen05 / TMEM / TMA variant (bf16, d = 128, chunk 64 or 128); err receives a non-zero code
 // when one of its bounded waits times out.
 bool attend_tc_supported(const Shape& s, int dtype);
+// perm: workspace of batch * h_kv * n ints for the grouped position order (null: sequence order)
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
-                                     const Routes& rt, int* err, cudaStream_t st);
+                                     const Routes& rt, int* perm, int* err, cudaStream_t st);
 bool legacy_stage2();
 // Decode: Stage 1 (logits, thresholds, GQA aggregation) and Stage 2 (split + merge).
 struct DecodeWs {

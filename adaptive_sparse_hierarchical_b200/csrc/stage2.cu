@@ -453,9 +453,10 @@ cudaError_t rows_t(const Shape& s, const void* Q, const void* K, const void* V, 
 }  // namespace
 
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K, const void* V,
-                                  void* O, const Routes& rt, int* err, cudaStream_t st)
+                                  void* O, const Routes& rt, int* perm, int* err, cudaStream_t st)
 {
-    if (attend_tc_supported(s, dtype) && !legacy_stage2()) return launch_attend_prefill_tc(s, Q, K, V, O, rt, err, st);
+    if (attend_tc_supported(s, dtype) && !legacy_stage2())
+        return launch_attend_prefill_tc(s, Q, K, V, O, rt, perm, err, st);
     if (dtype == DASH_BF16)
         return s.d == 128 ? prefill_bf16_d<128>(s, Q, K, V, O, rt, st) : prefill_bf16_d<64>(s, Q, K, V, O, rt, st);
     return s.d == 128 ? rows_t<float, 128>(s, Q, K, V, O, rt, nullptr, st)

@@ -107,6 +107,55 @@ __device__ __forceinline__ Bars make_bars(uint32_t base)
     return b;
 }
 
+// Position order for the 128-row tiles (one block per window of kWinTiles tiles of P positions of
+// one (sequence, KV head)).  Rows of a tile share the union of their positions' routed chunks, so
+// positions with similar routes should share tiles.  A sparse window (under 1/8 of the visible
+// chunks routed) is sorted by (first routed chunk, routed count, position): queries that route
+// the same chunks -- the same keys region -- land in the same tiles, whatever their distance.
+// Denser windows keep each run of 8 tiles and sort it by (routed count, position), so that
+// positions with few routes (e.g. queries matching a few strong chunks) share tiles.  perm[br][k]
+// = the position at slot k.
+constexpr int kWinTiles = 64, kSubTiles = 8;
+__global__ void __launch_bounds__(1024) group_positions_kernel(Shape s, Routes rt, int P, int* __restrict__ perm)
+{
+    __shared__ unsigned long long key[kWinTiles * 16];
+    __shared__ int red[2][32];
+    const int br = blockIdx.y, tid = threadIdx.x;
+    const int Wn = kWinTiles * P, w0 = blockIdx.x * Wn, nw = min(Wn, s.n - w0);
+    const int* counts = rt.counts + (long long)br * s.n;
+    const int* ridx = rt.idx + (long long)br * rt.cap;
+    int cs = 0, vs = 0;
+    for (int j = tid; j < nw; j += blockDim.x) {
+        const int i = w0 + j;
+        cs += counts[i];
+        vs += min(i / s.B, s.T);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        cs += __shfl_xor_sync(0xffffffffu, cs, o);
+        vs += __shfl_xor_sync(0xffffffffu, vs, o);
+    }
+    if ((tid & 31) == 0) { red[0][tid >> 5] = cs; red[1][tid >> 5] = vs; }
+    __syncthreads();
+    long long csum = 0, vsum = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { csum += red[0][w]; vsum += red[1][w]; }
+    const bool sparse = 8 * csum < vsum;
+    for (int j = tid; j < nw; j += blockDim.x) {
+        const int i = w0 + j, c = counts[i];
+        const unsigned long long first = c > 0 ? (unsigned long long)ridx[tri_offset(i, s.B)] : (unsigned long long)s.T;
+        key[j] = sparse ? (first << 40) | ((unsigned long long)c << 20) | (unsigned long long)j
+                        : ((unsigned long long)c << 20) | (unsigned long long)j;
+    }
+    __syncthreads();
+    const int span = sparse ? Wn : kSubTiles * P;   // positions ranked together
+    for (int j = tid; j < nw; j += blockDim.x) {
+        const int g0 = j / span * span, g1 = min(nw, g0 + span);
+        const unsigned long long kj = key[j];
+        int rank = 0;
+        for (int q = g0; q < g1; ++q) rank += key[q] < kj;
+        perm[(long long)br * s.n + w0 + g0 + rank] = w0 + j;
+    }
+}
+
 // CPT = chunks per 64-key tile: 1 for chunks of 64 or 128 keys (a chunk is one or two jobs), 2 for
 // 32-key chunks (a job covers two neighbouring chunks, each row with its own bias per half).
 template <int CPT>
@@ -116,7 +165,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                                                                    const __grid_constant__ CUtensorMap tmV,
                                                                    Shape s, Routes rt,
                                                                    __nv_bfloat16* __restrict__ O, int* err,
-                                                                   int cluster)
+                                                                   const int* __restrict__ perm)
 {
     extern __shared__ char smem_raw[];
     char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -165,25 +214,11 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         tc::tmem_alloc(tc::smem_addr(tmem_slot), kTmemCols);
     }
     for (int w = tid; w < W; w += blockDim.x) umask[w] = 0u;
-    if (cluster) {
-        // Rows of one tile share its union of routed chunks.  The window of 8 consecutive tiles
-        // is re-grouped by routed-chunk count (a stable order), so positions with small routes
-        // (here: queries matching the planted chunks) share tiles with small unions.
-        int* key = reinterpret_cast<int*>(sm + kOffScratch + 16384);
-        const int Wn = 8 * P, w0 = (pb / 8) * Wn, t8 = pb % 8;
-        for (int j = tid; j < Wn; j += blockDim.x) {
-            const int ii = w0 + j;
-            key[j] = ii < s.n ? ((counts[ii] << 8) | j) : INT_MAX - Wn + j;
-        }
-        __syncthreads();
-        for (int j = tid; j < Wn; j += blockDim.x) {
-            const int kj = key[j];
-            int rank = 0;
-            for (int q = 0; q < Wn; ++q) rank += key[q] < kj;
-            if (rank / P == t8) spos[rank % P] = w0 + j;
-        }
-    } else {
-        for (int p = tid; p < P; p += blockDim.x) spos[p] = i0 + p;
+    // the block's positions: slots pb*P .. pb*P+P-1 of the grouped order (positions past the end
+    // of the sequence stay in place and are masked)
+    for (int p = tid; p < P; p += blockDim.x) {
+        const int k = i0 + p;
+        spos[p] = perm && k < s.n ? perm[(long long)br * s.n + k] : k;
     }
     __syncthreads();
     for (int p = 0; p < P; ++p) {
@@ -236,7 +271,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             tc::prefetch_tmap(&tmK);
             tc::prefetch_tmap(&tmV);
             tc::mbar_expect_tx(bar.q_full, kQBytes);
-            if (cluster) {
+            if (perm) {
                 // one box of g rows per position (g = 8 or 16 keeps every box 1024-byte aligned)
                 tc::prefetch_tmap(&tmQ1);
                 for (int p = 0; p < P; ++p) {
@@ -615,11 +650,17 @@ size_t attend_tc_smem(const Shape& s)
 }
 
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
-                                     const Routes& rt, int* err, cudaStream_t st)
+                                     const Routes& rt, int* perm, int* err, cudaStream_t st)
 {
     CUtensorMap mq, mq1, mk, mv;
     const int P = kRows / s.g;
-    const int cluster = (s.g == 8 || s.g == 16) && !cluster_disabled() ? 1 : 0;
+    const bool group = perm && (s.g == 8 || s.g == 16) && !cluster_disabled();
+    if (group && s.n > 0) {
+        const int Wn = kWinTiles * P;
+        group_positions_kernel<<<dim3((s.n + Wn - 1) / Wn, s.batch * s.hkv), 1024, 0, st>>>(s, rt, P, perm);
+        const cudaError_t eg = cudaGetLastError();
+        if (eg != cudaSuccess) return eg;
+    }
     if (!make_map(&mq, Q, s.batch, s.n, s.hq, s.qs, s.g, P) || !make_map(&mq1, Q, s.batch, s.n, s.hq, s.qs, s.g, 1) ||
         !make_map(&mk, K, s.batch, s.n, s.hkv, s.ks, 1, kKT) || !make_map(&mv, V, s.batch, s.n, s.hkv, s.vs, 1, kKT))
         return cudaErrorInvalidValue;
@@ -630,7 +671,7 @@ cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* 
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    kern<<<grid, 192, smem, st>>>(mq, mq1, mk, mv, s, rt, (__nv_bfloat16*)O, err, cluster);
+    kern<<<grid, 192, smem, st>>>(mq, mq1, mk, mv, s, rt, (__nv_bfloat16*)O, err, group ? (const int*)perm : nullptr);
     return cudaGetLastError();
 }
 
