@@ -30,13 +30,16 @@ namespace dash {
 namespace {
 
 constexpr int kR = 128, kCT = 64, kDd = 128;
-constexpr int kQB = kR * kDd * 2;               // Q tile, two 16 KB d-halves
 constexpr int kPlaneHalf = kCT * 64 * 2;        // [64 chunks][64 d] bf16 = 8 KB
 constexpr int kStage = 2 * kPlaneHalf;          // one plane of a tile, two d-halves = 16 KB
 constexpr int kNS = 4;                          // ring stages
-constexpr int kBW = 256;                        // chunks per block = columns of a TMEM half
+constexpr int kBW = 192;                        // chunks per block = columns of a TMEM half
 constexpr int kTPB = kBW / kCT;                 // 64-chunk tiles per block
-constexpr int kOffQ1 = 0, kOffRing = kQB, kOffLists = kOffRing + kNS * kStage;
+constexpr int kPieces = kBW / 32;               // 32-column pieces per block
+// TMEM: X halves at columns [0, 192) and [192, 384); the Q tile (the MMAs' A operand, 128 rows x
+// 128 bf16, two per 32-bit column) at [384, 448)
+constexpr int kColQ = 2 * kBW;
+constexpr int kOffRing = 0, kOffLists = kOffRing + kNS * kStage;
 constexpr uint32_t kIdescX = tc::idesc_bf16(128, 64, false, false);
 // after every pass but the first the workers post whether another pass over the blocks follows
 // (kPlanGo) or not (kPlanStop); at most kMaxExtract extraction passes per set of rows in play
@@ -45,7 +48,7 @@ constexpr int kMaxExtract = 2;
 
 // candidate list entries per (worker warp, lane); the lists also hold the weights buffer
 // [P][kBW] of the emission pass (the lists are dead by then)
-constexpr int kCap = 56;
+constexpr int kCap = 72;
 constexpr int kOffMisc = kOffLists + 16 * 32 * kCap * 4;
 // misc: 16 barriers (128 B), tmem slot / abort / overflow / plan (16 B), red [3][4][kR] float2
 // (12 KB), per position: running log-sum, count, list base (3 x 32 words)
@@ -121,8 +124,8 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane, i
 }
 
 template <int G>
-__global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                                    const __grid_constant__ CUtensorMap tmP,
+__global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid_constant__ CUtensorMap tmP,
+                                                                    const __nv_bfloat16* __restrict__ Q,
                                                                     Shape s, Routes rt, unsigned char* redo,
                                                                     int* err)
 {
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
     const int nbk = (ntiles + kTPB - 1) / kTPB;   // 256-chunk blocks
 
     if (tid == 0) {
-        tc::mbar_init(q_full, 1);
+        tc::mbar_init(q_full, 128);   // the four warps that write the Q rows into TMEM
         for (int k = 0; k < kNS; ++k) {
             tc::mbar_init(full0 + 8 * k, 1);
             tc::mbar_init(empty0 + 8 * k, 1);
@@ -199,11 +202,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
     if (warp == 0) {
         // ---- TMA producer: Q once, then the plane tiles of every block, once per pass ----------
         if (lane == 0) {
-            tc::prefetch_tmap(&tmQ);
             tc::prefetch_tmap(&tmP);
-            tc::mbar_expect_tx(q_full, kQB);
-            tc::tma_load_4d(base + kOffQ1, &tmQ, q_full, 0, r * G, i0, b);
-            tc::tma_load_4d(base + kOffQ1 + kQB / 2, &tmQ, q_full, 64, r * G, i0, b);
             int last[kNS] = {-1, -1, -1, -1};
             int gs = 0;   // ring stage counter: one stage per (tile, plane)
             bool pok = true;
@@ -229,14 +228,11 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                     if (last[j] >= 0)
                         for (long long it = 0; it < (1ll << 22); ++it)
                             if (tc::mbar_try(full0 + 8 * j, (last[j] / kNS) & 1)) break;
-                for (long long it = 0; it < (1ll << 22); ++it)
-                    if (tc::mbar_try(q_full, 0)) break;
             }
         }
     } else if (warp == 1) {
         // ---- MMA issuer: TMEM half u & 1 takes the u-th block of the pass sequence ------------
         if (lane == 0) {
-            const uint64_t dQ = tc::sw128_desc(base + kOffQ1, 16, 1024);
             const uint64_t dP0 = tc::sw128_desc(base + kOffRing, 16, 1024);
             bool ok = tc::mbar_wait(q_full, 0, abort, err, 32);
             int gs = 0, u = 0;
@@ -254,7 +250,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                             const uint64_t dp = dP0 + (uint64_t)((st * kStage) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < kDd / 16; ++kk)
-                                tc::mma_f16_ss(xd, dQ + (uint64_t)(((kk >> 2) * (kQB / 2) + (kk & 3) * 32) >> 4),
+                                tc::mma_f16_ts(xd, tmem + kColQ + kk * 8,
                                                dp + (uint64_t)(((kk >> 2) * kPlaneHalf + (kk & 3) * 32) >> 4),
                                                kIdescX, (pl > 0 || kk > 0) ? 1u : 0u);
                             tc::mma_commit(empty0 + 8 * st);
@@ -302,6 +298,20 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
         // Lists: region (cq, q4) holds [CAP][32 lanes]; the regions of quarters q4 and q4 ^ 2 sit
         // side by side, so that with only half of the rows in play a thread's list runs on into
         // its idle partner's region (capacity 2 CAP).
+        if (cq == 0) {
+            // row (position i0 + row / g, head r g + row % g) of the Q tile into this lane of TMEM
+            // columns [kColQ, kColQ + 64): the row's bf16 pairs are already the 32-bit columns
+            uint4 qw[16];
+            const __nv_bfloat16* qrow = Q + (long long)b * s.qs[0] + (long long)i * s.qs[1] + (long long)(r * G + row % G) * s.qs[2];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                qw[k] = i < s.n ? __ldg(reinterpret_cast<const uint4*>(qrow) + k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tc::tmem_st16(lane_base + kColQ + 16 * k, reinterpret_cast<const uint32_t*>(qw + 4 * k));
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            tc::mbar_arrive(q_full);
+        }
         float* const own_list = lists + ((cq * 2 + (q4 & 1)) * 2 + (q4 >> 1)) * CAP * 32 + lane;
         float* const pair_list = lists + ((cq * 2 + (q4 & 1)) * 2) * CAP * 32 + lane;
         float* cl = own_list;   // this thread's list, entry k at cl[32 k]
@@ -323,8 +333,10 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                 ok = workers_all(got);   // uniform: a time-out anywhere stops every worker together
                 if (ok && active) {
                     tc::fence_after_sync();
-                    // pieces lp = cq, cq + 4 of this block; column = kb * kBW + 32 lp + e
-                    for (int lp = cq; lp < kBW / 32; lp += 4) {
+                    // the pieces of this block whose global index (column / 32) is cq mod 4;
+                    // column = kb * kBW + 32 lp + e
+                    for (int lp = 0; lp < kPieces; ++lp) {
+                        if ((kb * kPieces + lp) % 4 != cq) continue;
                         const int c0 = kb * kBW + lp * 32;
                         // columns past every row of the warp: never read (the g rows of a position
                         // sit in one warp, and the emission stops at the position's own bound)
@@ -579,19 +591,7 @@ cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* pl
     auto fn = encode_fn_l();
     if (!fn) return cudaErrorInvalidValue;
     constexpr int P = kR / G;
-    CUtensorMap mq, mp;
-    {
-        // Q [b][n][hq][128] (strided): box = 64 d x the g heads of KV head r x P positions
-        cuuint64_t dims[4] = {128, (cuuint64_t)s.hq, (cuuint64_t)s.n, (cuuint64_t)s.batch};
-        cuuint64_t strides[3] = {(cuuint64_t)s.qs[2] * 2, (cuuint64_t)s.qs[1] * 2, (cuuint64_t)s.qs[0] * 2};
-        if (s.batch == 1) strides[2] = strides[1] * (cuuint64_t)s.n;
-        cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)P, 1};
-        cuuint32_t es[4] = {1, 1, 1, 1};
-        if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(Q), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    CUtensorMap mp;
     {
         // planes [b*hkv*3][T][128] viewed as (d, chunk, plane-row, 1)
         cuuint64_t dims[4] = {128, (cuuint64_t)s.T, (cuuint64_t)s.batch * s.hkv * 3, 1};
@@ -610,7 +610,7 @@ cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* pl
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 576, smem, st>>>(mq, mp, s, rt, redo, err);
+    k<<<grid, 576, smem, st>>>(mp, static_cast<const __nv_bfloat16*>(Q), s, rt, redo, err);
     return cudaGetLastError();
 }
 
