@@ -50,9 +50,11 @@ constexpr int kMaxExtract = 2;
 // [P][kBW] of the emission pass (the lists are dead by then)
 constexpr int kCap = 72;
 constexpr int kOffMisc = kOffLists + 16 * 32 * kCap * 4;
-// misc: 16 barriers (128 B), tmem slot / abort / overflow / plan (16 B), red [3][4][kR] float2
+// misc: barriers (kBarBytes), tmem slot / abort / overflow / plan (16 B), red [3][4][kR] float2
 // (12 KB), per position: running log-sum, count, list base (3 x 32 words)
-constexpr int kMiscBytes = 128 + 16 + 3 * 4 * kR * 8 + 3 * 32 * 4;
+constexpr int kBarBytes = 8 * (1 + 2 * kNS + 2 + 2 + 2);   // q_full, full/empty ring, x_ready/x_free, drain, dec
+constexpr int kMiscBase = (kBarBytes + 15) / 16 * 16;
+constexpr int kMiscBytes = kMiscBase + 16 + 3 * 4 * kR * 8 + 3 * 32 * 4;
 constexpr size_t kLongSmem = 1024 + kOffMisc + kMiscBytes;
 static_assert(kLongSmem <= 227 * 1024, "shared memory of the long-row routing kernel");
 static_assert((kR / 4) * kBW * 4 <= 16 * 32 * kCap * 4, "weights buffer inside the lists");
@@ -137,16 +139,16 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
     float* wbuf = lists;                                                // [P][kBW] group sums of one block
     char* misc = sm + kOffMisc;
     const uint32_t bar0 = tc::smem_addr(misc);
-    const uint32_t q_full = bar0, full0 = bar0 + 8, empty0 = bar0 + 40;   // ring [kNS] each
-    const uint32_t x_ready0 = bar0 + 72, x_free0 = bar0 + 88;            // TMEM halves [2] each
-    const uint32_t drain = bar0 + 104;
-    const uint32_t dec = bar0 + 112;                                      // pass decisions
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 128);
-    volatile int* abort = reinterpret_cast<volatile int*>(misc + 132);
-    int* overflow = reinterpret_cast<int*>(misc + 136);
-    volatile int* plan_word = reinterpret_cast<volatile int*>(misc + 140);
-    float2* red = reinterpret_cast<float2*>(misc + 144);                  // [3][4][kR]
-    float* pslog = reinterpret_cast<float*>(misc + 144 + 3 * 4 * kR * 8);  // [P] log-sum so far
+    const uint32_t q_full = bar0, full0 = bar0 + 8, empty0 = full0 + 8 * kNS;   // ring [kNS] each
+    const uint32_t x_ready0 = empty0 + 8 * kNS, x_free0 = x_ready0 + 16;       // TMEM halves [2] each
+    const uint32_t drain = x_free0 + 16;
+    const uint32_t dec = drain + 8;                                             // pass decisions
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + kMiscBase);
+    volatile int* abort = reinterpret_cast<volatile int*>(misc + kMiscBase + 4);
+    int* overflow = reinterpret_cast<int*>(misc + kMiscBase + 8);
+    volatile int* plan_word = reinterpret_cast<volatile int*>(misc + kMiscBase + 12);
+    float2* red = reinterpret_cast<float2*>(misc + kMiscBase + 16);                  // [3][4][kR]
+    float* pslog = reinterpret_cast<float*>(misc + kMiscBase + 16 + 3 * 4 * kR * 8);  // [P] log-sum so far
     int* pcnt = reinterpret_cast<int*>(pslog + 32);                        // [P] entries so far
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -203,13 +205,15 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
         // ---- TMA producer: Q once, then the plane tiles of every block, once per pass ----------
         if (lane == 0) {
             tc::prefetch_tmap(&tmP);
-            int last[kNS] = {-1, -1, -1, -1};
+            int last[kNS];
+#pragma unroll
+            for (int j = 0; j < kNS; ++j) last[j] = -1;
             int gs = 0;   // ring stage counter: one stage per (tile, plane)
             bool pok = true;
             for (int k = 0; pok; ++k) {
                 for (int t = 0; pok && t < ntiles; ++t) {
                     for (int pl = 0; pl < 3; ++pl, ++gs) {
-                        const int st = gs & (kNS - 1);
+                        const int st = gs % kNS;
                         if (gs >= kNS && !tc::mbar_wait(empty0 + 8 * st, ((gs / kNS) - 1) & 1, abort, err, 31)) { pok = false; break; }
                         last[st] = gs;
                         const uint32_t dst = base + kOffRing + st * kStage, fb = full0 + 8 * st;
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                     for (int t = kb * kTPB; ok && t < min(ntiles, (kb + 1) * kTPB); ++t) {
                         const uint32_t xd = tmem + hlf * kBW + (t - kb * kTPB) * kCT;
                         for (int pl = 0; pl < 3; ++pl, ++gs) {
-                            const int st = gs & (kNS - 1);
+                            const int st = gs % kNS;
                             if (!tc::mbar_wait(full0 + 8 * st, (gs / kNS) & 1, abort, err, 34)) { ok = false; break; }
                             tc::fence_after_sync();
                             const uint64_t dp = dP0 + (uint64_t)((st * kStage) >> 4);
