@@ -75,6 +75,9 @@ def get(name: str) -> Workload:
         _, _, a, B = name.split("_")      # sweep_128k_<alpha>_<B>
         return Workload(name, 1, 131072, 16, 2, 128, int(B), float(a), 1.0, "bf16", "mixture",
                         extra={"seed": 5})
+    if name == "mixture_32k_b32":   # profiling case of the long-row routing kernel: the 128K sweep's
+        # inputs at n=32768 with 32-key chunks (T = 1024 > 512), alpha 1.5, gamma 1
+        return Workload(name, 1, 32768, 16, 2, 128, 32, 1.5, 1.0, "bf16", "mixture", extra={"seed": 5})
     raise KeyError(name)
 
 
