@@ -1,5 +1,9 @@
 """GPU parity of the prefill path (dash_prefill through the C ABI) against the float64 oracle on
 the same seeded inputs: Stage 0 summaries, Stage 1 routed sets and biases, Stage 2 outputs."""
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -226,3 +230,36 @@ def test_sweep_128k_full_size_sampled(name):
     frac_rows = (cnt / vis)[:, wl.chunk:]
     print(name, st, "support fraction p10/p50/p90",
           [round(v, 3) for v in torch.quantile(frac_rows.flatten()[::97], torch.tensor([0.1, 0.5, 0.9], device=cnt.device)).tolist()])
+
+
+_GROUPING_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import adaptive_sparse_hierarchical_b200 as D
+from adaptive_sparse_hierarchical_b200 import inputs
+x = inputs.mixture(7, 1, 8192, 16, 2, 128)
+Q, K, V = (torch.from_numpy(x[k]).cuda().to(torch.bfloat16) for k in ("Q", "K", "V"))
+pf = D.Prefill(Q, K, V, torch.from_numpy(x["qbar"]).cuda(), chunk=64, alpha=1.5, gamma=1.0, want_route=True)
+O = pf()
+torch.cuda.synchronize()
+assert pf.error_word() == 0
+np.save(sys.argv[2], O.view(torch.int16).cpu().numpy())
+"""
+
+
+def test_position_grouping_changes_only_the_schedule(tmp_path):
+    """Stage 2 orders a sparse window's positions by their first routed chunk before forming the
+    128-row tiles.  A row's arithmetic does not depend on its tile-mates (a tile the row does not
+    route adds exact zeros to its sums), so the output equals the sequence-order run
+    (DASH_CLUSTER=0) bit for bit.  Mixture inputs at gamma 1 route ~2% of the chunks, so every
+    window takes the grouped order."""
+    here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = []
+    for flag in ("1", "0"):
+        f = tmp_path / f"o_{flag}.npy"
+        env = dict(os.environ, DASH_CLUSTER=flag)
+        r = subprocess.run([sys.executable, "-c", _GROUPING_CHILD, here, str(f)], env=env,
+                           capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+        outs.append(np.load(f))
+    assert np.array_equal(outs[0], outs[1])
