@@ -155,6 +155,17 @@ def stage2_routed_flops(counts, n, B, g, d, hq):
     return 4.0 * d * (float(counts.sum()) * B * g + counts.shape[0] * hq * diag)
 
 
+def prefill_launches(wl):
+    """Kernels of this library one prefill step launches: Stage 0, Stage 1, Stage 2, plus the
+    position grouping ahead of the tensor-core Stage 2 (g = 8 or 16) and, for rows of more than
+    512 chunks, the per-shape routing kernel that recomputes overflowed position blocks."""
+    g = wl.h_q // wl.h_kv
+    tc = wl.dtype == "bf16" and wl.d == 128
+    group = tc and wl.chunk in (32, 64, 128) and g in (8, 16) and os.environ.get("DASH_CLUSTER", "") != "0"
+    long_rows = tc and wl.n // wl.chunk > 512 and g in (4, 8, 16)
+    return 3 + int(group) + int(long_rows)
+
+
 def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
     import torch
     import adaptive_sparse_hierarchical_b200 as D
@@ -216,7 +227,7 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
                      "peak_kind": f"bf16 dense burst, of {pk_kind}",
                      "flops_per_launch": flops, "launch_ms": stage_ms[2]},
         "clocks": clk.summary(),
-        "gpu_launches": 3 * steps,
+        "gpu_launches": prefill_launches(wl) * steps,
     }
     if lite:   # sweep mode: the device-timed step and the per-row support only
         c = counts.reshape(-1, wl.n)[:, wl.chunk:].astype("float64")
@@ -421,7 +432,7 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
                         "achieved": achieved,
                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
                         "peak_kind": f"hbm copy, of {pk_kind}", "bytes_per_step": bps},
-           "clocks": clk.summary(), "gpu_launches": 6 * (nst - 1),
+           "clocks": clk.summary(), "gpu_launches": 4 * (nst - 1),   # append, routing, attend, merge
            "l2": "KV caches (1.07 GB) larger than L2"}
     res["us_per_token"] = res["us_per_step"] / wl.batch   # per sequence-token, one GPU
     return res
