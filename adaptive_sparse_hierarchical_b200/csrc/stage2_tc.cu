@@ -34,11 +34,11 @@ constexpr int kKVHalf = kKT * 64 * 2;             // 8 KB: [64 keys][64 d]
 constexpr int kSlot = 4 * kKVHalf;                // K (2 halves) + V (2 halves) = 32 KB
 constexpr int kTmemCols = 256;                    // S0 [0,64), S1 [64,128), O [128,256); P_k over S_k
 constexpr int kOffQ = 0, kOffSlots = kQBytes;
-constexpr int kOffScratch = kOffSlots;            // set-up scratch (chunk bitmask, sort keys) in the ring
+constexpr int kOffScratch = kOffSlots;            // set-up scratch (the union bitmask) in the ring
 constexpr int kOffBar = kOffSlots + kNS * kSlot;  // 98304: two blocks fit on one SM
 constexpr int kNumBars = 1 + 2 * kNS + 2 + 2 + 2 + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, njobs
-constexpr int kOffPos = kOffMisc + 32;             // the block's positions (<= 16 when clustered)
+constexpr int kOffPos = kOffMisc + 32;             // the block's positions (128 / g of them)
 constexpr int kOffJobs = kOffPos + 4 * kRows;
 
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, 64, false, false);
@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
 
 bool cluster_disabled()
 {
-    // DASH_CLUSTER=0 keeps positions in sequence order inside each tile (comparison runs)
+    // DASH_CLUSTER=0 keeps positions in sequence order (no grouping; comparison runs and tests)
     static int v = -1;
     if (v < 0) {
         const char* e = getenv("DASH_CLUSTER");
