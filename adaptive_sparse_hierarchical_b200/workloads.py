@@ -75,6 +75,11 @@ def get(name: str) -> Workload:
         _, _, a, B = name.split("_")      # sweep_128k_<alpha>_<B>
         return Workload(name, 1, 131072, 16, 2, 128, int(B), float(a), 1.0, "bf16", "mixture",
                         extra={"seed": 5})
+    if name.startswith("decode_96k_b24_"):   # the pages' decode shape: batch 24, 96K contexts
+        frac = name.rsplit("_", 1)[1]        # routed fraction "25" or "6.25" (sparsity 75 / 93.75%)
+        return Workload(name, 24, 98304 + 256, 32, 2, 128, 64, 1.5, g.get(name, 8.0), "bf16", "planted",
+                        extra={"seed": 6, "q_rows": (98304, 256), "prefix": 98304, "steps": 256,
+                               "target": float(frac) / 100})
     if name == "mixture_32k_b32":   # profiling case of the long-row routing kernel: the 128K sweep's
         # inputs at n=32768 with 32-key chunks (T = 1024 > 512), alpha 1.5, gamma 1
         return Workload(name, 1, 32768, 16, 2, 128, 32, 1.5, 1.0, "bf16", "mixture", extra={"seed": 5})
@@ -83,3 +88,4 @@ def get(name: str) -> Workload:
 
 PREFILL_64K = ["prefill_64k_50", "prefill_64k_25", "prefill_64k_12.5"]
 SWEEP_128K = [f"sweep_128k_{a}_{B}" for a in ("1.25", "1.5", "2.0") for B in (32, 64, 128)]
+DECODE_96K = ["decode_96k_b24_25", "decode_96k_b24_6.25"]

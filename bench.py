@@ -343,12 +343,12 @@ def dense_denominators(wl, tq, qbar, pf, steps, flush, sparse_ms, dev):
 
 
 # ---------------------------------------------------------------------------------------- decode
-def run_decode(steps, warmup, ranks, pk, pk_kind):
+def run_decode(steps, warmup, ranks, pk, pk_kind, name="decode_128k"):
     import torch
     import adaptive_sparse_hierarchical_b200 as D
     from adaptive_sparse_hierarchical_b200 import workloads as W
 
-    wl = W.get("decode_128k")
+    wl = W.get(name)
     dev = torch.device("cuda", ranks.local)
     x = wl.make()
     prefix = wl.extra["prefix"]
@@ -421,8 +421,9 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
         byts.append(2 * wl.d * 2 * (float(c.sum()) * wl.chunk + wl.batch * wl.h_kv * diag))
     bps = statistics.mean(byts)
     achieved = bps / (ms / 1e3) / 1e9   # whole graph step (append + route + attend + merge)
-    res = {"workload": "decode_128k: b=8, 131072-token caches (+1 per step), 32/2 heads, d=128, B=64, alpha 1.5, "
-                       f"gamma {wl.gamma} (~25% routed)",
+    res = {"workload": f"{name}: b={wl.batch}, {prefix}-token caches (+1 per step), {wl.h_q}/{wl.h_kv} heads, "
+                       f"d={wl.d}, B={wl.chunk}, alpha {wl.alpha}, gamma {wl.gamma} "
+                       f"(~{100 * wl.extra.get('target', 0.25):g}% routed)",
            "us_per_step": ms * 1e3, "us_per_step_eager": eager_ms * 1e3,
            "timing": "per step: one copy of the packed q, k, v into the captured graph's staging buffer + graph replay (append + decode)",
            "steps": nst, "append_us": statistics.mean(a.elapsed_time(b) for a, b, c in evs) * 1e3,
@@ -433,7 +434,7 @@ def run_decode(steps, warmup, ranks, pk, pk_kind):
                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
                         "peak_kind": f"hbm copy, of {pk_kind}", "bytes_per_step": bps},
            "clocks": clk.summary(), "gpu_launches": 4 * (nst - 1),   # append, routing, attend, merge
-           "l2": "KV caches (1.07 GB) larger than L2"}
+           "l2": f"KV caches ({2 * wl.batch * wl.n * wl.h_kv * wl.d * 2 / 1e9:.2f} GB) larger than L2"}
     res["us_per_token"] = res["us_per_step"] / wl.batch   # per sequence-token, one GPU
     return res
 
@@ -517,6 +518,17 @@ def run_sweep(args, ranks, pk, pk_kind):
                            "chunk": wl.chunk, "alpha": wl.alpha, "gamma": wl.gamma}}
         if ranks.rank == 0:
             print(json.dumps(line), flush=True)
+    cache.clear()
+    gc.collect()
+    # decode at the pages' own shape: batch 24, 96K contexts, 75% and 93.75% sparsity
+    for name in W.DECODE_96K:
+        r = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind, name=name)
+        line = {"sweep": name, "metric": "decode us/token", "value": r["us_per_token"], "unit": "us/token",
+                "higher_is_better": False, "us_per_step": r["us_per_step"], "routed_fraction": r["routed_fraction"],
+                "roofline": r["roofline"], "clocks": r["clocks"], "steps": r["steps"], "workload": r["workload"]}
+        if ranks.rank == 0:
+            print(json.dumps(line), flush=True)
+        gc.collect()
 
 
 def main():

@@ -63,15 +63,16 @@ def decode_case(name):
     sel = np.arange(0, steps, 8)
     pos = (prefix + sel).astype(np.int32)
     Qrows = x["Q"][:, sel]
-    g, f = tune(Qrows, np.broadcast_to(pos, (wl.batch, pos.size)), x["K"], kbar, wl.chunk, wl.alpha, 0.25)
-    print(f"{name}: gamma={g:.4f} routed fraction={f:.4f} (target 0.25)", flush=True)
+    target = wl.extra.get("target", 0.25)
+    g, f = tune(Qrows, np.broadcast_to(pos, (wl.batch, pos.size)), x["K"], kbar, wl.chunk, wl.alpha, target)
+    print(f"{name}: gamma={g:.4f} routed fraction={f:.4f} (target {target})", flush=True)
     return g
 
 
 def main():
     path = os.path.join(ROOT, "adaptive_sparse_hierarchical_b200", "workloads.json")
     out = W.tuned_gammas()
-    todo = sys.argv[1:] or ["prefill_32k", "decode_128k", *W.PREFILL_64K]
+    todo = sys.argv[1:] or ["prefill_32k", "decode_128k", *W.PREFILL_64K, *W.DECODE_96K]
     for name in todo:
         out[name] = round(prefill_case(name, 64) if name.startswith("prefill") else decode_case(name), 4)
         with open(path, "w") as fh:

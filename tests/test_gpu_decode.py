@@ -149,6 +149,34 @@ def test_decode_128k_full_size_sampled():
     assert 0.15 < frac < 0.35, frac
 
 
+def test_decode_96k_batch24_full_size_sampled():
+    """The pages' decode shape: batch 24, 96K-token caches (32/2 heads, d=128, B=64) at 75% and
+    93.75% sparsity (one set of inputs, gamma tuned per sparsity); 8 append+decode steps each,
+    steps 0 and 7 checked against the oracle."""
+    wl0 = W.get(W.DECODE_96K[0])
+    x = wl0.make()
+    prefix = wl0.extra["prefix"]
+    Kt = torch.from_numpy(x["K"][:, prefix:prefix + 8]).to("cuda", torch.bfloat16)
+    Vt = torch.from_numpy(x["V"][:, prefix:prefix + 8]).to("cuda", torch.bfloat16)
+    Qt = torch.from_numpy(x["Q"][:, :8]).to("cuda", torch.bfloat16)
+    for name in W.DECODE_96K:
+        wl = W.get(name)
+        st = _state(x, [prefix] * wl.batch, wl.n, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma, dtype="bf16")
+        for s in range(8):
+            st.step(Qt[:, s].contiguous(), Kt[:, s].contiguous(), Vt[:, s].contiguous())
+            if s in (0, 7):
+                torch.cuda.synchronize()
+                lengths = np.full(wl.batch, prefix + s + 1)
+                stt = _check_step(st, x, x["Q"][:, s], lengths, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
+                                  dtype="bf16")
+                print(name, "step", s, stt)
+        frac = st.rt[0].sum().item() / (wl.batch * 2 * ((prefix + 7) // 64))
+        target = wl.extra["target"]
+        assert 0.6 * target < frac < 1.4 * target, (name, frac)
+        del st
+        torch.cuda.empty_cache()
+
+
 def test_decode_long_run_is_deterministic():
     """300 append+decode steps, run twice from the same saved state: the outputs must agree bit for
     bit at every step (a race between the producer and consumer warps of a K/V ring would show up
