@@ -34,6 +34,12 @@ class dash_route_out(ctypes.Structure):
                 ("bias", ctypes.c_void_p), ("bitmask", ctypes.c_void_p)]
 
 
+class dash_paged_kv(ctypes.Structure):
+    _fields_ = [("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("num_pages", ctypes.c_int), ("k_page_stride", ctypes.c_longlong),
+                ("v_page_stride", ctypes.c_longlong)]
+
+
 class DashError(RuntimeError):
     pass
 
@@ -67,6 +73,13 @@ def load():
         lib.dash_summary_append.restype = ctypes.c_int
         lib.dash_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, R, vp, sz, vp]
         lib.dash_decode.restype = ctypes.c_int
+        PK = ctypes.POINTER(dash_paged_kv)
+        lib.dash_summary_build_paged.argtypes = [P, PK, vp, vp, vp, vp, vp, vp]
+        lib.dash_summary_build_paged.restype = ctypes.c_int
+        lib.dash_summary_append_paged.argtypes = [P, PK, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.dash_summary_append_paged.restype = ctypes.c_int
+        lib.dash_decode_paged.argtypes = [P, PK, vp, vp, vp, vp, vp, vp, R, vp, sz, vp]
+        lib.dash_decode_paged.restype = ctypes.c_int
         lib.dash_status_string.argtypes = [ctypes.c_int]
         lib.dash_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -177,4 +190,37 @@ def dash_decode(p, q, K_cache, V_cache, kbar_cache, seqlens, O, route=None, work
                             _ptr(seqlens), _ptr(O), ctypes.byref(route) if route is not None else None,
                             _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dash_decode")
+    return rc
+
+
+def paged_kv(page_table, page_size, num_pages, k_page_stride, v_page_stride):
+    """Page description of paged K/V pools (page_table: device int32 [batch, max_pages])."""
+    return dash_paged_kv(_ptr(page_table), int(page_table.shape[1]), int(page_size), int(num_pages),
+                         int(k_page_stride), int(v_page_stride))
+
+
+def dash_summary_build_paged(p, pk, K_pool, qbar, seqlens, kbar_cache, partial_state, stream=None) -> int:
+    rc = load().dash_summary_build_paged(ctypes.byref(p), ctypes.byref(pk), _ptr(K_pool), _ptr(qbar), _ptr(seqlens),
+                                         _ptr(kbar_cache), _ptr(partial_state), _stream(stream))
+    _check(rc, "dash_summary_build_paged")
+    return rc
+
+
+def dash_summary_append_paged(p, pk, k_new, v_new, qbar, K_pool, V_pool, kbar_cache, partial_state, seqlens,
+                              stream=None) -> int:
+    rc = load().dash_summary_append_paged(ctypes.byref(p), ctypes.byref(pk), _ptr(k_new), _ptr(v_new), _ptr(qbar),
+                                          _ptr(K_pool), _ptr(V_pool), _ptr(kbar_cache), _ptr(partial_state),
+                                          _ptr(seqlens), _stream(stream))
+    _check(rc, "dash_summary_append_paged")
+    return rc
+
+
+def dash_decode_paged(p, pk, q, K_pool, V_pool, kbar_cache, seqlens, O, route=None, workspace=None, ws_bytes=None,
+                      stream=None) -> int:
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None and workspace is not None else (ws_bytes or 0)
+    rc = load().dash_decode_paged(ctypes.byref(p), ctypes.byref(pk), _ptr(q), _ptr(K_pool), _ptr(V_pool),
+                                  _ptr(kbar_cache), _ptr(seqlens), _ptr(O),
+                                  ctypes.byref(route) if route is not None else None, _ptr(workspace), ws_bytes,
+                                  _stream(stream))
+    _check(rc, "dash_decode_paged")
     return rc

@@ -155,3 +155,59 @@ class DecodeState:
         self._stage.copy_(qkv)
         self._graph.replay()
         return self.O
+
+class PagedDecodeState:
+    """DecodeState on paged K/V pools [num_pages, page_size, h_kv, d] with a page table
+    [batch, max_pages] (device int32) that the caller may rewrite between steps; the summary
+    cache and the incomplete-chunk state stay per sequence.  bf16, d = 128."""
+
+    def __init__(self, batch, capacity, h_q, h_kv, d, *, chunk, alpha, gamma, page_size, num_pages,
+                 page_table, inv_sigma=1.0, device="cuda", qbar=None):
+        self.K = torch.zeros((num_pages, page_size, h_kv, d), dtype=torch.bfloat16, device=device)
+        self.V = torch.zeros_like(self.K)
+        self.page_table = page_table.to(device=device, dtype=torch.int32).contiguous()
+        self.page_size = page_size
+        self.T = capacity // chunk
+        self.kbar = torch.zeros((batch, h_kv, self.T, d), dtype=torch.float32, device=device)
+        self.state = torch.zeros((batch, h_kv, d + 2), dtype=torch.float32, device=device)
+        self.seqlens = torch.zeros(batch, dtype=torch.int32, device=device)
+        self.qbar = qbar
+        self.O = torch.empty((batch, h_q, d), dtype=torch.bfloat16, device=device)
+        row, head = h_kv * d, d
+        self.p = L.params(batch=batch, seqlen=capacity, h_q=h_q, h_kv=h_kv, d_h=d, chunk=chunk, alpha=alpha,
+                          gamma=gamma, inv_sigma=inv_sigma, dtype=L.DASH_BF16,
+                          k_strides=(0, row, head), v_strides=(0, row, head))
+        self.pk = L.paged_kv(self.page_table, page_size, num_pages, page_size * row, page_size * row)
+        ws = L.dash_workspace_size(self.p, L.DASH_OP_DECODE)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.route = None
+
+    def fill(self, K0, V0, lengths, stream=None):
+        """Copy the first lengths[b] prefilled keys/values of K0, V0 [b, L0, h_kv, d] into the
+        sequences' pages and build the summary cache (Eq. 4)."""
+        pt = self.page_table.cpu()
+        for b in range(K0.shape[0]):
+            n = int(lengths[b])
+            for j in range((n + self.page_size - 1) // self.page_size):
+                pid = int(pt[b, j])
+                if not 0 <= pid < self.K.shape[0]:
+                    raise ValueError(f"sequence {b}: page slot {j} holds prefilled tokens but is unmapped ({pid})")
+                t0, t1 = j * self.page_size, min(n, (j + 1) * self.page_size)
+                self.K[pid, :t1 - t0].copy_(K0[b, t0:t1])
+                self.V[pid, :t1 - t0].copy_(V0[b, t0:t1])
+        self.seqlens.copy_(torch.as_tensor(lengths, dtype=torch.int32))
+        L.dash_summary_build_paged(self.p, self.pk, self.K, self.qbar, self.seqlens, self.kbar, self.state,
+                                   stream=stream)
+
+    def append(self, k_new, v_new, stream=None):
+        L.dash_summary_append_paged(self.p, self.pk, k_new, v_new, self.qbar, self.K, self.V, self.kbar,
+                                    self.state, self.seqlens, stream=stream)
+
+    def decode(self, q, stream=None):
+        L.dash_decode_paged(self.p, self.pk, q, self.K, self.V, self.kbar, self.seqlens, self.O, self.route,
+                            self.workspace, stream=stream)
+        return self.O
+
+    def step(self, q, k_new, v_new, stream=None):
+        self.append(k_new, v_new, stream)
+        return self.decode(q, stream)

@@ -52,7 +52,36 @@ Shape make_shape(const dash_params* p)
         s.qs[k] = p->q_strides[k]; s.ks[k] = p->k_strides[k];
         s.vs[k] = p->v_strides[k]; s.os[k] = p->o_strides[k];
     }
+    s.pt = nullptr;
+    s.psz = s.pmax = s.npages = 0;
+    s.kps = s.vps = 0;
     return s;
+}
+
+// Paged caches: checks of the page description (null: contiguous caches, nothing to check) and
+// the Shape fields the kernels address the pools with.
+int check_paged(const dash_params* p, const dash_paged_kv* pk)
+{
+    if (!pk) return DASH_OK;
+    if (!pk->page_table || pk->page_size <= 0 || pk->max_pages <= 0 || pk->num_pages <= 0) return DASH_EINVAL;
+    if (pk->page_size % 64 || pk->page_size % p->chunk) return DASH_EUNSUPPORTED;
+    if ((long long)pk->max_pages * pk->page_size < p->seqlen) return DASH_EINVAL;
+    if (p->dtype != DASH_BF16 || p->d_h != 128) return DASH_EUNSUPPORTED;
+    if (pk->k_page_stride <= 0 || pk->v_page_stride <= 0 || (pk->k_page_stride * 2) % 16 || (pk->v_page_stride * 2) % 16)
+        return DASH_EALIGN;
+    if (reinterpret_cast<uintptr_t>(pk->page_table) & 3u) return DASH_EALIGN;
+    return DASH_OK;
+}
+
+void apply_paged(Shape& s, const dash_paged_kv* pk)
+{
+    if (!pk) return;
+    s.pt = pk->page_table;
+    s.psz = pk->page_size;
+    s.pmax = pk->max_pages;
+    s.npages = pk->num_pages;
+    s.kps = pk->k_page_stride;
+    s.vps = pk->v_page_stride;
 }
 
 long long route_cap(const dash_params* p)
@@ -191,25 +220,41 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     return rc;
 }
 
-int dash_summary_build(const dash_params* p, const void* K_cache, const float* qbar, const int* seqlens,
-                       float* kbar_cache, float* partial_state, void* stream)
+static int summary_build(const dash_params* p, const dash_paged_kv* pk, const void* K_cache, const float* qbar,
+                         const int* seqlens, float* kbar_cache, float* partial_state, void* stream)
 {
     int rc = check_params(p);
     if (rc != DASH_OK) return rc;
+    if ((rc = check_paged(p, pk)) != DASH_OK) return rc;
     if (!K_cache || !qbar || !seqlens || !kbar_cache || !partial_state) return DASH_EINVAL;
     if (!aligned16(K_cache) || !strides_ok(p->k_strides, p->dtype) || !aligned16(qbar)) return DASH_EALIGN;
     if (!aligned4(seqlens) || !aligned4(kbar_cache) || !aligned4(partial_state)) return DASH_EALIGN;
-    const Shape s = make_shape(p);
+    Shape s = make_shape(p);
+    apply_paged(s, pk);
     return launch_status(launch_stage0(s, p->dtype, K_cache, qbar, seqlens, kbar_cache, s.T, partial_state,
                                        static_cast<cudaStream_t>(stream)));
 }
 
-int dash_summary_append(const dash_params* p, const void* k_new, const void* v_new, const float* qbar,
-                        void* K_cache, void* V_cache, float* kbar_cache, float* partial_state, int* seqlens,
-                        void* stream)
+int dash_summary_build(const dash_params* p, const void* K_cache, const float* qbar, const int* seqlens,
+                       float* kbar_cache, float* partial_state, void* stream)
+{
+    return summary_build(p, nullptr, K_cache, qbar, seqlens, kbar_cache, partial_state, stream);
+}
+
+int dash_summary_build_paged(const dash_params* p, const dash_paged_kv* pk, const void* K_pool, const float* qbar,
+                             const int* seqlens, float* kbar_cache, float* partial_state, void* stream)
+{
+    if (!pk) return DASH_EINVAL;
+    return summary_build(p, pk, K_pool, qbar, seqlens, kbar_cache, partial_state, stream);
+}
+
+static int summary_append(const dash_params* p, const dash_paged_kv* pk, const void* k_new, const void* v_new,
+                          const float* qbar, void* K_cache, void* V_cache, float* kbar_cache, float* partial_state,
+                          int* seqlens, void* stream)
 {
     int rc = check_params(p);
     if (rc != DASH_OK) return rc;
+    if ((rc = check_paged(p, pk)) != DASH_OK) return rc;
     if (!k_new || !v_new || !qbar || !K_cache || !V_cache || !kbar_cache || !partial_state || !seqlens)
         return DASH_EINVAL;
     if (p->h_kv > 32) return DASH_EUNSUPPORTED;
@@ -217,17 +262,35 @@ int dash_summary_append(const dash_params* p, const void* k_new, const void* v_n
         return DASH_EALIGN;
     if (!strides_ok(p->k_strides, p->dtype) || !strides_ok(p->v_strides, p->dtype)) return DASH_EALIGN;
     if (!aligned4(seqlens) || !aligned4(kbar_cache) || !aligned4(partial_state)) return DASH_EALIGN;
-    const Shape s = make_shape(p);
+    Shape s = make_shape(p);
+    apply_paged(s, pk);
     return launch_status(launch_append(s, p->dtype, k_new, v_new, qbar, K_cache, V_cache, kbar_cache, s.T,
                                        partial_state, seqlens, static_cast<cudaStream_t>(stream)));
 }
 
-int dash_decode(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
-                const float* kbar_cache, const int* seqlens, void* O, const dash_route_out* route,
-                void* workspace, size_t ws_bytes, void* stream)
+int dash_summary_append(const dash_params* p, const void* k_new, const void* v_new, const float* qbar,
+                        void* K_cache, void* V_cache, float* kbar_cache, float* partial_state, int* seqlens,
+                        void* stream)
+{
+    return summary_append(p, nullptr, k_new, v_new, qbar, K_cache, V_cache, kbar_cache, partial_state, seqlens,
+                          stream);
+}
+
+int dash_summary_append_paged(const dash_params* p, const dash_paged_kv* pk, const void* k_new, const void* v_new,
+                              const float* qbar, void* K_pool, void* V_pool, float* kbar_cache, float* partial_state,
+                              int* seqlens, void* stream)
+{
+    if (!pk) return DASH_EINVAL;
+    return summary_append(p, pk, k_new, v_new, qbar, K_pool, V_pool, kbar_cache, partial_state, seqlens, stream);
+}
+
+static int decode(const dash_params* p, const dash_paged_kv* pk, const void* q, const void* K_cache,
+                  const void* V_cache, const float* kbar_cache, const int* seqlens, void* O,
+                  const dash_route_out* route, void* workspace, size_t ws_bytes, void* stream)
 {
     int rc = check_params(p);
     if (rc != DASH_OK) return rc;
+    if ((rc = check_paged(p, pk)) != DASH_OK) return rc;
     if (!q || !K_cache || !V_cache || !kbar_cache || !seqlens || !O) return DASH_EINVAL;
     if (!aligned16(q) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(O) || !aligned16(kbar_cache))
         return DASH_EALIGN;
@@ -239,7 +302,9 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
     if (L.splits > 1024) return DASH_EUNSUPPORTED;   // the merge step holds at most 1024 split weights
     if (!workspace || ws_bytes < L.total) return DASH_EWORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DASH_EALIGN;
-    const Shape s = make_shape(p);
+    Shape s = make_shape(p);
+    apply_paged(s, pk);
+    if (pk && !dec_tma_supported(s, p->dtype)) return DASH_EUNSUPPORTED;   // paged: the TMA attend only
     char* ws = static_cast<char*>(workspace);
     Routes rt;
     rt.counts = route && route->counts ? route->counts : reinterpret_cast<int*>(ws + L.counts);
@@ -255,6 +320,21 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
     dw.err = reinterpret_cast<int*>(ws + L.err);   // cleared by the routing launch
     return launch_status(launch_decode(s, p->dtype, q, K_cache, V_cache, kbar_cache, s.T, seqlens, O, rt, dw,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+int dash_decode(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
+                const float* kbar_cache, const int* seqlens, void* O, const dash_route_out* route,
+                void* workspace, size_t ws_bytes, void* stream)
+{
+    return decode(p, nullptr, q, K_cache, V_cache, kbar_cache, seqlens, O, route, workspace, ws_bytes, stream);
+}
+
+int dash_decode_paged(const dash_params* p, const dash_paged_kv* pk, const void* q, const void* K_pool,
+                      const void* V_pool, const float* kbar_cache, const int* seqlens, void* O,
+                      const dash_route_out* route, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!pk) return DASH_EINVAL;
+    return decode(p, pk, q, K_pool, V_pool, kbar_cache, seqlens, O, route, workspace, ws_bytes, stream);
 }
 
 const char* dash_status_string(int status)

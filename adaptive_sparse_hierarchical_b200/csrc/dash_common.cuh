@@ -17,7 +17,25 @@ struct Shape {
     int batch, n, hq, hkv, g, d, B, T;   // T = floor(n / B) complete chunks
     float alpha, gamma, inv_sigma;
     long long qs[3], ks[3], vs[3], os[3];
+    // paged decode caches (pt == null: contiguous [b][t][head][d] by ks / vs)
+    const int* pt;                       // page table [batch][pmax]
+    int psz, pmax, npages;               // page size (tokens), pages per sequence, pool pages
+    long long kps, vps;                  // elements between pages of the K / V pools
 };
+
+// Element offset of token t of sequence b, KV head r in a K (st = ks, ps = kps) or V cache; -1
+// when the token's page is unmapped (a page id outside [0, npages), or t beyond the table), so
+// that callers skip the access instead of leaving the pool.
+__device__ __forceinline__ long long kv_off(const Shape& s, const long long st[3], long long ps, int b, long long t,
+                                            int r)
+{
+    if (!s.pt) return (long long)b * st[0] + t * st[1] + (long long)r * st[2];
+    const long long slot = t / s.psz;
+    if (slot >= s.pmax) return -1;
+    const int pg = s.pt[(long long)b * s.pmax + slot];
+    if (pg < 0 || pg >= s.npages) return -1;
+    return (long long)pg * ps + (t % s.psz) * st[1] + (long long)r * st[2];
+}
 
 // Route storage: where Stage 1 writes and Stage 2 reads.
 struct Routes {

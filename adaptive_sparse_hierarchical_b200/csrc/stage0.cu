@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
     const int cfull = min(n / s.B, kbar_T);
     const bool complete = c < cfull;
     if (!complete && !(state && c == n / s.B)) return;
-    const int t0 = c * s.B, t1 = complete ? t0 + s.B : n;
+    const int t0 = c * s.B, t1c = complete ? t0 + s.B : n;
 
     const int grp = lane / L::LPK, sub = lane % L::LPK;
     const float qscale = kLog2e * rsqrtf((float)D);
@@ -71,7 +71,12 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
 
     Run<L::EPL> run;
     run.init();
-    const T* kb = K + (long long)b * s.ks[0] + (long long)r * s.ks[2] + sub * L::EPL;
+    // the chunk's keys are consecutive rows (of a page, for paged caches: a chunk never
+    // straddles two pages), so one base serves the whole chunk; no page lookup for an empty
+    // chunk, and a chunk on an unmapped page reads nothing (its summary is left undefined)
+    const long long koff = t1c > t0 ? kv_off(s, s.ks, s.kps, b, t0, r) : 0;
+    const T* kb = K + (koff < 0 ? 0 : koff) + sub * L::EPL;
+    const int t1 = koff < 0 ? t0 : t1c;
     constexpr int U = 4;
     // the loop bounds are warp-uniform so that every lane reaches the shuffles
     for (int base = t0; base < t1; base += U * L::KPI) {
@@ -79,7 +84,7 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             int tt = base + u * L::KPI + grp;
-            if (tt < t1) Vec<T>::load(kb + (long long)tt * s.ks[1], kv[u]);
+            if (tt < t1) Vec<T>::load(kb + (long long)(tt - t0) * s.ks[1], kv[u]);
             else for (int e = 0; e < L::EPL; ++e) kv[u][e] = 0.f;
         }
 #pragma unroll
@@ -142,11 +147,10 @@ __global__ void append_kernel(Shape s, const T* __restrict__ k_new, const T* __r
         constexpr int EPL = Vec<T>::N, PIECES = D / EPL;
         const T* kn = k_new + ((long long)b * s.hkv + r) * D;
         const T* vn = v_new + ((long long)b * s.hkv + r) * D;
-        if (lane < PIECES) {
-            T* kd = Kc + (long long)b * s.ks[0] + (long long)L * s.ks[1] + (long long)r * s.ks[2];
-            T* vd = Vc + (long long)b * s.vs[0] + (long long)L * s.vs[1] + (long long)r * s.vs[2];
-            reinterpret_cast<uint4*>(kd)[lane] = reinterpret_cast<const uint4*>(kn)[lane];
-            reinterpret_cast<uint4*>(vd)[lane] = reinterpret_cast<const uint4*>(vn)[lane];
+        const long long ko = kv_off(s, s.ks, s.kps, b, L, r), vo = kv_off(s, s.vs, s.vps, b, L, r);
+        if (lane < PIECES && ko >= 0 && vo >= 0) {   // (an unmapped page is not written)
+            reinterpret_cast<uint4*>(Kc + ko)[lane] = reinterpret_cast<const uint4*>(kn)[lane];
+            reinterpret_cast<uint4*>(Vc + vo)[lane] = reinterpret_cast<const uint4*>(vn)[lane];
         }
         constexpr int E = D / 32;
         float kv[E], dot = 0.f;

@@ -486,11 +486,12 @@ cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* 
 {
     cudaError_t e = launch_route_decode(s, dtype, q, kbar, kbar_T, seqlens, rt, ws.x, ws.err, st);
     if (e != cudaSuccess) return e;
-    if (dec_tma_supported(s, dtype) && !legacy_stage2()) {
+    if (dec_tma_supported(s, dtype) && (!legacy_stage2() || s.pt)) {   // paged caches: the TMA path only
         e = launch_dec_attend_tma(s, q, Kc, Vc, seqlens, rt, ws.part, O, ws.err, st);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
+    if (s.pt) return cudaErrorInvalidValue;
     if (dtype == DASH_BF16)
         return s.d == 128 ? dec_bf16_d<128>(s, q, Kc, Vc, seqlens, rt, ws, O, st)
                           : dec_bf16_d<64>(s, q, Kc, Vc, seqlens, rt, ws, O, st);

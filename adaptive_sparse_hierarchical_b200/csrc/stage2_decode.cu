@@ -125,12 +125,19 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 float bdummy;
                 job(k, x, &key0, &bdummy);
                 const int bb = x / s.hkv, r = x % s.hkv;
+                // coordinates (row, sequence), or (row in page, page) for paged caches: a 64-key
+                // tile never straddles two pages (the page size is a multiple of 64 and of B)
+                int c2 = key0, c3 = bb;
+                if (s.pt) {
+                    c2 = key0 % s.psz;
+                    c3 = s.pt[(long long)bb * s.pmax + key0 / s.psz];
+                }
                 const uint32_t dst = base + slot * kSlotB, fb = bar_full + 8 * slot;
                 tc::mbar_expect_tx(fb, kSlotB);
-                tc::tma_load_4d(dst, &tmK, fb, 0, r, key0, bb);
-                tc::tma_load_4d(dst + kHalf, &tmK, fb, 64, r, key0, bb);
-                tc::tma_load_4d(dst + 2 * kHalf, &tmV, fb, 0, r, key0, bb);
-                tc::tma_load_4d(dst + 3 * kHalf, &tmV, fb, 64, r, key0, bb);
+                tc::tma_load_4d(dst, &tmK, fb, 0, r, c2, c3);
+                tc::tma_load_4d(dst + kHalf, &tmK, fb, 64, r, c2, c3);
+                tc::tma_load_4d(dst + 2 * kHalf, &tmV, fb, 0, r, c2, c3);
+                tc::tma_load_4d(dst + 3 * kHalf, &tmV, fb, 64, r, c2, c3);
             }
             if (*abort)   // let copies still in flight land before the block's shared memory goes away
                 for (int k = 0; k < kNSd; ++k)
@@ -367,13 +374,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_d()
     return fn;
 }
 
-bool map_kv(CUtensorMap* map, const void* ptr, const Shape& s, const long long st[3])
+// 4-D map (d, head, row, sequence) over a contiguous cache, or (d, head, row in page, page) over
+// a paged pool (ps = elements between pages)
+bool map_kv(CUtensorMap* map, const void* ptr, const Shape& s, const long long st[3], long long ps)
 {
     auto fn = encode_fn_d();
     if (!fn) return false;
     cuuint64_t dims[4] = {128, (cuuint64_t)s.hkv, (cuuint64_t)s.n, (cuuint64_t)s.batch};
     cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
     if (s.batch == 1) strides[2] = strides[1] * (cuuint64_t)s.n;
+    if (s.pt) {
+        dims[2] = (cuuint64_t)s.psz;
+        dims[3] = (cuuint64_t)s.npages;
+        strides[2] = (cuuint64_t)ps * 2;
+    }
     cuuint32_t box[4] = {64, 1, 64, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
@@ -405,7 +419,7 @@ cudaError_t launch_dec_attend_tma(const Shape& s, const void* q, const void* Kc,
                                   const Routes& rt, float* part, void* O, int* err, cudaStream_t st)
 {
     CUtensorMap mk, mv;
-    if (!map_kv(&mk, Kc, s, s.ks) || !map_kv(&mv, Vc, s, s.vs)) return cudaErrorInvalidValue;
+    if (!map_kv(&mk, Kc, s, s.ks, s.kps) || !map_kv(&mv, Vc, s, s.vs, s.vps)) return cudaErrorInvalidValue;
     const size_t smem = 1024 + kNSd * kSlotB + 16 * kNSd + 16 + kCons * 16 * 2 * 4 + (kMaxBR + 1) * 4 +
                         16 * 128 * 4 + 2 * kMaxJobs * 4;
     cudaError_t e = cudaFuncSetAttribute(dec_attend_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -139,6 +139,35 @@ int dash_decode(const dash_params* p, const void* q, const void* K_cache, const 
                 const float* kbar_cache, const int* seqlens, void* O, const dash_route_out* route,
                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Paged K/V caches for incremental decoding (a serving layout; the paper's kernels take
+ * contiguous caches).  K and V live in pools of pages [num_pages][page_size][h_kv][d_h]: token t
+ * of sequence b sits in page page_table[b * max_pages + t / page_size], row t % page_size.
+ * p->k_strides / p->v_strides give the row (token) stride in [1] and the head stride in [2], in
+ * elements ([0] is unused); k_page_stride / v_page_stride are the elements between consecutive
+ * pages.  page_size must be a multiple of 64 and of the chunk B (a chunk never straddles two
+ * pages), max_pages * page_size >= p->seqlen, and every page that holds a position < seqlen_b
+ * (after the append) must be mapped.  bf16 with d_h = 128 only (other configurations return
+ * DASH_EUNSUPPORTED).  The page table is read by the kernels on the device; it may change
+ * between calls (the caller owns the allocation policy).  Results equal the contiguous-cache
+ * calls bit for bit. */
+typedef struct {
+    const int* page_table;            /* device int32 [batch, max_pages] */
+    int max_pages, page_size, num_pages;
+    long long k_page_stride, v_page_stride;
+} dash_paged_kv;
+
+/* dash_summary_build / dash_summary_append / dash_decode on paged caches (same arguments plus
+ * the page description; K_pool / V_pool take the place of K_cache / V_cache). */
+int dash_summary_build_paged(const dash_params* p, const dash_paged_kv* pk, const void* K_pool,
+                             const float* qbar, const int* seqlens, float* kbar_cache, float* partial_state,
+                             void* stream);
+int dash_summary_append_paged(const dash_params* p, const dash_paged_kv* pk, const void* k_new,
+                              const void* v_new, const float* qbar, void* K_pool, void* V_pool,
+                              float* kbar_cache, float* partial_state, int* seqlens, void* stream);
+int dash_decode_paged(const dash_params* p, const dash_paged_kv* pk, const void* q, const void* K_pool,
+                      const void* V_pool, const float* kbar_cache, const int* seqlens, void* O,
+                      const dash_route_out* route, void* workspace, size_t ws_bytes, void* stream);
+
 /* dash_decode without a workspace, for callers that cannot obtain device memory of their own
  * (for example a plugin inside a runtime that owns every device allocation and gives it no
  * allocator, or a service that must not grow its device footprint once running).  The paper has

@@ -27,7 +27,8 @@ def test_header_symbols_exported():
     syms = L.header_symbols()
     assert set(syms) == {"dash_workspace_size", "dash_route_capacity", "dash_prefill", "dash_prefill_stage",
                          "dash_summary_build", "dash_error_word_offset", "dash_decode_noalloc",
-                         "dash_summary_append", "dash_decode", "dash_status_string"}
+                         "dash_summary_append", "dash_decode", "dash_status_string", "dash_summary_build_paged",
+                         "dash_summary_append_paged", "dash_decode_paged"}
     lib = D.load()
     for s in syms:
         assert hasattr(lib, s), s
@@ -84,3 +85,34 @@ def test_missing_pointers_workspace_and_alignment():
 def test_status_strings():
     for rc in (0, -1, -2, -3, -4, -5, -99):
         assert isinstance(L.dash_status_string(rc), str) and L.dash_status_string(rc)
+
+
+@pytest.mark.parametrize("kw,pkw,code", [
+    (dict(), dict(page_size=96), L.DASH_EUNSUPPORTED),        # not a multiple of 64
+    (dict(chunk=128), dict(page_size=64), L.DASH_EUNSUPPORTED),   # a chunk would straddle two pages
+    (dict(), dict(max_pages=7), L.DASH_EINVAL),               # 7 * 128 < seqlen 1024
+    (dict(), dict(page_size=0), L.DASH_EINVAL),
+    (dict(), dict(num_pages=0), L.DASH_EINVAL),
+    (dict(), dict(page_table=0), L.DASH_EINVAL),
+    (dict(d_h=64, q_strides=(1024 * 8 * 64, 8 * 64, 64), k_strides=(1024 * 2 * 64, 128, 64),
+          v_strides=(1024 * 2 * 64, 128, 64), o_strides=(1024 * 8 * 64, 8 * 64, 64)), dict(), L.DASH_EUNSUPPORTED),
+    (dict(dtype=L.DASH_F32), dict(), L.DASH_EUNSUPPORTED),
+    (dict(), dict(k_page_stride=128 * 256 + 4), L.DASH_EALIGN),   # pages 8 bytes apart from a 16-byte boundary
+])
+def test_paged_description_rejected_before_launch(kw, pkw, code):
+    """The paged entry points check the page description before touching the device."""
+    base = dict(page_table=256, max_pages=8, page_size=128, num_pages=64, k_page_stride=128 * 256,
+                v_page_stride=128 * 256)
+    base.update(pkw)
+    pk = L.dash_paged_kv(base["page_table"], base["max_pages"], base["page_size"], base["num_pages"],
+                         base["k_page_stride"], base["v_page_stride"])
+    p = _p(**kw)
+    lib = D.load()
+    assert lib.dash_decode_paged(ctypes.byref(p), ctypes.byref(pk), 256, 256, 256, 256, 256, 256, None, 256,
+                                 1 << 40, None) == code
+    assert lib.dash_summary_build_paged(ctypes.byref(p), ctypes.byref(pk), 256, 256, 256, 256, 256, None) == code
+    assert lib.dash_summary_append_paged(ctypes.byref(p), ctypes.byref(pk), 256, 256, 256, 256, 256, 256, 256,
+                                         256, None) == code
+    # a null page description is an error, not the contiguous layout
+    assert lib.dash_decode_paged(ctypes.byref(_p()), None, 256, 256, 256, 256, 256, 256, None, 256, 1 << 40,
+                                 None) == L.DASH_EINVAL
