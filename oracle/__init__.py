@@ -59,6 +59,7 @@ def _load():
         lib.orc_rows.argtypes = [cfgp, fp, ip, ctypes.c_int, fp, llp, fp, llp, dp, ctypes.c_int,
                                  ctypes.c_int, dp, ip, dp, dp, dp, ctypes.c_int]
         lib.orc_num_threads.restype = ctypes.c_int
+        lib.orc_backward.argtypes = [cfgp, fp, fp, fp, fp, fp, dp, dp, dp, dp, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -223,3 +224,23 @@ def decode(q, K_cache, V_cache, qbar, seqlens, *, chunk, alpha, gamma, inv_sigma
     if want_route:
         return res[0][:, 0], res[1]
     return res[:, 0]
+
+
+def backward(Q, K, V, qbar, dO, *, chunk, alpha, gamma, inv_sigma=1.0, nthreads: int = 0):
+    """Gradients of L = sum(dO * O) for the causal prefill forward (prefill()) with respect to
+    Q, K, V and qbar, in float64.  Q, dO [b, n, h_q, d]; K, V [b, n, h_kv, d]; qbar [h_kv, d].
+    Returns dQ, dK, dV (same shapes) and dqbar [h_kv, d] (summed over the batch).  The routed
+    support is held fixed (it is piecewise constant in the inputs)."""
+    Q, K, V, qbar, dO = (_f32(a) for a in (Q, K, V, qbar, dO))
+    b, n, hq, d = Q.shape
+    hkv = K.shape[2]
+    dQ = np.zeros(Q.shape, dtype=np.float64)
+    dK = np.zeros(K.shape, dtype=np.float64)
+    dV = np.zeros(V.shape, dtype=np.float64)
+    dqbar = np.zeros((hkv, d), dtype=np.float64)
+    cf = _cfg(b, n, hq, hkv, d, chunk, alpha, gamma, inv_sigma)
+    _load().orc_backward(ctypes.byref(cf), _p(Q, ctypes.c_float), _p(K, ctypes.c_float), _p(V, ctypes.c_float),
+                         _p(qbar, ctypes.c_float), _p(dO, ctypes.c_float), _p(dQ, ctypes.c_double),
+                         _p(dK, ctypes.c_double), _p(dV, ctypes.c_double), _p(dqbar, ctypes.c_double),
+                         int(nthreads))
+    return dQ, dK, dV, dqbar

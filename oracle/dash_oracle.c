@@ -1,5 +1,6 @@
 /*
- * dash_oracle.c -- plain float64 CPU oracle for the DashAttention forward pass.
+ * dash_oracle.c -- plain float64 CPU oracle for the DashAttention forward pass and its
+ * backward pass (gradients of Q, K, V and the Stage 0 query qbar; orc_backward at the end).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call this file;
  * only the tests, the smoke check and the benchmark's CPU-baseline / reference legs use it.
@@ -379,4 +380,207 @@ int orc_num_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Backward pass.  The paper review page (section 3, after Eq. 9) states that the output is    */
+/* differentiable in q, k, v and in the prior g, so that the gradient reaches the Stage 1      */
+/* entmax scores and through them the Stage 0 summaries (the Stage 2 kernel row: the training  */
+/* backward reuses the routed support, the entmax Jacobian being sparse).  The routed support  */
+/* R itself is piecewise constant, so no gradient flows through the choice of R.               */
+/*                                                                                             */
+/* Chain, for the scalar L = sum dO . O, per (b, r) and position i (g heads h of group r):     */
+/*   Stage 2 (Prop. 4.1): p = softmax(z + d) over R u D;  dv_j += p_j dO;  dp_j = dO . v_j;     */
+/*     ds_j = p_j (dp_j - sum_t p_t dp_t);  dq += ds_j k_j / sqrt(d);  dk_j += ds_j q / sqrt(d); */
+/*     dbias_c = sum over the group's heads and the tokens j of chunk c of ds_j.               */
+/*   bias_c = (log w_c - mean_{R} log w) / sigma  =>  dlog w_c = (dbias_c - mean_R dbias)/sigma, */
+/*     dw_c = dlog w_c / w_c;  w = mean_h what^(h)  =>  dwhat^(h)_c = dw_c / g.                 */
+/*   alpha-entmax(theta), theta = gamma zbar: on the support the Jacobian is                   */
+/*     diag(s) - s s^T / sum s with s_c = what_c^(2 - alpha)  (zero off the support), so        */
+/*     dtheta = s * dwhat - s (s . dwhat) / sum s;  dzbar = gamma dtheta.                       */
+/*   Eq. 6: dq += dzbar_c kbar_c / sqrt(d);  dkbar_c += dzbar_c q / sqrt(d).                    */
+/*   Eq. 4: kbar_c = sum_t pi_t k_t, pi = softmax_t(<qbar, k_t>/sqrt(d)):                       */
+/*     dk_t += pi_t dkbar_c + pi_t (k_t . dkbar_c - kbar_c . dkbar_c) qbar / sqrt(d);           */
+/*     dqbar += sum_t pi_t (k_t . dkbar_c - kbar_c . dkbar_c) k_t / sqrt(d).                    */
+/*                                                                                             */
+/* Layouts (contiguous): Q, dO, dQ [batch][n][h_q][d]; K, V, dK, dV [batch][n][h_kv][d];        */
+/* qbar, dqbar [h_kv][d] (dqbar sums over the batch).                                          */
+/* ------------------------------------------------------------------------------------------ */
+
+static void bwd_pair(const orc_cfg* cf, const float* Q, const float* K, const float* V, const float* qbar,
+                     const float* dO, double* dQ, double* dK, double* dV, double* dqbar_part, int b, int r)
+{
+    const int n = cf->seqlen, d = cf->d, B = cf->chunk, hq = cf->h_q, hkv = cf->h_kv, g = hq / hkv;
+    const int T = n / B;
+    const double scale = 1.0 / sqrt((double)d), am1 = cf->alpha - 1.0;
+    const long long ks[3] = {(long long)n * hkv * d, (long long)hkv * d, d};
+    const int Tc = T > 0 ? T : 1;
+    double* kbar = (double*)calloc((size_t)Tc * d, sizeof(double));
+    double* dkbar = (double*)calloc((size_t)Tc * d, sizeof(double));
+    double* what = (double*)calloc((size_t)g * Tc, sizeof(double));
+    double* w = (double*)calloc((size_t)Tc, sizeof(double));
+    double* bias = (double*)calloc((size_t)Tc, sizeof(double));
+    double* dbias = (double*)calloc((size_t)Tc, sizeof(double));
+    double* x = (double*)calloc((size_t)Tc, sizeof(double));
+    double* zl = (double*)malloc(sizeof(double) * (size_t)(n + B));
+    double* pl = (double*)malloc(sizeof(double) * (size_t)(n + B));
+    int* idx = (int*)malloc(sizeof(int) * (size_t)(n + B));
+    for (int c = 0; c < T; ++c)
+        orc_chunk_summary(cf, K, ks, qbar, b, r, c * B, (c + 1) * B, kbar + (long long)c * d);
+
+#define KV_AT(base, j) ((base) + (((long long)b * n + (j)) * hkv + r) * d)
+#define Q_AT(base, i, hh) ((base) + (((long long)b * n + (i)) * hq + (long long)r * g + (hh)) * d)
+
+    for (int i = 0; i < n; ++i) {
+        const int ci = i / B;
+        const int nvis = ci < T ? ci : T;
+        /* Stage 1 forward: per-head weights, their average, the routed set and the biases */
+        int nR = 0;
+        double mu = 0.0;
+        for (int c = 0; c < nvis; ++c) { w[c] = 0.0; dbias[c] = 0.0; }
+        for (int hh = 0; hh < g && nvis > 0; ++hh) {
+            const float* q = Q_AT(Q, i, hh);
+            for (int c = 0; c < nvis; ++c) {
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e) dot += (double)q[e] * kbar[(long long)c * d + e];
+                x[c] = am1 * cf->gamma * dot * scale;
+            }
+            const double tau = orc_entmax_threshold(x, nvis, cf->alpha);
+            for (int c = 0; c < nvis; ++c) {
+                const double u = x[c] - tau;
+                what[(long long)hh * Tc + c] = u > 0.0 ? pow(u, 1.0 / am1) : 0.0;
+                w[c] += what[(long long)hh * Tc + c] / g;
+            }
+        }
+        for (int c = 0; c < nvis; ++c)
+            if (w[c] > 0.0) { ++nR; mu += log(w[c]); }
+        if (nR) mu /= nR;
+        for (int c = 0; c < nvis; ++c) bias[c] = w[c] > 0.0 ? (log(w[c]) - mu) * cf->inv_sigma : 0.0;
+
+        /* Stage 2 forward and backward, one head at a time */
+        int m = 0;
+        for (int c = 0; c < nvis; ++c)
+            if (w[c] > 0.0)
+                for (int j = c * B; j < (c + 1) * B; ++j) idx[m++] = j;
+        const int mR = m;
+        for (int j = ci * B; j <= i; ++j) idx[m++] = j;
+        for (int hh = 0; hh < g; ++hh) {
+            const float* q = Q_AT(Q, i, hh);
+            const float* go = Q_AT(dO, i, hh);
+            double* gq = Q_AT(dQ, i, hh);
+            double zmax = -INFINITY;
+            for (int t = 0; t < m; ++t) {
+                const float* k = KV_AT(K, idx[t]);
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e) dot += (double)q[e] * (double)k[e];
+                zl[t] = dot * scale + (t < mR ? bias[idx[t] / B] : 0.0);
+                if (zl[t] > zmax) zmax = zl[t];
+            }
+            double den = 0.0;
+            for (int t = 0; t < m; ++t) { pl[t] = exp(zl[t] - zmax); den += pl[t]; }
+            double delta = 0.0;
+            for (int t = 0; t < m; ++t) {
+                pl[t] /= den;
+                const float* v = KV_AT(V, idx[t]);
+                double dp = 0.0;
+                for (int e = 0; e < d; ++e) dp += (double)go[e] * (double)v[e];
+                zl[t] = dp;                                   /* zl now holds dp_t */
+                delta += pl[t] * dp;
+            }
+            for (int t = 0; t < m; ++t) {
+                const int j = idx[t];
+                const double ds = pl[t] * (zl[t] - delta);
+                const float* k = KV_AT(K, j);
+                double* gk = KV_AT(dK, j);
+                double* gv = KV_AT(dV, j);
+                for (int e = 0; e < d; ++e) {
+                    gv[e] += pl[t] * (double)go[e];
+                    gk[e] += ds * (double)q[e] * scale;
+                    gq[e] += ds * (double)k[e] * scale;
+                }
+                if (t < mR) dbias[j / B] += ds;
+            }
+        }
+
+        /* Stage 1 backward through the bias, the GQA mean and each head's entmax */
+        if (nR > 0) {
+            double mdb = 0.0;
+            for (int c = 0; c < nvis; ++c) if (w[c] > 0.0) mdb += dbias[c];
+            mdb /= nR;
+            for (int hh = 0; hh < g; ++hh) {
+                const double* wh = what + (long long)hh * Tc;
+                double s1 = 0.0, s2 = 0.0;
+                for (int c = 0; c < nvis; ++c) {
+                    if (!(wh[c] > 0.0)) continue;
+                    const double s = pow(wh[c], 2.0 - cf->alpha);
+                    const double dwh = cf->inv_sigma * (dbias[c] - mdb) / w[c] / g;
+                    s1 += s;
+                    s2 += s * dwh;
+                }
+                const float* q = Q_AT(Q, i, hh);
+                double* gq = Q_AT(dQ, i, hh);
+                for (int c = 0; c < nvis; ++c) {
+                    if (!(wh[c] > 0.0)) continue;
+                    const double s = pow(wh[c], 2.0 - cf->alpha);
+                    const double dwh = cf->inv_sigma * (dbias[c] - mdb) / w[c] / g;
+                    const double dz = cf->gamma * (s * dwh - s * s2 / s1);
+                    for (int e = 0; e < d; ++e) {
+                        gq[e] += dz * kbar[(long long)c * d + e] * scale;
+                        dkbar[(long long)c * d + e] += dz * (double)q[e] * scale;
+                    }
+                }
+            }
+        }
+    }
+
+    /* Stage 0 backward (Eq. 4) */
+    for (int c = 0; c < T; ++c) {
+        const double* kb = kbar + (long long)c * d;
+        const double* gkb = dkbar + (long long)c * d;
+        double amax = -INFINITY, den = 0.0, kbg = 0.0;
+        for (int e = 0; e < d; ++e) kbg += kb[e] * gkb[e];
+        for (int t = 0; t < B; ++t) {
+            const float* k = KV_AT(K, c * B + t);
+            double dot = 0.0;
+            for (int e = 0; e < d; ++e) dot += (double)qbar[r * d + e] * (double)k[e];
+            zl[t] = dot * scale;
+            if (zl[t] > amax) amax = zl[t];
+        }
+        for (int t = 0; t < B; ++t) { pl[t] = exp(zl[t] - amax); den += pl[t]; }
+        for (int t = 0; t < B; ++t) {
+            const float* k = KV_AT(K, c * B + t);
+            double* gk = KV_AT(dK, c * B + t);
+            const double pi = pl[t] / den;
+            double kg = 0.0;
+            for (int e = 0; e < d; ++e) kg += (double)k[e] * gkb[e];
+            const double da = pi * (kg - kbg);
+            for (int e = 0; e < d; ++e) {
+                gk[e] += pi * gkb[e] + da * (double)qbar[r * d + e] * scale;
+                dqbar_part[e] += da * (double)k[e] * scale;
+            }
+        }
+    }
+#undef KV_AT
+#undef Q_AT
+    free(kbar); free(dkbar); free(what); free(w); free(bias); free(dbias); free(x);
+    free(zl); free(pl); free(idx);
+}
+
+void orc_backward(const orc_cfg* cf, const float* Q, const float* K, const float* V, const float* qbar,
+                  const float* dO, double* dQ, double* dK, double* dV, double* dqbar, int nthreads)
+{
+    const int d = cf->d, hkv = cf->h_kv;
+    const long long pairs = (long long)cf->batch * hkv;
+    double* part = (double*)calloc((size_t)pairs * d, sizeof(double));
+#ifdef _OPENMP
+    #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads > 0 ? nthreads : omp_get_max_threads())
+#endif
+    for (long long u = 0; u < pairs; ++u)
+        bwd_pair(cf, Q, K, V, qbar, dO, dQ, dK, dV, part + u * d, (int)(u / hkv), (int)(u % hkv));
+    for (int r = 0; r < hkv; ++r)
+        for (int e = 0; e < d; ++e) dqbar[(long long)r * d + e] = 0.0;
+    for (long long u = 0; u < pairs; ++u)
+        for (int e = 0; e < d; ++e) dqbar[(u % hkv) * d + e] += part[u * d + e];
+    free(part);
+    (void)nthreads;
 }
