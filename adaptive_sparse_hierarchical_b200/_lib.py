@@ -16,7 +16,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "dash.h")
 
 DASH_OK, DASH_EINVAL, DASH_EUNSUPPORTED, DASH_EWORKSPACE, DASH_EALIGN, DASH_ELAUNCH = 0, -1, -2, -3, -4, -5
 DASH_F32, DASH_BF16 = 0, 1
-DASH_OP_PREFILL, DASH_OP_DECODE = 0, 1
+DASH_OP_PREFILL, DASH_OP_DECODE, DASH_OP_BACKWARD = 0, 1, 2
 DASH_STAGE0, DASH_STAGE1, DASH_STAGE2 = 0, 1, 2
 
 
@@ -80,6 +80,8 @@ def load():
         lib.dash_summary_append_paged.restype = ctypes.c_int
         lib.dash_decode_paged.argtypes = [P, PK, vp, vp, vp, vp, vp, vp, R, vp, sz, vp]
         lib.dash_decode_paged.restype = ctypes.c_int
+        lib.dash_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, R, vp, vp, vp, vp, vp, sz, vp]
+        lib.dash_backward.restype = ctypes.c_int
         lib.dash_status_string.argtypes = [ctypes.c_int]
         lib.dash_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -223,4 +225,14 @@ def dash_decode_paged(p, pk, q, K_pool, V_pool, kbar_cache, seqlens, O, route=No
                                   ctypes.byref(route) if route is not None else None, _ptr(workspace), ws_bytes,
                                   _stream(stream))
     _check(rc, "dash_decode_paged")
+    return rc
+
+
+def dash_backward(p, Q, K, V, qbar, dO, kbar, route, dQ, dK, dV, dqbar, workspace=None, ws_bytes=None,
+                  stream=None) -> int:
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None and workspace is not None else (ws_bytes or 0)
+    rc = load().dash_backward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(qbar), _ptr(dO), _ptr(kbar),
+                              ctypes.byref(route) if route is not None else None, _ptr(dQ), _ptr(dK), _ptr(dV),
+                              _ptr(dqbar), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dash_backward")
     return rc

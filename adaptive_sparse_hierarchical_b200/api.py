@@ -69,6 +69,25 @@ class Prefill:
                        stream=stream)
         return self.O
 
+    def backward(self, dO, stream=None):
+        """Gradients (fp32) of sum(dO * O) for the last call: dQ, dK, dV and dqbar [h_kv, d].  Needs
+        want_route=True (the backward reads the forward's route lists and summaries)."""
+        if self.route is None:
+            raise ValueError("Prefill.backward needs the route lists: construct with want_route=True")
+        assert dO.shape == self.O.shape and dO.dtype == self.O.dtype and dO.stride() == self.O.stride()
+        if getattr(self, "_grads", None) is None:
+            dev = self.Q.device
+            ws = L.dash_workspace_size(self.p, L.DASH_OP_BACKWARD)
+            self._bws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+            self._grads = (torch.empty(self.Q.shape, dtype=torch.float32, device=dev),
+                           torch.empty(self.K.shape, dtype=torch.float32, device=dev),
+                           torch.empty(self.V.shape, dtype=torch.float32, device=dev),
+                           torch.empty((self.K.shape[2], self.Q.shape[3]), dtype=torch.float32, device=dev))
+        dQ, dK, dV, dqbar = self._grads
+        L.dash_backward(self.p, self.Q, self.K, self.V, self.qbar, dO, self.kbar, self.route, dQ, dK, dV, dqbar,
+                        self._bws, stream=stream)
+        return dQ, dK, dV, dqbar
+
 
 def prefill(Q, K, V, qbar, **kw):
     return Prefill(Q, K, V, qbar, **kw)()

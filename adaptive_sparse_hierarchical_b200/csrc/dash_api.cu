@@ -129,6 +129,27 @@ DecodeLayout decode_layout(const dash_params* p)
     return L;
 }
 
+struct BackwardLayout { size_t lse, del, dzbar, tcnt, toff, tpos, tent, dkbar, qpart, total; };
+BackwardLayout backward_layout(const dash_params* p)
+{
+    BackwardLayout L;
+    const size_t bh = (size_t)p->batch * p->h_kv, rows = (size_t)p->batch * p->h_q * p->seqlen;
+    const size_t T = (size_t)(p->seqlen / p->chunk), Tn = T > 0 ? T : 1;
+    const size_t cap = (size_t)route_cap(p) > 0 ? (size_t)route_cap(p) : 1;
+    const size_t g = (size_t)(p->h_q / p->h_kv);
+    L.lse = 0;
+    L.del = L.lse + up(rows * 4);
+    L.dzbar = L.del + up(rows * 4);
+    L.tcnt = L.dzbar + up(bh * cap * g * 4);
+    L.toff = L.tcnt + up(bh * Tn * 4);
+    L.tpos = L.toff + up(bh * (Tn + 1) * 4);
+    L.tent = L.tpos + up(bh * cap * 4);
+    L.dkbar = L.tent + up(bh * cap * 4);
+    L.qpart = L.dkbar + up(bh * Tn * p->d_h * 4);
+    L.total = L.qpart + up(bh * Tn * p->d_h * 4);
+    return L;
+}
+
 int launch_status(cudaError_t e) { return e == cudaSuccess ? DASH_OK : DASH_ELAUNCH; }
 
 }  // namespace
@@ -140,6 +161,7 @@ size_t dash_workspace_size(const dash_params* p, int op)
     if (check_params(p) != DASH_OK) return 0;
     if (op == DASH_OP_PREFILL) return prefill_layout(p).total;
     if (op == DASH_OP_DECODE) return decode_layout(p).total;
+    if (op == DASH_OP_BACKWARD) return backward_layout(p).total;
     return 0;
 }
 
@@ -351,3 +373,47 @@ const char* dash_status_string(int status)
 }
 
 }  // extern "C"
+
+extern "C" int dash_backward(const dash_params* p, const void* Q, const void* K, const void* V, const float* qbar,
+                             const void* dO, const float* kbar, const dash_route_out* route, float* dQ, float* dK,
+                             float* dV, float* dqbar, void* workspace, size_t ws_bytes, void* stream)
+{
+    int rc = check_params(p);
+    if (rc != DASH_OK) return rc;
+    if (!Q || !K || !V || !qbar || !dO || !kbar || !route || !route->counts || !route->chunk_idx || !route->bias ||
+        !dQ || !dK || !dV || !dqbar)
+        return DASH_EINVAL;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(qbar)) return DASH_EALIGN;
+    if (!strides_ok(p->q_strides, p->dtype) || !strides_ok(p->k_strides, p->dtype) ||
+        !strides_ok(p->v_strides, p->dtype) || !strides_ok(p->o_strides, p->dtype))
+        return DASH_EALIGN;
+    if (!aligned4(kbar) || !aligned4(route->counts) || !aligned4(route->chunk_idx) || !aligned4(route->bias) ||
+        !aligned4(dQ) || !aligned4(dK) || !aligned4(dV) || !aligned4(dqbar))
+        return DASH_EALIGN;
+    const Shape s = make_shape(p);
+    // shared memory of the query-major kernel grows with the group's chunk logits (g * T floats)
+    if (backward_rows_smem(s) > 220 * 1024 || backward_keys_smem(s) > 220 * 1024) return DASH_EUNSUPPORTED;
+    const BackwardLayout L = backward_layout(p);
+    if (!workspace || ws_bytes < L.total) return DASH_EWORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DASH_EALIGN;
+    char* ws = static_cast<char*>(workspace);
+    BackwardWs bw;
+    bw.lse = reinterpret_cast<float*>(ws + L.lse);
+    bw.del = reinterpret_cast<float*>(ws + L.del);
+    bw.dzbar = reinterpret_cast<float*>(ws + L.dzbar);
+    bw.tcnt = reinterpret_cast<int*>(ws + L.tcnt);
+    bw.toff = reinterpret_cast<int*>(ws + L.toff);
+    bw.tpos = reinterpret_cast<int*>(ws + L.tpos);
+    bw.tent = reinterpret_cast<int*>(ws + L.tent);
+    bw.dkbar = reinterpret_cast<float*>(ws + L.dkbar);
+    bw.qpart = reinterpret_cast<float*>(ws + L.qpart);
+    Routes rt;
+    rt.counts = route->counts;
+    rt.idx = route->chunk_idx;
+    rt.bias = route->bias;
+    rt.bitmask = nullptr;
+    rt.cap = route_cap(p);
+    rt.words = (s.T + 31) / 32;
+    return launch_status(launch_backward(s, p->dtype, Q, K, V, dO, qbar, kbar, rt, dQ, dK, dV, dqbar, bw,
+                                         static_cast<cudaStream_t>(stream)));
+}

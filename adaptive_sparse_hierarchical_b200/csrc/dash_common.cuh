@@ -191,4 +191,22 @@ cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* 
                           const Routes& rt, const DecodeWs& ws, cudaStream_t st);
 int decode_splits(const Shape& s, int kbar_T);
 
+// Backward pass (backward.cu): scratch of one call, all in the caller's workspace.
+struct BackwardWs {
+    float* lse;    // [b, h_q, n] log-sum-exp of each row's biased logits
+    float* del;    // [b, h_q, n] Delta = dO . O
+    float* dzbar;  // [b, h_kv, route capacity, g] gradient of the chunk logits, per routed entry
+    int* tcnt;     // [b, h_kv, T] routing positions per chunk
+    int* toff;     // [b, h_kv, T + 1] their offsets
+    int* tpos;     // [b, h_kv, route capacity] positions routing each chunk, ascending
+    int* tent;     // [b, h_kv, route capacity] the chunk's entry index in each position's list
+    float* dkbar;  // [b, h_kv, T, d]
+    float* qpart;  // [b, h_kv, T, d] dqbar partial per chunk
+};
+size_t backward_rows_smem(const Shape& s);
+size_t backward_keys_smem(const Shape& s);
+cudaError_t launch_backward(const Shape& s, int dtype, const void* Q, const void* K, const void* V, const void* dO,
+                            const float* qbar, const float* kbar, const Routes& rt, float* dQ, float* dK, float* dV,
+                            float* dqbar, const BackwardWs& ws, cudaStream_t st);
+
 }  // namespace dash

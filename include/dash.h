@@ -47,7 +47,7 @@ enum {
 };
 
 enum { DASH_F32 = 0, DASH_BF16 = 1 };
-enum { DASH_OP_PREFILL = 0, DASH_OP_DECODE = 1 };
+enum { DASH_OP_PREFILL = 0, DASH_OP_DECODE = 1, DASH_OP_BACKWARD = 2 };
 
 typedef struct {
     int batch;
@@ -184,6 +184,26 @@ int dash_decode_paged(const dash_params* p, const dash_paged_kv* pk, const void*
  *   Allocates nothing (no cudaMalloc / cudaFree / allocating library routine). */
 int dash_decode_noalloc(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
                         const float* kbar_cache, const int* seqlens, void* O, void* stream);
+
+/* Backward pass of dash_prefill: gradients of L = sum(dO * O) with respect to Q, K, V and qbar.
+ * The paper review page (section 3, the text after Eq. 9) states that the output is
+ * differentiable in q, k, v and the prior, the gradient reaching the Stage 1 entmax scores and
+ * through them the Stage 0 summaries; its Stage 2 kernel row says the training backward reuses
+ * the routed support (the entmax Jacobian is sparse).  The routed set is piecewise constant in
+ * the inputs: no gradient flows through its choice.
+ *   Inputs: Q, K, V, qbar, p and the route lists (counts, chunk_idx, bias: all three required)
+ *   and kbar_out of the dash_prefill call whose output is being differentiated; dO with O's
+ *   layout (p->o_strides, p->dtype).
+ *   Outputs (fp32, contiguous, overwritten): dQ [batch, n, h_q, d_h], dK, dV [batch, n, h_kv, d_h],
+ *   dqbar [h_kv, d_h] (summed over the batch).
+ *   Workspace: dash_workspace_size(p, DASH_OP_BACKWARD) bytes (per-row log-sum-exp, the chunk
+ *   logit gradients per routed entry, the route lists transposed per chunk), 256-byte aligned.
+ *   DASH_EUNSUPPORTED when g_q * floor(n / B) chunk logits of one position do not fit the
+ *   query-major kernel's shared memory (about 50K floats).  Deterministic: no atomics on
+ *   floating-point results. */
+int dash_backward(const dash_params* p, const void* Q, const void* K, const void* V, const float* qbar,
+                  const void* dO, const float* kbar, const dash_route_out* route, float* dQ, float* dK, float* dV,
+                  float* dqbar, void* workspace, size_t ws_bytes, void* stream);
 
 /* Static text for a status code. */
 const char* dash_status_string(int status);

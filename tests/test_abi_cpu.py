@@ -28,7 +28,7 @@ def test_header_symbols_exported():
     assert set(syms) == {"dash_workspace_size", "dash_route_capacity", "dash_prefill", "dash_prefill_stage",
                          "dash_summary_build", "dash_error_word_offset", "dash_decode_noalloc",
                          "dash_summary_append", "dash_decode", "dash_status_string", "dash_summary_build_paged",
-                         "dash_summary_append_paged", "dash_decode_paged"}
+                         "dash_summary_append_paged", "dash_decode_paged", "dash_backward"}
     lib = D.load()
     for s in syms:
         assert hasattr(lib, s), s
