@@ -37,8 +37,7 @@ namespace dash {
 namespace {
 
 constexpr int kBW = 4;        // warps per block
-constexpr int kMaxG = 16;
-constexpr int kMaxE = 4;      // d / 32 elements per lane (d <= 128)
+constexpr int kMaxE = 4;      // d / 32 elements per lane in the Stage 0 kernel (d <= 128)
 
 template <typename T>
 __device__ __forceinline__ void load_lane(const T* row, int nE, float* out)
@@ -58,7 +57,7 @@ __device__ __forceinline__ void load_lane(const T* row, int nE, float* out)
 //   tau[g], s12[kBW*g*2], misc[kBW]
 //   dqp[kBW*g*d]                per-warp dQ partials
 // ------------------------------------------------------------------------------------------
-template <typename T>
+template <typename T, int G, int D>
 __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __restrict__ Q, const T* __restrict__ K,
                                                            const T* __restrict__ V, const T* __restrict__ dO,
                                                            const float* __restrict__ kbar, Routes rt,
@@ -66,7 +65,8 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
                                                            float* __restrict__ del_out, float* __restrict__ dzbar)
 {
     extern __shared__ float smf[];
-    const int G = s.g, D = s.d, B = s.B, nE = D / 32, Tn = s.T > 0 ? s.T : 1;
+    constexpr int nE = D / 32;
+    const int B = s.B, Tn = s.T > 0 ? s.T : 1;
     float* qs = smf;
     float* gs = qs + G * D;
     float* red = gs + G * D;
@@ -113,18 +113,21 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
     };
 
     // pass 1: per head, the running max / sum and sum of p * dp (Delta = dO . o)
-    float m[kMaxG], l[kMaxG], a[kMaxG];
+    float m[G], l[G], a[G];
+#pragma unroll
     for (int h = 0; h < G; ++h) { m[h] = -INFINITY; l[h] = 0.f; a[h] = 0.f; }
     for (int u = warp; u <= cnt; u += kBW) {
         int j0, j1;
         float bias;
         unit(u, &j0, &j1, &bias);
         for (int j = j0; j < j1; ++j) {
-            float kv[kMaxE], vv[kMaxE];
+            float kv[nE], vv[nE];
             load_lane(kv_row(K, s.ks, j), nE, kv);
             load_lane(kv_row(V, s.vs, j), nE, vv);
+#pragma unroll
             for (int h = 0; h < G; ++h) {
                 float sd = 0.f, pd = 0.f;
+#pragma unroll
                 for (int k = 0; k < nE; ++k) {
                     sd += qs[h * D + lane + 32 * k] * kv[k];
                     pd += gs[h * D + lane + 32 * k] * vv[k];
@@ -163,20 +166,24 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
     __syncthreads();
 
     // pass 2: ds, the Stage 2 part of dQ, and dbias per routed entry
-    float dq[kMaxG][kMaxE];
+    float dq[G][nE];
+#pragma unroll
     for (int h = 0; h < G; ++h)
-        for (int k = 0; k < kMaxE; ++k) dq[h][k] = 0.f;
+#pragma unroll
+        for (int k = 0; k < nE; ++k) dq[h][k] = 0.f;
     for (int u = warp; u <= cnt; u += kBW) {
         int j0, j1;
         float bias;
         unit(u, &j0, &j1, &bias);
         float db = 0.f;
         for (int j = j0; j < j1; ++j) {
-            float kv[kMaxE], vv[kMaxE];
+            float kv[nE], vv[nE];
             load_lane(kv_row(K, s.ks, j), nE, kv);
             load_lane(kv_row(V, s.vs, j), nE, vv);
+#pragma unroll
             for (int h = 0; h < G; ++h) {
                 float sd = 0.f, pd = 0.f;
+#pragma unroll
                 for (int k = 0; k < nE; ++k) {
                     sd += qs[h * D + lane + 32 * k] * kv[k];
                     pd += gs[h * D + lane + 32 * k] * vv[k];
@@ -185,6 +192,7 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
                 const float p = __expf(z - lse[h]);
                 const float ds = p * (dp - del[h]);
                 db += ds;
+#pragma unroll
                 for (int k = 0; k < nE; ++k) dq[h][k] += ds * kv[k] * scale;
             }
         }
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
         const int mode = ent_mode(s.alpha);
         const float* kb0 = kbar + (long long)x * s.T * D;
         for (int c = warp; c < nvis; c += kBW) {
-            float kv[kMaxE];
+            float kv[nE];
             for (int k = 0; k < nE; ++k) kv[k] = kb0[(long long)c * D + lane + 32 * k];
             for (int h = 0; h < G; ++h) {
                 float sd = 0.f;
@@ -232,11 +240,13 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
         for (int w = 0; w < kBW; ++w) mdb += misc[w];
         mdb /= cnt;
         // per head: sum s and sum s * dwhat over the support
-        float S1[kMaxG], S2[kMaxG];
+        float S1[G], S2[G];
+#pragma unroll
         for (int h = 0; h < G; ++h) { S1[h] = 0.f; S2[h] = 0.f; }
         for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
             const int c = min(max(rt.idx[lbase + e], 0), nvis - 1);
             const float dw = wsum[e] > 0.f ? s.inv_sigma * (dbias[e] - mdb) / wsum[e] / G : 0.f;
+#pragma unroll
             for (int h = 0; h < G; ++h) {
                 const float u = xl[h * Tn + c] - tau[h];
                 if (u > 0.f) {
@@ -246,6 +256,7 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
                 }
             }
         }
+#pragma unroll
         for (int h = 0; h < G; ++h) {
             const float a1 = warp_sum(S1[h]), a2 = warp_sum(S2[h]);
             if (lane == 0) { s12[(warp * G + h) * 2] = a1; s12[(warp * G + h) * 2 + 1] = a2; }
@@ -271,15 +282,20 @@ __global__ void __launch_bounds__(32 * kBW) bwd_rows_kernel(Shape s, const T* __
         // the Stage 1 part of dQ
         for (int e = warp; e < cnt; e += kBW) {
             const int c = min(max(rt.idx[lbase + e], 0), nvis - 1);
-            float kv[kMaxE];
+            float kv[nE];
+#pragma unroll
             for (int k = 0; k < nE; ++k) kv[k] = kb0[(long long)c * D + lane + 32 * k];
+#pragma unroll
             for (int h = 0; h < G; ++h) {
                 const float v = dz[e * G + h] * scale;
+#pragma unroll
                 for (int k = 0; k < nE; ++k) dq[h][k] += v * kv[k];
             }
         }
     }
+#pragma unroll
     for (int h = 0; h < G; ++h)
+#pragma unroll
         for (int k = 0; k < nE; ++k) dqp[(warp * G + h) * D + lane + 32 * k] = dq[h][k];
     __syncthreads();
     for (int t = threadIdx.x; t < G * D; t += blockDim.x) {
@@ -369,7 +385,7 @@ __global__ void bwd_tfill_kernel(Shape s, Routes rt, const int* __restrict__ tof
 // Dynamic shared memory (floats): Ks[KT][D+1], Vs[KT][D+1], dKa[kBW][KT][D+1], dVa[kBW][KT][D+1],
 // qv[kBW][D], gv[kBW][D], dkb[kBW][D].
 // ------------------------------------------------------------------------------------------
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(32 * kBW) bwd_keys_kernel(Shape s, const T* __restrict__ Q, const T* __restrict__ K,
                                                            const T* __restrict__ V, const T* __restrict__ dO, Routes rt,
                                                            const float* __restrict__ lse_in, const float* __restrict__ del_in,
@@ -379,7 +395,8 @@ __global__ void __launch_bounds__(32 * kBW) bwd_keys_kernel(Shape s, const T* __
                                                            float* __restrict__ dkbar, int KT)
 {
     extern __shared__ float smf[];
-    const int D = s.d, G = s.g, B = s.B, P = D + 1;
+    constexpr int P = D + 1;
+    const int G = s.g, B = s.B;
     float* Ks = smf;
     float* Vs = Ks + KT * P;
     float* dKa = Vs + KT * P;
@@ -454,12 +471,14 @@ __global__ void __launch_bounds__(32 * kBW) bwd_keys_kernel(Shape s, const T* __
             const bool valid = jj < jn && (ent >= 0 || j0 + jj <= i);
             if (valid) {
                 float sd = 0.f, pd = 0.f;
+#pragma unroll 16
                 for (int e = 0; e < D; ++e) {
                     sd += q_w[e] * Ks[jj * P + e];
                     pd += g_w[e] * Vs[jj * P + e];
                 }
                 const float p = __expf(sd * scale + bias - lse);
                 const float ds = p * (pd - dl) * scale;
+#pragma unroll 16
                 for (int e = 0; e < D; ++e) {
                     dva[jj * P + e] += p * g_w[e];
                     dka[jj * P + e] += ds * q_w[e];
@@ -565,6 +584,32 @@ __global__ void bwd_qbar_reduce_kernel(Shape s, const float* __restrict__ qpart,
     dqbar[r * s.d + e] = a;
 }
 
+template <typename T, int G, int D>
+cudaError_t rows_g(const Shape& s, const T* Q, const T* K, const T* V, const T* dO, const float* kbar, const Routes& rt,
+                   float* dQ, const BackwardWs& ws, cudaStream_t st)
+{
+    const size_t smem = backward_rows_smem(s);
+    cudaError_t e = cudaFuncSetAttribute(bwd_rows_kernel<T, G, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_rows_kernel<T, G, D><<<dim3(s.n, s.batch * s.hkv), 32 * kBW, smem, st>>>(s, Q, K, V, dO, kbar, rt, dQ, ws.lse,
+                                                                                ws.del, ws.dzbar);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t rows_d(const Shape& s, const T* Q, const T* K, const T* V, const T* dO, const float* kbar, const Routes& rt,
+                   float* dQ, const BackwardWs& ws, cudaStream_t st)
+{
+    switch (s.g) {
+    case 1: return rows_g<T, 1, D>(s, Q, K, V, dO, kbar, rt, dQ, ws, st);
+    case 2: return rows_g<T, 2, D>(s, Q, K, V, dO, kbar, rt, dQ, ws, st);
+    case 4: return rows_g<T, 4, D>(s, Q, K, V, dO, kbar, rt, dQ, ws, st);
+    case 8: return rows_g<T, 8, D>(s, Q, K, V, dO, kbar, rt, dQ, ws, st);
+    case 16: return rows_g<T, 16, D>(s, Q, K, V, dO, kbar, rt, dQ, ws, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <typename T>
 cudaError_t backward_t(const Shape& s, const T* Q, const T* K, const T* V, const T* dO, const float* qbar,
                        const float* kbar, const Routes& rt, float* dQ, float* dK, float* dV, float* dqbar,
@@ -580,16 +625,15 @@ cudaError_t backward_t(const Shape& s, const T* Q, const T* K, const T* V, const
         bwd_tscan_kernel<<<pairs, 1024, 0, st>>>(s, ws.tcnt, ws.toff);
         bwd_tfill_kernel<<<dim3(s.T, pairs), 32, 0, st>>>(s, rt, ws.toff, ws.tpos, ws.tent);
     }
-    const size_t rows_smem = backward_rows_smem(s);
-    e = cudaFuncSetAttribute(bwd_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rows_smem);
+    e = s.d == 128 ? rows_d<T, 128>(s, Q, K, V, dO, kbar, rt, dQ, ws, st)
+                   : rows_d<T, 64>(s, Q, K, V, dO, kbar, rt, dQ, ws, st);
     if (e != cudaSuccess) return e;
-    bwd_rows_kernel<T><<<dim3(s.n, pairs), 32 * kBW, rows_smem, st>>>(s, Q, K, V, dO, kbar, rt, dQ, ws.lse, ws.del,
-                                                                       ws.dzbar);
     const int KT = s.B >= 32 ? 32 : s.B;
     const size_t keys_smem = backward_keys_smem(s);
-    e = cudaFuncSetAttribute(bwd_keys_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)keys_smem);
+    auto keys = s.d == 128 ? bwd_keys_kernel<T, 128> : bwd_keys_kernel<T, 64>;
+    e = cudaFuncSetAttribute(keys, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)keys_smem);
     if (e != cudaSuccess) return e;
-    bwd_keys_kernel<T><<<dim3((s.n + KT - 1) / KT, pairs), 32 * kBW, keys_smem, st>>>(
+    keys<<<dim3((s.n + KT - 1) / KT, pairs), 32 * kBW, keys_smem, st>>>(
         s, Q, K, V, dO, rt, ws.lse, ws.del, ws.dzbar, ws.toff, ws.tpos, ws.tent, dK, dV, ws.dkbar, KT);
     if (s.T > 0)
         bwd_stage0_kernel<T><<<dim3(s.T, pairs), 32 * kBW, 0, st>>>(s, K, qbar, kbar, ws.dkbar, dK, ws.qpart);

@@ -4,7 +4,8 @@
 Default (N=1): the 1B-class prefill layer (b=1, n=32768, 16 query / 2 KV heads, d=128, chunk 64,
 alpha 1.5, gamma tuned for 25% routed chunks), one step = Stage 0 + Stage 1 + Stage 2 over the
 whole sequence, plus the decode workload (b=8, 131072-token caches, 32/2 heads, one append +
-decode per step) reported under "decode".  Under torchrun every rank runs its own replica
+decode per step) reported under "decode", and the backward pass of the prefill workload (dQ, dK,
+dV, dqbar) reported under "backward".  Under torchrun every rank runs its own replica
 (no data-path collective): scaling is weak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dash|reference]
@@ -52,6 +53,9 @@ def args_():
     ap.add_argument("--workload", default="prefill_32k")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--only-backward", action="store_true",
+                    help="time the backward pass of the workload alone and print its object")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=16384)
     ap.add_argument("--sweep", action="store_true",
@@ -291,6 +295,57 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
     out["dense_causal"] = dense_denominators(wl, tq, qbar, pf, steps, flush, ms, dev)
     out["_inputs"] = x
     return out
+
+
+def run_backward(wl, steps, warmup, ranks, pk, pk_kind, x=None):
+    """The backward pass (dash_backward) of the prefill workload: gradients of Q, K, V and qbar
+    for a seeded dO, device-timed with CUDA events, L2 flushed between steps.  Algorithmic FLOPs:
+    the five Stage 2 products of a softmax-attention backward (S, dP, dV, dQ, dK: 10 d per routed
+    or diagonal (row, key) pair, 2.5x the forward's 4 d); the Stage 1 / Stage 0 chain is not
+    counted."""
+    import torch
+    import adaptive_sparse_hierarchical_b200 as D
+
+    dev = torch.device("cuda", ranks.local)
+    x = wl.make() if x is None else x
+    tq = {k: torch.from_numpy(x[k]).to(dev, torch.bfloat16) for k in ("Q", "K", "V")}
+    qbar = torch.from_numpy(x["qbar"]).to(dev)
+    pf = D.Prefill(tq["Q"], tq["K"], tq["V"], qbar, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
+                   inv_sigma=wl.inv_sigma, want_route=True)
+    pf()
+    g = torch.Generator(device=dev).manual_seed(1234)
+    dO = torch.randn(tq["Q"].shape, device=dev, generator=g).to(torch.bfloat16)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(warmup, 3)):
+        pf.backward(dO)
+    torch.cuda.synchronize(dev)
+    counts = pf.counts.cpu().numpy()
+    flops = 2.5 * stage2_routed_flops(counts, wl.n, wl.chunk, wl.h_q // wl.h_kv, wl.d, wl.h_q)
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    with Clocks(ranks.local) as clk:
+        for k in range(steps):
+            flush.fill_(k & 0xff)
+            recs[k][0].record(stream)
+            pf.backward(dO)
+            recs[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+    ranks.barrier()
+    ms = ranks.max(statistics.mean(r[0].elapsed_time(r[1]) for r in recs))
+    achieved = flops / (ms / 1e3) / 1e12
+    T = wl.n // wl.chunk
+    launches = 2 + (5 if T > 0 else 0)
+    del pf
+    torch.cuda.empty_cache()
+    return {"workload": f"{wl.name} backward: dQ, dK, dV, dqbar of sum(dO * O), dO ~ N(0, 1) bf16",
+            "ms_per_step": ms, "tokens_per_s_M": ranks.world * wl.batch * wl.n / (ms / 1e3) / 1e6,
+            "roofline": {"kernel": "bwd_rows_kernel + bwd_keys_kernel (fp32 CUDA cores)", "bound": "tensor",
+                         "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                         "peak_kind": f"bf16 dense burst, of {pk_kind}", "flops_per_step": flops},
+            "clocks": clk.summary(), "steps": steps, "gpu_launches": launches * steps}
 
 
 def dense_denominators(wl, tq, qbar, pf, steps, flush, sparse_ms, dev):
@@ -552,6 +607,12 @@ def main():
         ranks.close()
         return
     wl = W.get(args.workload)
+    if args.only_backward:
+        bw = run_backward(wl, args.steps, args.warmup, ranks, pk, pk_kind)
+        if ranks.rank == 0:
+            print(json.dumps({"backward": bw}), flush=True)
+        ranks.close()
+        return
     pre = run_prefill(wl, args.steps, args.warmup, ranks, pk, pk_kind)
     x = pre.pop("_inputs")
     line = {"metric": METRIC, "value": pre["value"], "unit": "Mtok/s", "n_gpus": ranks.world, "steps": args.steps,
@@ -563,6 +624,9 @@ def main():
     if not args.no_decode:
         line["decode"] = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind)
         line["gpu_launches"] += line["decode"]["gpu_launches"]
+    if not args.no_backward:
+        line["backward"] = run_backward(wl, max(2, min(args.steps, 5)), args.warmup, ranks, pk, pk_kind, x=x)
+        line["gpu_launches"] += line["backward"]["gpu_launches"]
     if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
         v, secs, thr = oracle_sample(wl, x, args.cpu_rows)
         line["cpu_baseline"] = {"value": v / 1e6, "unit": "Mtok/s", "cores": thr, "kind": "oracle",
