@@ -116,3 +116,32 @@ def test_paged_description_rejected_before_launch(kw, pkw, code):
     # a null page description is an error, not the contiguous layout
     assert lib.dash_decode_paged(ctypes.byref(_p()), None, 256, 256, 256, 256, 256, 256, None, 256, 1 << 40,
                                  None) == L.DASH_EINVAL
+
+
+def test_backward_arguments_rejected_before_launch():
+    """dash_backward checks its arguments before touching the device: the route lists are
+    required, the workspace must cover dash_workspace_size(p, DASH_OP_BACKWARD), and a group whose
+    chunk logits do not fit the query-major kernel's shared memory is unsupported."""
+    lib = D.load()
+    p = _p()
+    ws = L.dash_workspace_size(p, L.DASH_OP_BACKWARD)
+    T, cap, g = 1024 // 64, L.dash_route_capacity(p), 4
+    assert ws >= 2 * 8 * 1024 * 4 + 2 * cap * g * 4 + 2 * 2 * cap * 4 + 2 * 2 * T * 128 * 4
+    full = L.dash_route_out(256, 256, 256, None)
+    no_bias = L.dash_route_out(256, 256, None, None)
+
+    def call(pp, route, workspace=256, nbytes=ws):
+        return lib.dash_backward(ctypes.byref(pp), 256, 256, 256, 256, 256, 256,
+                                 ctypes.byref(route) if route is not None else None, 256, 256, 256, 256,
+                                 workspace, nbytes, None)
+
+    assert call(p, None) == L.DASH_EINVAL
+    assert call(p, no_bias) == L.DASH_EINVAL
+    assert call(p, full, workspace=None) == L.DASH_EWORKSPACE
+    assert call(p, full, nbytes=ws - 1) == L.DASH_EWORKSPACE
+    assert call(p, full, workspace=384) == L.DASH_EALIGN
+    assert call(_p(alpha=1.0), full) == L.DASH_EINVAL
+    # 16 heads per group x 4096 chunks of logits (plus the per-entry buffers) exceed shared memory
+    big = _p(seqlen=131072, h_q=32, h_kv=2, chunk=32, q_strides=(0, 32 * 128, 128), k_strides=(0, 256, 128),
+             v_strides=(0, 256, 128), o_strides=(0, 32 * 128, 128))
+    assert call(big, full, nbytes=1 << 50) == L.DASH_EUNSUPPORTED
