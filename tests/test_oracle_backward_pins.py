@@ -153,3 +153,46 @@ def test_no_prior_reduces_to_masked_softmax_autograd(alpha, gamma, inv_sigma):
     assert np.all(dqbar == 0.0)
     for a, ref in ((dQ, rQ), (dK, rK), (dV, rV)):
         np.testing.assert_allclose(a, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_chunk_one_degenerate_case():
+    """B = 1: every token is its own chunk, k̄_c = k_c (Stage 0 of one key), so qbar has no effect
+    (dqbar = 0 exactly) and the routing runs over the previous tokens themselves.  Finite
+    differences of the forward oracle pin dQ, dK and dV there."""
+    alpha, gamma, inv_sigma, b, n, hq, hkv, d, B = 1.5, 3.0, 1.0, 1, 24, 2, 1, 8, 1
+    kw = dict(chunk=B, alpha=alpha, gamma=gamma, inv_sigma=inv_sigma)
+    t = _case(9, b, n, hq, hkv, d, B)
+    dQ, dK, dV, dqbar = oracle.backward(t["Q"], t["K"], t["V"], t["qbar"], t["dO"], nthreads=1, **kw)
+    assert np.all(dqbar == 0.0)
+    rng = np.random.default_rng(13)
+    for name, g in (("Q", dQ), ("K", dK), ("V", dV)):
+        gmax = np.abs(g).max()
+        checked = 0
+        for _ in range(10):
+            idx = tuple(int(rng.integers(s)) for s in t[name].shape)
+            f1, same1 = _fd(t, name, idx, H, kw)
+            f2, same2 = _fd(t, name, idx, H / 2, kw)
+            if not (same1 and same2) or abs(f1 - f2) > 1e-6 + 1e-5 * gmax:
+                continue
+            checked += 1
+            assert abs(g[idx] - f2) <= 2e-6 + 2e-5 * gmax, (name, idx, g[idx], f2, gmax)
+        assert checked >= 7, (name, checked)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_dv_identity_on_random_shapes(seed):
+    """sum_j dV_j = sum of the group's dO rows on random shapes, chunk sizes, alpha and sigma."""
+    rng = np.random.default_rng(200 + seed)
+    hkv = int(rng.choice([1, 2]))
+    g = int(rng.choice([1, 2, 4]))
+    B = int(rng.choice([1, 4, 16, 32]))
+    n = int(rng.integers(B + 1, 5 * B + 40))
+    d = int(rng.choice([8, 16]))
+    alpha = float(rng.choice([1.25, 1.5, 2.0]))
+    inv_sigma = float(rng.choice([0.0, 0.5, 1.0]))
+    t = _case(300 + seed, 1, n, hkv * g, hkv, d, B)
+    _, _, dV, dqbar = oracle.backward(t["Q"], t["K"], t["V"], t["qbar"], t["dO"], chunk=B, alpha=alpha, gamma=4.0,
+                                      inv_sigma=inv_sigma)
+    want = t["dO"].astype(np.float64).reshape(1, n, hkv, g, d).sum(axis=(1, 3))
+    np.testing.assert_allclose(dV.sum(axis=1), want, rtol=1e-12, atol=1e-10)
+    assert np.all(np.isfinite(dqbar)) and (inv_sigma > 0 or np.all(dqbar == 0.0))
