@@ -297,7 +297,7 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
     return out
 
 
-def run_backward(wl, steps, warmup, ranks, pk, pk_kind, x=None):
+def run_backward(wl, steps, warmup, ranks, pk, pk_kind, x=None, cpu=False):
     """The backward pass (dash_backward) of the prefill workload: gradients of Q, K, V and qbar
     for a seeded dO, device-timed with CUDA events, L2 flushed between steps.  Algorithmic FLOPs:
     the five Stage 2 products of a softmax-attention backward (S, dP, dV, dQ, dK: 10 d per routed
@@ -339,13 +339,36 @@ def run_backward(wl, steps, warmup, ranks, pk, pk_kind, x=None):
     launches = 2 + (5 if T > 0 else 0)
     del pf
     torch.cuda.empty_cache()
+    base = oracle_backward_sample(wl, x, counts) if cpu else None
     return {"workload": f"{wl.name} backward: dQ, dK, dV, dqbar of sum(dO * O), dO ~ N(0, 1) bf16",
+            "cpu_baseline": base,
             "ms_per_step": ms, "tokens_per_s_M": ranks.world * wl.batch * wl.n / (ms / 1e3) / 1e6,
             "roofline": {"kernel": "bwd_rows_kernel + bwd_keys_kernel (fp32 CUDA cores)", "bound": "tensor",
                          "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_tflops"], "traffic": None,
                          "peak_kind": f"bf16 dense burst, of {pk_kind}", "flops_per_step": flops},
             "clocks": clk.summary(), "steps": steps, "gpu_launches": launches * steps}
+
+
+def oracle_backward_sample(wl, x, counts, ntok=2048):
+    """Time the float64 oracle's backward on a bounded sample of the workload: the first `ntok`
+    positions of every sequence (all heads; routing is causal, so these rows route exactly as in
+    the full sequence).  Rows near the start see fewer chunks than the average row, so the
+    per-token rate overstates the oracle's full-sequence rate; the algorithmic rate on the same
+    prefix (2.5x the forward's Stage 2 FLOPs of those rows) is comparable with the GPU's."""
+    import oracle
+    from adaptive_sparse_hierarchical_b200 import inputs
+
+    dO = inputs.round_bf16(np.random.default_rng(5).standard_normal((wl.batch, ntok, wl.h_q, wl.d)))
+    t0 = time.perf_counter()
+    oracle.backward(x["Q"][:, :ntok], x["K"][:, :ntok], x["V"][:, :ntok], x["qbar"], dO, chunk=wl.chunk,
+                    alpha=wl.alpha, gamma=wl.gamma, inv_sigma=wl.inv_sigma)
+    secs = time.perf_counter() - t0
+    flops = 2.5 * stage2_routed_flops(counts[..., :ntok], ntok, wl.chunk, wl.h_q // wl.h_kv, wl.d, wl.h_q)
+    return {"value": wl.batch * ntok / secs / 1e6, "unit": "Mtok/s", "tflops": flops / secs / 1e12,
+            "cores": min(oracle.num_threads(), wl.batch * wl.h_kv), "kind": "oracle",
+            "sample": f"oracle.backward on the first {ntok} positions of each sequence, all heads ({secs:.1f} s); "
+                      f"the oracle parallelises over (sequence, KV head) pairs"}
 
 
 def dense_denominators(wl, tq, qbar, pf, steps, flush, sparse_ms, dev):
@@ -663,7 +686,8 @@ def main():
         return
     wl = W.get(args.workload)
     if args.only_backward:
-        bw = run_backward(wl, args.steps, args.warmup, ranks, pk, pk_kind)
+        bw = run_backward(wl, args.steps, args.warmup, ranks, pk, pk_kind,
+                          cpu=ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline)
         if ranks.rank == 0:
             print(json.dumps({"backward": bw}), flush=True)
         ranks.close()
@@ -681,7 +705,8 @@ def main():
         line["gpu_launches"] += line["decode"]["gpu_launches"]
     if not args.no_backward:
         try:
-            line["backward"] = run_backward(wl, max(2, min(args.steps, 5)), args.warmup, ranks, pk, pk_kind, x=x)
+            line["backward"] = run_backward(wl, max(2, min(args.steps, 5)), args.warmup, ranks, pk, pk_kind, x=x,
+                                            cpu=ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline)
             line["gpu_launches"] += line["backward"]["gpu_launches"]
         except Exception as e:   # reported in the line; the forward numbers above stand
             line["backward"] = {"error": f"{type(e).__name__}: {e}"[:300]}
