@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "dash.h")
 DASH_OK, DASH_EINVAL, DASH_EUNSUPPORTED, DASH_EWORKSPACE, DASH_EALIGN, DASH_ELAUNCH = 0, -1, -2, -3, -4, -5
 DASH_F32, DASH_BF16 = 0, 1
 DASH_OP_PREFILL, DASH_OP_DECODE, DASH_OP_BACKWARD = 0, 1, 2
-DASH_STAGE0, DASH_STAGE1, DASH_STAGE2 = 0, 1, 2
+DASH_STAGE0, DASH_STAGE1, DASH_STAGE2, DASH_STAGE2_BITMASK = 0, 1, 2, 3
 
 
 class dash_params(ctypes.Structure):

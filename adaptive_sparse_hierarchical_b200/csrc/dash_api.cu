@@ -9,12 +9,11 @@ using namespace dash;
 
 namespace {
 
-constexpr size_t kAlign = 256;
-inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-
 bool pow2_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
-int esize(int dtype) { return dtype == DASH_BF16 ? 2 : 4; }
+}  // namespace
+
+namespace dash {
 
 // Shape checks shared by every entry point.
 int check_params(const dash_params* p)
@@ -27,10 +26,20 @@ int check_params(const dash_params* p)
     if (p->dtype != DASH_F32 && p->dtype != DASH_BF16) return DASH_EINVAL;
     if (p->chunk < 1 || p->d_h < 1) return DASH_EINVAL;
     if (p->d_h != 64 && p->d_h != 128) return DASH_EUNSUPPORTED;
-    if (p->chunk != 16 && p->chunk != 32 && p->chunk != 64 && p->chunk != 128) return DASH_EUNSUPPORTED;
+    if (p->chunk != 1 && p->chunk != 16 && p->chunk != 32 && p->chunk != 64 && p->chunk != 128)
+        return DASH_EUNSUPPORTED;
     if (!pow2_group(p->h_q / p->h_kv)) return DASH_EUNSUPPORTED;
     return DASH_OK;
 }
+
+}  // namespace dash
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int esize(int dtype) { return dtype == DASH_BF16 ? 2 : 4; }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
@@ -194,7 +203,7 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
                        const float* qbar, void* O, float* kbar_out, const dash_route_out* route, void* workspace,
                        size_t ws_bytes, void* stream)
 {
-    if (stage < -1 || stage > DASH_STAGE2) return DASH_EINVAL;
+    if (stage < -1 || stage > DASH_STAGE2_BITMASK) return DASH_EINVAL;
     int rc = check_params(p);
     if (rc != DASH_OK) return rc;
     if (!Q || !K || !V || !qbar || !O) return DASH_EINVAL;
@@ -239,6 +248,11 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     if (stage == -1 || stage == DASH_STAGE2)
         rc = launch_status(launch_attend_prefill(s, p->dtype, Q, K, V, O, rt,
                                                  reinterpret_cast<int*>(ws + L.perm), err, st));
+    if (stage == DASH_STAGE2_BITMASK) {
+        if (!rt.bitmask) return DASH_EINVAL;
+        if (!attend_pair_supported(s, p->dtype)) return DASH_EUNSUPPORTED;
+        rc = launch_status(launch_attend_prefill_mask(s, Q, K, V, O, rt, reinterpret_cast<int*>(ws + L.perm), err, st));
+    }
     return rc;
 }
 

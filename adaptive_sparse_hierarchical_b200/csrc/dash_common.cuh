@@ -2,6 +2,7 @@
 // B200 DashAttention library.  Internal only: the public interface is include/dash.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -107,18 +108,29 @@ template <> struct Vec<float> {
         float4 v = *reinterpret_cast<const float4*>(p);
         out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
     }
+    // the raw 16 bytes, and their conversion (split so that several loads can be in flight)
+    __device__ __forceinline__ static uint4 raw(const float* p) { return *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ static void cvt(uint4 v, float* out)
+    {
+        out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+        out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+    }
 };
 template <> struct Vec<__nv_bfloat16> {
     static constexpr int N = 8;
-    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out)
+    __device__ __forceinline__ static void cvt(uint4 v, float* out)
     {
-        uint4 v = *reinterpret_cast<const uint4*>(p);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             out[2 * k] = __uint_as_float(w[k] << 16);
             out[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
         }
+    }
+    __device__ __forceinline__ static uint4 raw(const __nv_bfloat16* p) { return *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out)
+    {
+        cvt(*reinterpret_cast<const uint4*>(p), out);
     }
 };
 
@@ -127,6 +139,9 @@ __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Shape and hyper-parameter checks shared by every entry point (DASH_OK or a DASH_E* status).
+int check_params(const dash_params* p);
 
 // ---- launchers (each returns cudaGetLastError() of its launches) -------------------------
 // Stage 0: summaries of complete chunks of positions [0, len_b) and, if state != null, the
@@ -166,6 +181,23 @@ bool attend_tc_supported(const Shape& s, int dtype);
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
                                      const Routes& rt, int* perm, int* err, cudaStream_t st);
 bool legacy_stage2();
+bool single_tile_stage2();
+// Helpers of the tensor-core Stage 2 kernels (stage2_tc.cu): a 4-D TMA map over a
+// [batch, n, heads, 128] bf16 tensor with box (64 d, bh heads, bp positions, 1) and 128-byte
+// swizzle; whether positions are grouped by route similarity before tiling; the grouping launch.
+bool s2_make_map(CUtensorMap* map, const void* ptr, int batch, int n, int heads, const long long st[3], int bh, int bp);
+bool s2_encode_available();
+bool s2_grouping_enabled(const Shape& s);
+cudaError_t launch_group_positions(const Shape& s, const Routes& rt, int P, int* perm, cudaStream_t st);
+// Paired-tile Stage 2 (stage2_pair.cu): one block per two 128-row tiles sharing one key walk of
+// 128-key jobs (bf16, d = 128, chunk 32 / 64 / 128, 128 % g == 0).
+bool attend_pair_supported(const Shape& s, int dtype);
+cudaError_t launch_attend_prefill_pair(const Shape& s, const void* Q, const void* K, const void* V, void* O,
+                                       const Routes& rt, int* perm, int* err, cudaStream_t st);
+// The same kernel driven by the bit-packed block mask rt.bitmask (plus the bias lists) instead of
+// the chunk lists.
+cudaError_t launch_attend_prefill_mask(const Shape& s, const void* Q, const void* K, const void* V, void* O,
+                                       const Routes& rt, int* perm, int* err, cudaStream_t st);
 // Decode: Stage 1 (logits, thresholds, GQA aggregation) and Stage 2 (split + merge).
 struct DecodeWs {
     float* x;        // [b, hkv, g, T]  scaled logits, then head weights

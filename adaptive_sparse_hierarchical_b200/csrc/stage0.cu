@@ -5,9 +5,9 @@
 // The keys double as values, so one pass over each key serves both the logit and the weighted
 // sum (online softmax); a finished chunk's summary is written once and never recomputed.
 //
-// One warp per (sequence, KV head, chunk).  A key of d elements is read as 16-byte vectors by
-// d*sizeof(T)/16 lanes, so a warp covers 32*16/(d*sizeof(T)) keys per load instruction; each
-// lane group keeps its own online-softmax state and the groups merge at the end.
+// A key of d elements is read as 16-byte vectors by d*sizeof(T)/16 lanes, so a warp covers
+// 32*16/(d*sizeof(T)) keys per load instruction; each lane group keeps its own online-softmax state
+// and the groups merge at the end.
 #include "dash_common.cuh"
 
 namespace dash {
@@ -44,6 +44,9 @@ struct Run {
     }
 };
 
+// One block (4 warps) per (sequence, KV head, chunk): warp w takes the w-th quarter of the chunk's
+// keys with all of its loads in flight at once (8 per lane), keeps an online-softmax state per
+// lane group, and the four warps' states merge through shared memory.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restrict__ K,
                                                      const float* __restrict__ qbar,
@@ -51,8 +54,9 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
                                                      int kbar_T, float* state, __nv_bfloat16* planes)
 {
     using L = KeyLanes<T, D>;
-    const int lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+    __shared__ float wst[4][D + 2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long item = blockIdx.x;
     const int per = kbar_T + 1;
     if (item >= (long long)s.batch * s.hkv * per) return;
     const int c = (int)(item % per);
@@ -61,7 +65,7 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
     const int n = len ? len[b] : s.n;
     const int cfull = min(n / s.B, kbar_T);
     const bool complete = c < cfull;
-    if (!complete && !(state && c == n / s.B)) return;
+    if (!complete && !(state && c == n / s.B)) return;   // block-uniform
     const int t0 = c * s.B, t1c = complete ? t0 + s.B : n;
 
     const int grp = lane / L::LPK, sub = lane % L::LPK;
@@ -77,25 +81,30 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
     const long long koff = t1c > t0 ? kv_off(s, s.ks, s.kps, b, t0, r) : 0;
     const T* kb = K + (koff < 0 ? 0 : koff) + sub * L::EPL;
     const int t1 = koff < 0 ? t0 : t1c;
-    constexpr int U = 4;
+    // this warp's quarter of [t0, t1)
+    const int len_all = t1 - t0, q = (len_all + 3) / 4;
+    const int w0 = t0 + min(len_all, warp * q), w1 = t0 + min(len_all, (warp + 1) * q);
+    constexpr int U = 8;
     // the loop bounds are warp-uniform so that every lane reaches the shuffles
-    for (int base = t0; base < t1; base += U * L::KPI) {
-        float kv[U][L::EPL];
+    for (int base = w0; base < w1; base += U * L::KPI) {
+        // all U loads first (rows past the quarter re-read its last row and are not pushed)
+        uint4 raw[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            int tt = base + u * L::KPI + grp;
-            if (tt < t1) Vec<T>::load(kb + (long long)(tt - t0) * s.ks[1], kv[u]);
-            else for (int e = 0; e < L::EPL; ++e) kv[u][e] = 0.f;
+            const int tt = min(base + u * L::KPI + grp, w1 - 1);
+            raw[u] = Vec<T>::raw(kb + (long long)(tt - t0) * s.ks[1]);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             int tt = base + u * L::KPI + grp;
+            float kv[L::EPL];
+            Vec<T>::cvt(raw[u], kv);
             float dot = 0.f;
 #pragma unroll
-            for (int e = 0; e < L::EPL; ++e) dot += qv[e] * kv[u][e];
+            for (int e = 0; e < L::EPL; ++e) dot += qv[e] * kv[e];
 #pragma unroll
             for (int o = L::LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            if (tt < t1) run.push(dot, kv[u]);
+            if (tt < w1) run.push(dot, kv);
         }
     }
     // merge the lane groups (lanes sub, sub+LPK, sub+2LPK, ... hold the same elements)
@@ -107,7 +116,18 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
         for (int e = 0; e < L::EPL; ++e) a2[e] = __shfl_xor_sync(0xffffffffu, run.acc[e], o);
         run.merge(m2, l2, a2);
     }
-    if (grp != 0) return;
+    // merge the four warps' states in warp order
+    if (grp == 0) {
+        for (int e = 0; e < L::EPL; ++e) wst[warp][sub * L::EPL + e] = run.acc[e];
+        if (sub == 0) { wst[warp][D] = run.m; wst[warp][D + 1] = run.l; }
+    }
+    __syncthreads();
+    if (warp != 0 || grp != 0) return;
+    for (int w = 1; w < 4; ++w) {
+        float a2[L::EPL];
+        for (int e = 0; e < L::EPL; ++e) a2[e] = wst[w][sub * L::EPL + e];
+        run.merge(wst[w][D], wst[w][D + 1], a2);
+    }
     if (complete) {
         float* out = kbar + (((long long)b * s.hkv + r) * kbar_T + c) * D + sub * L::EPL;
         const float inv = 1.f / run.l;
@@ -186,7 +206,7 @@ cudaError_t stage0_t(const Shape& s, const void* K, const float* qbar, const int
                      int kbar_T, float* state, __nv_bfloat16* planes, cudaStream_t st)
 {
     const long long items = (long long)s.batch * s.hkv * (kbar_T + 1);
-    const unsigned grid = (unsigned)((items + 3) / 4);
+    const unsigned grid = (unsigned)items;
     if (grid == 0) return cudaSuccess;
     if (s.d == 128)
         stage0_kernel<T, 128><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes);

@@ -376,7 +376,43 @@ __global__ void __launch_bounds__(128) attend_rows_kernel(Shape s, const T* __re
             m = mn;
         }
     };
-    for (int k = 0; k < cnt; ++k) range(li[k] * s.B, li[k] * s.B + s.B, lb[k] * kLog2e);
+    // chunks shorter than a warp (B = 1: each chunk is one token, B = 16): 32 / B listed chunks
+    // per step, lane -> (entry k0 + lane / B, key lane % B), each lane with its chunk's bias
+    auto gather = [&](int k0) {
+        const int e = k0 + lane / s.B;
+        const bool ok = e < cnt;
+        const int j = ok ? li[e] * s.B + lane % s.B : 0;
+        float sv = -INFINITY;
+        if (ok) {
+            const T* kr = Kb + (long long)j * s.ks[1];
+            float dot = 0.f;
+            for (int x = 0; x < D; x += Vec<T>::N) {
+                float kv[Vec<T>::N];
+                Vec<T>::load(kr + x, kv);
+                for (int u = 0; u < Vec<T>::N; ++u) dot += qsh[warp][x + u] * kv[u];
+            }
+            sv = dot + lb[e] * kLog2e;
+        }
+        const float mn = fmaxf(m, warp_max(sv));   // lane 0 always holds a listed key
+        const float corr = exp2f(m - mn);
+        const float p = ok ? exp2f(sv - mn) : 0.f;
+        l = l * corr + warp_sum(p);
+#pragma unroll
+        for (int x = 0; x < D / 32; ++x) acc[x] *= corr;
+        const int nl = min(32, (cnt - k0) * s.B);
+        for (int jj = 0; jj < nl; ++jj) {
+            const float pj = __shfl_sync(0xffffffffu, p, jj);
+            const int tj = __shfl_sync(0xffffffffu, j, jj);
+            const T* vr = Vb + (long long)tj * s.vs[1];
+#pragma unroll
+            for (int x = 0; x < D / 32; ++x) acc[x] += pj * to_f(vr[lane + 32 * x]);
+        }
+        m = mn;
+    };
+    if (s.B < 32)
+        for (int k = 0; k < cnt; k += 32 / s.B) gather(k);
+    else
+        for (int k = 0; k < cnt; ++k) range(li[k] * s.B, li[k] * s.B + s.B, lb[k] * kLog2e);
     range((i / s.B) * s.B, i + 1, 0.f);
     const float inv = 1.f / l;
 #pragma unroll
@@ -455,12 +491,31 @@ cudaError_t rows_t(const Shape& s, const void* Q, const void* K, const void* V, 
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K, const void* V,
                                   void* O, const Routes& rt, int* perm, int* err, cudaStream_t st)
 {
+    if (attend_pair_supported(s, dtype) && !legacy_stage2() && !single_tile_stage2())
+        return launch_attend_prefill_pair(s, Q, K, V, O, rt, perm, err, st);
     if (attend_tc_supported(s, dtype) && !legacy_stage2())
         return launch_attend_prefill_tc(s, Q, K, V, O, rt, perm, err, st);
+    if (s.B == 1)   // one token per chunk (Stage 1 is entmax over tokens): the row kernel
+        return dtype == DASH_BF16
+                   ? (s.d == 128 ? rows_t<__nv_bfloat16, 128>(s, Q, K, V, O, rt, nullptr, st)
+                                 : rows_t<__nv_bfloat16, 64>(s, Q, K, V, O, rt, nullptr, st))
+                   : (s.d == 128 ? rows_t<float, 128>(s, Q, K, V, O, rt, nullptr, st)
+                                 : rows_t<float, 64>(s, Q, K, V, O, rt, nullptr, st));
     if (dtype == DASH_BF16)
         return s.d == 128 ? prefill_bf16_d<128>(s, Q, K, V, O, rt, st) : prefill_bf16_d<64>(s, Q, K, V, O, rt, st);
     return s.d == 128 ? rows_t<float, 128>(s, Q, K, V, O, rt, nullptr, st)
                       : rows_t<float, 64>(s, Q, K, V, O, rt, nullptr, st);
+}
+
+bool single_tile_stage2()
+{
+    // DASH_STAGE2=tile selects the one-tile tcgen05 kernel (64-key jobs, two blocks per SM)
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("DASH_STAGE2");
+        v = (e && e[0] == 't') ? 1 : 0;
+    }
+    return v == 1;
 }
 
 bool legacy_stage2()
@@ -492,6 +547,12 @@ cudaError_t launch_decode(const Shape& s, int dtype, const void* q, const void* 
         return cudaGetLastError();
     }
     if (s.pt) return cudaErrorInvalidValue;
+    if (s.B == 1)
+        return dtype == DASH_BF16
+                   ? (s.d == 128 ? rows_t<__nv_bfloat16, 128>(s, q, Kc, Vc, O, rt, seqlens, st)
+                                 : rows_t<__nv_bfloat16, 64>(s, q, Kc, Vc, O, rt, seqlens, st))
+                   : (s.d == 128 ? rows_t<float, 128>(s, q, Kc, Vc, O, rt, seqlens, st)
+                                 : rows_t<float, 64>(s, q, Kc, Vc, O, rt, seqlens, st));
     if (dtype == DASH_BF16)
         return s.d == 128 ? dec_bf16_d<128>(s, q, Kc, Vc, seqlens, rt, ws, O, st)
                           : dec_bf16_d<64>(s, q, Kc, Vc, seqlens, rt, ws, O, st);

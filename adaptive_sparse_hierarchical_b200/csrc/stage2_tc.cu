@@ -635,6 +635,23 @@ bool make_map(CUtensorMap* map, const void* ptr, int batch, int n, int heads, co
 
 }  // namespace
 
+bool s2_make_map(CUtensorMap* map, const void* ptr, int batch, int n, int heads, const long long st[3], int bh, int bp)
+{
+    return make_map(map, ptr, batch, n, heads, st, bh, bp);
+}
+
+bool s2_encode_available() { return encode_fn() != nullptr; }
+
+bool s2_grouping_enabled(const Shape& s) { return (s.g == 8 || s.g == 16) && !cluster_disabled(); }
+
+cudaError_t launch_group_positions(const Shape& s, const Routes& rt, int P, int* perm, cudaStream_t st)
+{
+    if (s.n <= 0) return cudaSuccess;
+    const int Wn = kWinTiles * P;
+    group_positions_kernel<<<dim3((s.n + Wn - 1) / Wn, s.batch * s.hkv), 1024, 0, st>>>(s, rt, P, perm);
+    return cudaGetLastError();
+}
+
 // union units (chunks, or 64-key tiles of two 32-key chunks) a block's job list may hold
 int attend_units(const Shape& s) { return (s.B >= kKT ? s.T : s.T / 2) + 2; }
 

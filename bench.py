@@ -30,10 +30,19 @@ METRIC = "prefill Mtok/s and decode µs/token at 32K–128K ctx; % of HBM / bf16
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM bytes per launch of the Stage 2 tcgen05 kernel (dram__bytes_read.sum + dram__bytes_write.sum
-# from one ncu capture of the current kernel on that workload); reset to absent when the kernel
-# changes and the capture has not been repeated.
-STAGE2_TRAFFIC = {"prefill_32k": 314.7e6}
+# DRAM bytes per launch of a Stage 2 kernel (dram__bytes_read.sum + dram__bytes_write.sum from one
+# ncu capture of the current kernel on that workload), keyed by (kernel, workload); absent until
+# the current kernel has been captured.
+STAGE2_TRAFFIC = {}
+
+
+def stage2_kernel_name():
+    sel = os.environ.get("DASH_STAGE2", "")
+    if sel.startswith("m"):
+        return "attend_prefill_mma_kernel (mma.sync)"
+    if sel.startswith("t"):
+        return "attend_prefill_tc_kernel (tcgen05, one tile per block)"
+    return "attend_pair_kernel (tcgen05, two tiles per block)"
 
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -60,6 +69,10 @@ def args_():
     ap.add_argument("--cpu-rows", type=int, default=16384)
     ap.add_argument("--sweep", action="store_true",
                     help="time the 64K sparsity sweep and the 128K alpha x chunk-size sweep (one line each)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave the sweeps out of the default line (they run at N=1 only)")
+    ap.add_argument("--sweep-steps", type=int, default=3)
+    ap.add_argument("--sweep-decode-steps", type=int, default=64)
     return ap.parse_args()
 
 
@@ -223,11 +236,9 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
         "ms_per_step": ms, "value": ranks.world * tokens / (ms / 1e3) / 1e6,
         "stages_ms": {"stage0_summary": stage_ms[0], "stage1_route": stage_ms[1], "stage2_attend": stage_ms[2]},
         "routed_fraction": float(counts.sum()) / (wl.batch * wl.h_kv * sum(i // wl.chunk for i in range(wl.n))),
-        "roofline": {"kernel": ("attend_prefill_mma_kernel (mma.sync)" if os.environ.get("DASH_STAGE2", "").startswith("m")
-                               else "attend_prefill_tc_kernel (tcgen05)"), "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": stage2_kernel_name(), "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": (STAGE2_TRAFFIC.get(wl.name) if not os.environ.get("DASH_STAGE2", "").startswith("m")
-                                 else None),
+                     "traffic": STAGE2_TRAFFIC.get((stage2_kernel_name(), wl.name)),
                      "peak_kind": f"bf16 dense burst, of {pk_kind}",
                      "flops_per_launch": flops, "launch_ms": stage_ms[2]},
         "clocks": clk.summary(),
@@ -239,6 +250,10 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
         frac = (c / vis).reshape(-1)
         out["support_fraction_deciles"] = [round(float(v), 4) for v in np.quantile(frac, np.linspace(0.1, 0.9, 9))]
         out["support_chunks_deciles"] = [int(v) for v in np.quantile(c.reshape(-1), np.linspace(0.1, 0.9, 9))]
+        # per-row support histogram: rows (position, KV head) by routed / visible chunks
+        edges = [0.0, 0.005, 0.01, 0.02, 0.05, 0.1, 0.2, 0.3, 0.5, 0.75, 1.0]
+        hist, _ = np.histogram(frac, bins=edges)
+        out["support_histogram"] = {"bin_edges": edges, "rows": [int(h) for h in hist]}
         del pf
         return out
     # e2e: host (pinned) inputs copied in, result copied out, every step, through the public API.
@@ -293,6 +308,7 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
                   "pipelining": "double-buffered: copy-in of step k+1 and copy-out of step k-1 overlap step k"}
     del dbuf[1], pfs[1]
     out["dense_causal"] = dense_denominators(wl, tq, qbar, pf, steps, flush, ms, dev)
+    out["stage2_list_vs_bitmask"] = stage2_variants(wl, tq, qbar, steps, flush, dev)
     out["_inputs"] = x
     return out
 
@@ -371,6 +387,50 @@ def oracle_backward_sample(wl, x, counts, ntok=2048):
                       f"the oracle parallelises over (sequence, KV head) pairs"}
 
 
+def stage2_variants(wl, tq, qbar, steps, flush, dev):
+    """Stage 2 driven by the compact ascending chunk lists (the default) and by the bit-packed
+    block mask M_i (32 chunks per word, as the paper review's Stage 2 kernel walks it) on the same
+    routes, device-timed side by side (L2 flushed); the two outputs must agree bit for bit."""
+    import torch
+    import adaptive_sparse_hierarchical_b200 as D
+    from adaptive_sparse_hierarchical_b200 import _lib as L
+
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    pfm = D.Prefill(tq["Q"], tq["K"], tq["V"], qbar, chunk=wl.chunk, alpha=wl.alpha, gamma=wl.gamma,
+                    inv_sigma=wl.inv_sigma, want_route=True, bitmask=True)
+    try:
+        pfm()
+        torch.cuda.synchronize(dev)
+        o_list = pfm.O.clone()
+
+        def timed(stage):
+            for _ in range(3):
+                pfm.stage(stage)
+            torch.cuda.synchronize(dev)
+            tot = 0.0
+            for k in range(steps):
+                flush.fill_(k & 0xff)
+                a, b = ev(), ev()
+                a.record(stream)
+                pfm.stage(stage)
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                tot += a.elapsed_time(b)
+            return tot / steps
+
+        res = {"stage1_with_bitmask_output_ms": timed(L.DASH_STAGE1), "stage2_list_ms": timed(L.DASH_STAGE2)}
+        res["stage2_bitmask_ms"] = timed(L.DASH_STAGE2_BITMASK)
+        torch.cuda.synchronize(dev)
+        res["bit_identical"] = bool(torch.equal(pfm.O, o_list))
+        res["error_word"] = pfm.error_word()
+        return res
+    except Exception as e:   # reported, not fatal
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+    finally:
+        del pfm
+
+
 def dense_denominators(wl, tq, qbar, pf, steps, flush, sparse_ms, dev):
     """Same-box dense causal attention on the same Q, K, V (context for the sparse step, not part
     of `value`): (a) this library at gamma = 0, where every visible chunk is routed with bias 0 and
@@ -421,7 +481,7 @@ def dense_denominators(wl, tq, qbar, pf, steps, flush, sparse_ms, dev):
 
 
 # ---------------------------------------------------------------------------------------- decode
-def run_decode(steps, warmup, ranks, pk, pk_kind, name="decode_128k"):
+def run_decode(steps, warmup, ranks, pk, pk_kind, name="decode_128k", paged=True):
     import torch
     import adaptive_sparse_hierarchical_b200 as D
     from adaptive_sparse_hierarchical_b200 import workloads as W
@@ -514,6 +574,8 @@ def run_decode(steps, warmup, ranks, pk, pk_kind, name="decode_128k"):
            "clocks": clk.summary(), "gpu_launches": 4 * (nst - 1),   # append, routing, attend, merge
            "l2": f"KV caches ({2 * wl.batch * wl.n * wl.h_kv * wl.d * 2 / 1e9:.2f} GB) larger than L2"}
     res["us_per_token"] = res["us_per_step"] / wl.batch   # per sequence-token, one GPU
+    if not paged:
+        return res
     try:
         res["paged"] = paged_decode(wl, st, qn, kn, vn, prefix, nst, reset, stream, bps, pk, pk_kind, ranks)
         res["gpu_launches"] += res["paged"]["gpu_launches"]
@@ -625,7 +687,7 @@ def config_of(wl, args):
             "l2": "flushed between steps (256 MB write, outside the per-step events)"}
 
 
-def run_sweep(args, ranks, pk, pk_kind):
+def run_sweep(args, ranks, pk, pk_kind, steps=None, decode_steps=None, emit=True):
     """The 8B-class 64K prefill at 50 / 25 / 12.5% routed and the 128K alpha x chunk-size sweep on
     Gaussian-mixture inputs: per workload the device-timed step, Mtok/s, Stage 2 roofline and the
     per-row support (routed chunks / visible chunks) deciles.  Inputs shared by several workloads
@@ -633,6 +695,9 @@ def run_sweep(args, ranks, pk, pk_kind):
     import gc
     from adaptive_sparse_hierarchical_b200 import workloads as W
 
+    steps = args.steps if steps is None else steps
+    decode_steps = args.decode_steps if decode_steps is None else decode_steps
+    lines = []
     cache = {}
     for name in W.PREFILL_64K + W.SWEEP_128K:
         wl = W.get(name)
@@ -641,27 +706,33 @@ def run_sweep(args, ranks, pk, pk_kind):
             cache.clear()
             gc.collect()
             cache[key] = wl.make()
-        r = run_prefill(wl, args.steps, args.warmup, ranks, pk, pk_kind, x=cache[key], lite=True)
+        r = run_prefill(wl, steps, args.warmup, ranks, pk, pk_kind, x=cache[key], lite=True)
         line = {"sweep": name, "metric": "prefill Mtok/s", "value": r["value"], "unit": "Mtok/s",
                 "ms_per_step": r["ms_per_step"], "stages_ms": r["stages_ms"], "routed_fraction": r["routed_fraction"],
                 "stage2_roofline_frac": r["roofline"]["frac"], "stage2_routed_tflops": r["roofline"]["achieved"],
                 "support_fraction_deciles": r["support_fraction_deciles"],
-                "support_chunks_deciles": r["support_chunks_deciles"], "clocks": r["clocks"],
+                "support_chunks_deciles": r["support_chunks_deciles"],
+                "support_histogram": r["support_histogram"], "roofline": r["roofline"],
+                "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
                 "config": {"batch": wl.batch, "seq_len": wl.n, "h_q": wl.h_q, "h_kv": wl.h_kv, "d_h": wl.d,
                            "chunk": wl.chunk, "alpha": wl.alpha, "gamma": wl.gamma}}
-        if ranks.rank == 0:
+        lines.append(line)
+        if emit and ranks.rank == 0:
             print(json.dumps(line), flush=True)
     cache.clear()
     gc.collect()
     # decode at the pages' own shape: batch 24, 96K contexts, 75% and 93.75% sparsity
     for name in W.DECODE_96K:
-        r = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind, name=name)
+        r = run_decode(decode_steps, args.warmup, ranks, pk, pk_kind, name=name, paged=False)
         line = {"sweep": name, "metric": "decode us/token", "value": r["us_per_token"], "unit": "us/token",
                 "higher_is_better": False, "us_per_step": r["us_per_step"], "routed_fraction": r["routed_fraction"],
-                "roofline": r["roofline"], "clocks": r["clocks"], "steps": r["steps"], "workload": r["workload"]}
-        if ranks.rank == 0:
+                "roofline": r["roofline"], "clocks": r["clocks"], "steps": r["steps"], "workload": r["workload"],
+                "gpu_launches": r["gpu_launches"]}
+        lines.append(line)
+        if emit and ranks.rank == 0:
             print(json.dumps(line), flush=True)
         gc.collect()
+    return lines
 
 
 def main():
@@ -696,10 +767,11 @@ def main():
     x = pre.pop("_inputs")
     line = {"metric": METRIC, "value": pre["value"], "unit": "Mtok/s", "n_gpus": ranks.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, planted chunks; see DESIGN.md)",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian inputs with planted chunk directions)",
             "config": config_of(wl, args), "roofline": pre["roofline"], "e2e": pre["e2e"],
             "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "stages_ms": pre["stages_ms"],
-            "routed_fraction": pre["routed_fraction"], "dense_causal": pre["dense_causal"]}
+            "routed_fraction": pre["routed_fraction"], "dense_causal": pre["dense_causal"],
+            "stage2_list_vs_bitmask": pre["stage2_list_vs_bitmask"]}
     if not args.no_decode:
         line["decode"] = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind)
         line["gpu_launches"] += line["decode"]["gpu_launches"]
@@ -710,6 +782,16 @@ def main():
             line["gpu_launches"] += line["backward"]["gpu_launches"]
         except Exception as e:   # reported in the line; the forward numbers above stand
             line["backward"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if ranks.world == 1 and not args.no_sweep:
+        # the 8B-class 64K prefill at 50 / 25 / 12.5% routed, the 128K alpha x chunk-size sweep with
+        # its per-row support histogram, and the batch-24 decode at 96K (75% and 93.75% sparsity),
+        # a few device-timed steps each (the inputs are generated outside the timed regions)
+        try:
+            line["sweeps"] = run_sweep(args, ranks, pk, pk_kind, steps=args.sweep_steps,
+                                       decode_steps=args.sweep_decode_steps, emit=False)
+            line["gpu_launches"] += sum(ln.get("gpu_launches", 0) for ln in line["sweeps"])
+        except Exception as e:   # reported in the line; the numbers above stand
+            line["sweeps"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
         v, secs, thr = oracle_sample(wl, x, args.cpu_rows)
         line["cpu_baseline"] = {"value": v / 1e6, "unit": "Mtok/s", "cores": thr, "kind": "oracle",

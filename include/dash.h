@@ -26,6 +26,20 @@
  *     bytes; other pointers 4 bytes.
  *   - Return value: DASH_OK (0) or a negative DASH_E* status.  Arguments are checked before any
  *     launch; on an error nothing is enqueued.  DASH_ELAUNCH reports a failed kernel launch.
+ *
+ * Environment switches (read once per process; for comparison runs and tests -- every setting
+ * computes the same routes and outputs, only the kernels that produce them differ):
+ *   DASH_STAGE2=mma       prefill Stage 1 / Stage 2 and decode Stage 2 on the warp-level mma.sync
+ *                         kernels instead of the tcgen05 / TMA ones (paged decode keeps the TMA path)
+ *   DASH_STAGE2=tile      prefill Stage 2 on the one-tile tcgen05 kernel (64-key jobs, two blocks
+ *                         per SM) instead of the paired-tile kernel (128-key jobs shared by two tiles)
+ *   DASH_CLUSTER=0        prefill Stage 2 forms its 128-row tiles from consecutive positions
+ *                         instead of grouping positions with similar routes (the grouping changes
+ *                         only the schedule: outputs are bit-identical)
+ *   DASH_LONG_ROUTE=off   rows of more than 512 chunks are routed by the per-shape kernels instead
+ *                         of the long-row tcgen05 kernel
+ *   DASH_DEC_ROUTE=heads  decode Stage 1 runs as three per-head launches instead of one clustered
+ *                         launch (the path very long contexts take anyway)
  */
 #ifndef DASH_H
 #define DASH_H
@@ -54,7 +68,8 @@ typedef struct {
     int seqlen;     /* prefill: sequence length n; decode/append: K/V cache capacity (positions) */
     int h_q, h_kv;  /* h_q % h_kv == 0; group size g_q = h_q / h_kv in {1, 2, 4, 8, 16} */
     int d_h;        /* head dimension: 64 or 128 */
-    int chunk;      /* B: 16, 32, 64 or 128 */
+    int chunk;      /* B: 1, 16, 32, 64 or 128 (1: every token is its own chunk, Stage 0 is the identity
+                       and Stage 1 is entmax over the visible tokens) */
     float alpha;    /* entmax alpha in (1, 2] (section 3 background formula) */
     float gamma;    /* routing scale gamma >= 0 (Eq. 6); 0 routes every visible chunk uniformly */
     float inv_sigma;/* 1/sigma of Eq. 11 / Prop. 4.1; 1 = plain prior, 0 = sigma -> infinity */
@@ -102,8 +117,13 @@ int dash_prefill(const dash_params* p, const void* Q, const void* K, const void*
 /* One stage of dash_prefill on its own (same arguments): stage 0 writes the summaries, stage 1
  * reads them and writes the routing lists, stage 2 reads both and writes O.  Running the three
  * stages in order on one stream with the same buffers equals dash_prefill; the intermediate
- * results must stay in kbar_out / route / workspace between the calls. */
-enum { DASH_STAGE0 = 0, DASH_STAGE1 = 1, DASH_STAGE2 = 2 };
+ * results must stay in kbar_out / route / workspace between the calls.
+ * DASH_STAGE2_BITMASK is Stage 2 driven by the bit-packed block mask M_i (route->bitmask, written
+ * by a stage-1 call that was given a bitmask output; the paper review's Stage 2 kernel walks the
+ * active chunks of M) together with the bias lists, instead of the chunk-id lists; its output
+ * equals DASH_STAGE2's bit for bit.  DASH_EINVAL without route->bitmask; DASH_EUNSUPPORTED unless
+ * bf16, d_h = 128, chunk 32 / 64 / 128. */
+enum { DASH_STAGE0 = 0, DASH_STAGE1 = 1, DASH_STAGE2 = 2, DASH_STAGE2_BITMASK = 3 };
 int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const void* K, const void* V,
                        const float* qbar, void* O, float* kbar_out, const dash_route_out* route,
                        void* workspace, size_t ws_bytes, void* stream);
@@ -172,18 +192,22 @@ int dash_decode_paged(const dash_params* p, const dash_paged_kv* pk, const void*
  * (for example a plugin inside a runtime that owns every device allocation and gives it no
  * allocator, or a service that must not grow its device footprint once running).  The paper has
  * no counterpart; this is a deployment variant of dash_decode with the same arguments minus
- * route/workspace, and the same results.
+ * route/workspace, and the same results bit for bit.
  *   Scratch: a fixed 16 MiB device array inside the library (one per GPU that loads it, held
- *   until the process exits).  A request whose scratch (per-head logits, route lists, split
- *   partials) exceeds 16 MiB returns DASH_EWORKSPACE before anything is enqueued.
+ *   until the process exits).  A request whose decode workspace, dash_workspace_size(p,
+ *   DASH_OP_DECODE), exceeds 16 MiB returns DASH_EWORKSPACE before anything is enqueued; invalid
+ *   parameters return what dash_decode would (DASH_EINVAL or DASH_EUNSUPPORTED).
+ *   status: device int32 written on the stream after the decode kernels: 0, or the non-zero code
+ *   of a bounded on-chip wait that timed out (the output is then not valid).  NULL skips it.
  *   The array is shared by every call on a GPU and keeps the last call's contents (each call
  *   writes every scratch value before reading it): calls whose kernels overlap on the GPU race
  *   and must be serialised by the caller.
- *   The first call on each device looks up the array's device address with that device current
- *   and caches it; make that first call before any stream capture.
+ *   The array's device address is looked up the first time the call runs under a given (device,
+ *   CUDA context) pair, with that device current, and cached for that pair; make that first call
+ *   before any stream capture.
  *   Allocates nothing (no cudaMalloc / cudaFree / allocating library routine). */
 int dash_decode_noalloc(const dash_params* p, const void* q, const void* K_cache, const void* V_cache,
-                        const float* kbar_cache, const int* seqlens, void* O, void* stream);
+                        const float* kbar_cache, const int* seqlens, void* O, int* status, void* stream);
 
 /* Backward pass of dash_prefill: gradients of L = sum(dO * O) with respect to Q, K, V and qbar.
  * The paper review page (section 3, the text after Eq. 9) states that the output is

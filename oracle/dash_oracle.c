@@ -16,7 +16,7 @@
  * Stage 0 and Stage 2 wording is also confirmed by the gist.science technical summary,
  * "Methodology", Stage 0 / Stage 2.
  *
- * Readings where the pages are silent (each one is listed in the design notes):
+ * Readings where the pages are silent (the plainest reading each passage supports):
  *   chunks are contiguous from position 0, c(j) = floor(j/B); a query at position i routes only
  *   over complete chunks c < floor(i/B); its own chunk is the diagonal branch D_i = {c(i)B .. i}
  *   and carries bias 0; rows with floor(i/B) = 0 have no routed branch; 1/sqrt(d) scales the

@@ -63,6 +63,21 @@ def check_routes(gsets, orc_route, B, positions, T):
     return mism, len(gsets)
 
 
+def bias_tolerance(margins, alpha, gamma, inv_sigma):
+    """Allowed |GPU bias - oracle bias| for each routed chunk of one row (margins: the oracle's
+    max over the group's heads of x_c - tau, in units of x = (alpha-1) gamma zbar).
+
+    The bias is (log w_c - mu) / sigma with w_c the group mean of [x_c - tau]_+^(1/(alpha-1)).  A
+    logit error of delta (in x units) moves log w_c by at most delta / ((alpha-1) m_c) through the
+    head that sets the margin m_c, and mu by the mean of that over the routed chunks.  The GPU's
+    chunk logits carry an absolute error of about 1e-5 in zbar (fp32 summaries and fp32
+    accumulation), i.e. delta = 2e-5 (alpha-1) max(gamma, 1) with a factor 2 of headroom."""
+    m = np.maximum(np.asarray(margins, dtype=np.float64), 1e-12)
+    delta = 2e-5 * (alpha - 1) * max(gamma, 1.0)
+    s = delta / ((alpha - 1) * m)
+    return 1e-4 + inv_sigma * (s + s.mean())
+
+
 def check_outputs(O_gpu, O_ref, dtype, g, mism=(), orc_route=None, B=None, positions=None, T=None):
     """O_* [b, rows, h_q, d].  Returns dict of error statistics and the list of ill-conditioned rows
     that exceeded the tolerance (each explained by a near-threshold chunk)."""

@@ -87,7 +87,8 @@ def _check_step(st, x, q, lengths, *, chunk, alpha, gamma, dtype, inv_sigma=1.0)
 
 
 @pytest.mark.parametrize("dtype,d,B,g", [("bf16", 128, 64, 4), ("bf16", 64, 32, 16), ("f32", 128, 64, 8),
-                                         ("bf16", 128, 128, 8), ("bf16", 128, 16, 2)])
+                                         ("bf16", 128, 128, 8), ("bf16", 128, 16, 2), ("bf16", 128, 1, 4),
+                                         ("f32", 64, 1, 2)])
 def test_decode_steps_small(dtype, d, B, g):
     hkv, cap, b = 2, 1024, 3
     x = inputs.planted(21, b, cap, g * hkv, hkv, d, B, dtype=dtype, chunk_frac=0.1)

@@ -1,11 +1,12 @@
 """GPU parity of decoding on paged K/V caches (dash_summary_build_paged / dash_summary_append_paged /
 dash_decode_paged through the C ABI).
 
-A paged pool holds the same tokens as a contiguous cache, only scattered over pages in the order
-the page table gives, so every result must equal the contiguous calls bit for bit: the summary
-cache, the incomplete-chunk state and the outputs, step after step.  The contiguous calls are
-themselves checked against the float64 oracle in test_gpu_decode.py; the last step here is also
-checked against the oracle directly."""
+Every paged step is checked against the float64 oracle directly (oracle.decode on the same
+tokens: routed sets by the margin rule, outputs at the bf16 tolerance, the bitmask against the
+lists) on a schedule of steps that includes the steps around a page move, and the paged summary
+cache and incomplete-chunk state against oracle.stage0.  A paged pool holds the same tokens as a
+contiguous cache, only scattered over pages in the order the page table gives, so in addition
+every result must equal the contiguous calls bit for bit, step after step."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +15,7 @@ import adaptive_sparse_hierarchical_b200 as D
 from adaptive_sparse_hierarchical_b200 import inputs
 from adaptive_sparse_hierarchical_b200.api import PagedDecodeState
 
-from test_gpu_decode import _check_step, _state
+from test_gpu_decode import _check_step, _check_summaries, _state
 
 pytestmark = pytest.mark.gpu
 
@@ -53,6 +54,7 @@ def test_paged_decode_equals_contiguous(B, page_size):
     pg.fill(torch.from_numpy(x["K"][:, :L0]).to("cuda", torch.bfloat16),
             torch.from_numpy(x["V"][:, :L0]).to("cuda", torch.bfloat16), lengths)
     torch.cuda.synchronize()
+    _check_summaries(pg, x, B)
     assert torch.equal(pg.kbar, ref.kbar)
     assert torch.equal(pg.state, ref.state)
 
@@ -64,6 +66,10 @@ def test_paged_decode_equals_contiguous(B, page_size):
         o_ref = ref.step(q, k, v)
         o = pg.step(q, k, v)
         torch.cuda.synchronize()
+        if step % 20 == 0 or step in (59, 61, 62):
+            # the paged step against the float64 oracle on the same tokens
+            L = lengths + step + 1
+            _check_step(pg, x, x["Q"][np.arange(b), L - 1], L, chunk=B, alpha=1.5, gamma=6.0, dtype="bf16")
         assert torch.equal(o, o_ref), step
         assert torch.equal(pg.seqlens, ref.seqlens)
         if step == 60:
@@ -80,6 +86,7 @@ def test_paged_decode_equals_contiguous(B, page_size):
     assert torch.equal(pg.state, ref.state)
     assert torch.equal(pg.rt[0], ref.rt[0]) and torch.equal(pg.bm, ref.bm)
     _check_step(pg, x, x["Q"][np.arange(b), last - 1], last, chunk=B, alpha=1.5, gamma=6.0, dtype="bf16")
+    _check_summaries(pg, x, B)
 
     # the pool holds exactly the contiguous cache's tokens, at the places the table gives
     for bb in range(b):

@@ -44,24 +44,22 @@ def compare(x, pf, O, *, chunk, alpha, gamma, inv_sigma=1.0, dtype="bf16", posit
     gs = gpu_sets(pf.counts.cpu().numpy(), pf.chunk_idx.cpu().numpy(), positions, chunk)
     mism, nrows = check_routes(gs, rt, chunk, positions, T)
     assert len(mism) <= max(1, 0.01 * nrows), f"{len(mism)} of {nrows} rows differ"
-    # biases of matching rows (chunks clear of the threshold)
+    # biases of every row whose routed set matches, each chunk against a tolerance that grows as
+    # its margin to the threshold shrinks (log w is ill-conditioned there)
     idx = pf.chunk_idx.cpu().numpy()
     bias = pf.bias.cpu().numpy()
     cnts = pf.counts.cpu().numpy()
-    from parity import tri_offset
+    from parity import bias_tolerance, tri_offset
     worst = 0.0
     for (bb, r, t), lst in gs.items():
         if (bb, r, t) in mism or len(lst) == 0:
             continue
         i = int(positions[t])
         off = tri_offset(i, chunk)
-        # log w amplifies a logit error by 2/margin near the threshold (ill-conditioned there), so
-        # the bias is compared only on rows whose routed chunks all clear the threshold by 1e-2
-        mg = np.abs(rt["margin"][bb, r, t, lst])
-        if mg.min() < 1e-2:
-            continue
-        worst = max(worst, np.abs(bias[bb, r, off:off + cnts[bb, r, i]] - rt["bias"][bb, r, t, lst]).max())
-    assert worst < 5e-3, worst
+        err = np.abs(bias[bb, r, off:off + cnts[bb, r, i]] - rt["bias"][bb, r, t, lst])
+        tol = bias_tolerance(rt["margin"][bb, r, t, lst], alpha, gamma, inv_sigma)
+        assert np.all(err <= tol), (bb, r, i, err.max(), tol[np.argmax(err - tol)])
+        worst = max(worst, float((err / tol).max()))
     Og = O.float().cpu().numpy()[:, positions]
     return check_outputs(Og, Oref, dtype, hq // hkv, mism, rt, chunk, positions, T)
 
@@ -89,6 +87,11 @@ CASES = [
     (1000, 8, 2, 128, 32, 6.0, 1.5, 1.0, "bf16"),
     (700, 16, 1, 128, 32, 7.0, 2.0, 0.5, "bf16"),
     (1100, 4, 2, 128, 32, 3.0, 1.25, 1.0, "bf16"),
+    # B = 1: every token is its own chunk (Stage 0 is the identity, Stage 1 is entmax over the
+    # visible tokens, the diagonal branch is the query's own token)
+    (300, 8, 2, 128, 1, 6.0, 1.5, 1.0, "bf16"),
+    (530, 16, 2, 128, 1, 8.0, 1.5, 1.0, "bf16"),
+    (200, 4, 1, 64, 1, 4.0, 2.0, 0.5, "f32"),
 ]
 
 
@@ -247,19 +250,30 @@ np.save(sys.argv[2], O.view(torch.int16).cpu().numpy())
 """
 
 
-def test_position_grouping_changes_only_the_schedule(tmp_path):
+@pytest.mark.parametrize("kernel", ["tile", "pair"])
+def test_position_grouping_changes_only_the_schedule(tmp_path, kernel):
     """Stage 2 orders a sparse window's positions by their first routed chunk before forming the
-    128-row tiles.  A row's arithmetic does not depend on its tile-mates (a tile the row does not
-    route adds exact zeros to its sums), so the output equals the sequence-order run
-    (DASH_CLUSTER=0) bit for bit.  Mixture inputs at gamma 1 route ~2% of the chunks, so every
-    window takes the grouped order."""
+    128-row tiles.  With the one-tile kernel (DASH_STAGE2=tile) a row's arithmetic does not depend
+    on its tile-mates (a key tile the row does not route adds exact zeros to its sums, and every
+    chunk is its own job), so the output equals the sequence-order run (DASH_CLUSTER=0) bit for
+    bit.  The paired-tile kernel packs two union chunks into each 128-key job, so which chunks
+    share a job (and with it the fp32 summation order) depends on the grouping: the two runs then
+    agree to the rounding of the bf16 output.  Mixture inputs at gamma 1 route ~2% of the chunks,
+    so every window takes the grouped order."""
     here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     outs = []
     for flag in ("1", "0"):
         f = tmp_path / f"o_{flag}.npy"
         env = dict(os.environ, DASH_CLUSTER=flag)
+        if kernel == "tile":
+            env["DASH_STAGE2"] = "tile"
         r = subprocess.run([sys.executable, "-c", _GROUPING_CHILD, here, str(f)], env=env,
                            capture_output=True, text=True, timeout=600)
         assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
         outs.append(np.load(f))
-    assert np.array_equal(outs[0], outs[1])
+    if kernel == "tile":
+        assert np.array_equal(outs[0], outs[1])
+    else:
+        a, b = (torch.from_numpy(o).view(torch.bfloat16).float() for o in outs)
+        err = (a - b).abs()
+        assert err.max().item() <= 2e-2 and (err.mean() / b.abs().mean()).item() <= 1e-3
