@@ -250,8 +250,9 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
                                                  reinterpret_cast<int*>(ws + L.perm), err, st));
     if (stage == DASH_STAGE2_BITMASK) {
         if (!rt.bitmask) return DASH_EINVAL;
-        if (!attend_pair_supported(s, p->dtype)) return DASH_EUNSUPPORTED;
-        rc = launch_status(launch_attend_prefill_mask(s, Q, K, V, O, rt, reinterpret_cast<int*>(ws + L.perm), err, st));
+        if (!attend_mask_supported(s, p->dtype)) return DASH_EUNSUPPORTED;
+        rc = launch_status(launch_attend_prefill_bitmask(s, p->dtype, Q, K, V, O, rt,
+                                                         reinterpret_cast<int*>(ws + L.perm), err, st));
     }
     return rc;
 }

@@ -178,10 +178,17 @@ cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, cons
 // when one of its bounded waits times out.
 bool attend_tc_supported(const Shape& s, int dtype);
 // perm: workspace of batch * h_kv * n ints for the grouped position order (null: sequence order)
+// mask = true: the routed support is read from rt.bitmask (the bit-packed block mask) instead of
+// the chunk lists, with identical results.
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
-                                     const Routes& rt, int* perm, int* err, cudaStream_t st);
+                                     const Routes& rt, int* perm, int* err, cudaStream_t st, bool mask = false);
 bool legacy_stage2();
-bool single_tile_stage2();
+bool pair_stage2();
+// Stage 2 driven by the bit-packed block mask on the tensor-core kernel the list-driven Stage 2 uses
+// for these shapes; cudaErrorNotSupported where neither tensor-core kernel applies.
+bool attend_mask_supported(const Shape& s, int dtype);
+cudaError_t launch_attend_prefill_bitmask(const Shape& s, int dtype, const void* Q, const void* K, const void* V,
+                                          void* O, const Routes& rt, int* perm, int* err, cudaStream_t st);
 // Helpers of the tensor-core Stage 2 kernels (stage2_tc.cu): a 4-D TMA map over a
 // [batch, n, heads, 128] bf16 tensor with box (64 d, bh heads, bp positions, 1) and 128-byte
 // swizzle; whether positions are grouped by route similarity before tiling; the grouping launch.
@@ -190,7 +197,7 @@ bool s2_encode_available();
 bool s2_grouping_enabled(const Shape& s);
 cudaError_t launch_group_positions(const Shape& s, const Routes& rt, int P, int* perm, cudaStream_t st);
 // Paired-tile Stage 2 (stage2_pair.cu): one block per two 128-row tiles sharing one key walk of
-// 128-key jobs (bf16, d = 128, chunk 32 / 64 / 128, 128 % g == 0).
+// 128-key jobs (bf16, d = 128, chunk 32 / 64 / 128, g in {4, 8, 16}); selected by DASH_STAGE2=pair.
 bool attend_pair_supported(const Shape& s, int dtype);
 cudaError_t launch_attend_prefill_pair(const Shape& s, const void* Q, const void* K, const void* V, void* O,
                                        const Routes& rt, int* perm, int* err, cudaStream_t st);

@@ -491,7 +491,7 @@ cudaError_t rows_t(const Shape& s, const void* Q, const void* K, const void* V, 
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K, const void* V,
                                   void* O, const Routes& rt, int* perm, int* err, cudaStream_t st)
 {
-    if (attend_pair_supported(s, dtype) && !legacy_stage2() && !single_tile_stage2())
+    if (pair_stage2() && attend_pair_supported(s, dtype))
         return launch_attend_prefill_pair(s, Q, K, V, O, rt, perm, err, st);
     if (attend_tc_supported(s, dtype) && !legacy_stage2())
         return launch_attend_prefill_tc(s, Q, K, V, O, rt, perm, err, st);
@@ -507,15 +507,31 @@ cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, cons
                       : rows_t<float, 64>(s, Q, K, V, O, rt, nullptr, st);
 }
 
-bool single_tile_stage2()
+bool pair_stage2()
 {
-    // DASH_STAGE2=tile selects the one-tile tcgen05 kernel (64-key jobs, two blocks per SM)
+    // DASH_STAGE2=pair selects the paired-tile tcgen05 kernel (two tiles per block, 128-key jobs)
     static int v = -1;
     if (v < 0) {
         const char* e = getenv("DASH_STAGE2");
-        v = (e && e[0] == 't') ? 1 : 0;
+        v = (e && e[0] == 'p') ? 1 : 0;
     }
     return v == 1;
+}
+
+bool attend_mask_supported(const Shape& s, int dtype)
+{
+    if (pair_stage2() && attend_pair_supported(s, dtype)) return true;
+    return attend_tc_supported(s, dtype) && !legacy_stage2();
+}
+
+cudaError_t launch_attend_prefill_bitmask(const Shape& s, int dtype, const void* Q, const void* K, const void* V,
+                                          void* O, const Routes& rt, int* perm, int* err, cudaStream_t st)
+{
+    if (pair_stage2() && attend_pair_supported(s, dtype))
+        return launch_attend_prefill_mask(s, Q, K, V, O, rt, perm, err, st);
+    if (attend_tc_supported(s, dtype) && !legacy_stage2())
+        return launch_attend_prefill_tc(s, Q, K, V, O, rt, perm, err, st, true);
+    return cudaErrorNotSupported;
 }
 
 bool legacy_stage2()

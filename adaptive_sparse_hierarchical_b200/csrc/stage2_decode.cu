@@ -345,17 +345,31 @@ __global__ void __launch_bounds__(D) dec_merge_kernel(Shape s, const float* __re
     const bool all_nonempty = total >= nblocks;
     const float* basep = part + (long long)x * nblocks * G * 130 + (long long)row * 130;
     const long long sstride = (long long)G * 130;
-    float M = -INFINITY;
-    for (int c = c0; c <= c1; ++c)
-        if (all_nonempty || jlo(c) < jlo(c + 1)) M = fmaxf(M, basep[c * sstride + 128]);
-    float Lsum = 0.f, o = 0.f;
-    for (int c = c0; c <= c1; ++c) {
-        if (!(all_nonempty || jlo(c) < jlo(c + 1))) continue;
-        const float mk = basep[c * sstride + 128];
-        if (mk == -INFINITY) continue;
-        const float w = exp2f(mk - M);
-        Lsum += basep[c * sstride + 129] * w;
-        o += basep[c * sstride + col] * w;
+    // one pass with a running maximum; four partials' loads in flight at a time
+    float M = -INFINITY, Lsum = 0.f, o = 0.f;
+    for (int c = c0; c <= c1; c += 4) {
+        float mk[4], lk[4], ok[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int cc = c + q;
+            const bool use = cc <= c1 && (all_nonempty || jlo(cc) < jlo(cc + 1));
+            mk[q] = use ? basep[cc * sstride + 128] : -INFINITY;
+            lk[q] = use ? basep[cc * sstride + 129] : 0.f;
+            ok[q] = use ? basep[cc * sstride + col] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (mk[q] == -INFINITY) continue;
+            if (mk[q] > M) {
+                const float sc = exp2f(M - mk[q]);
+                Lsum *= sc;
+                o *= sc;
+                M = mk[q];
+            }
+            const float w = exp2f(mk[q] - M);
+            Lsum += lk[q] * w;
+            o += ok[q] * w;
+        }
     }
     O[((long long)b * s.hq + r * G + row) * D + col] = __float2bfloat16_rn(Lsum > 0.f ? o / Lsum : 0.f);
 }

@@ -14,24 +14,33 @@
 // which halves the L2-to-shared-memory traffic per FLOP of a one-tile walk; rows that did not
 // route a job's chunk get -inf there.
 //
-// TMEM (512 columns): tile u keeps S_u in columns [256u, 256u+128) (P_u, bf16, over the first 64
-// of them) and O_u in [256u+128, 256u+256).  Roles (10 warps):
-//   warp 0     TMA producer: both Q tiles once, then per job K and V (two-slot rings)
-//   warp 1     TMEM owner; one thread issues the MMAs (S = Q K^T: M=128, N=128, K=128;
-//              O += P V: M=128, N=128, K=128 with P from TMEM) in the order
-//                S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...
-//              so that one tile's softmax runs while the tensor core works on the other tile
-//   warps 2-5  softmax of tile 0, warps 6-9 softmax of tile 1, one thread per row (TMEM lane):
-//              S from TMEM in blocks of 32 columns, bias / causal mask per chunk of the job,
-//              p = 2^(s - m) against the row's running maximum m kept from earlier jobs (the
-//              values stay <= 2^8, exact in the final normalisation), P packed to bf16 in
-//              registers and stored to TMEM once per job.  When a job holds a value above
-//              m + 8, m moves to the job's maximum, O is rescaled, and the job is recomputed
-//              from S, which is still intact in TMEM (P has not been stored yet).
+// TMEM (512 columns): tile u keeps S_u in columns [256u, 256u+128) (P_u as bf16 pairs in columns
+// [0, 32) and [64, 96) of it: each 64-key half over the start of its own S columns) and O_u in
+// [256u+128, 256u+256).  Roles (20 warps):
+//   warp 0      TMA producer: both Q tiles once, then per job K and V (two-slot rings)
+//   warp 1      TMEM owner; one thread issues the MMAs (S = Q K^T: M=128, N=128, K=128;
+//               O += P V: M=128, N=128, K=128 with P from TMEM) in the order
+//                 S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...
+//               so that one tile's softmax runs while the tensor core works on the other tile
+//   warp 2      routing: one lane per position walks the position's routed chunks and writes,
+//               for every job, each position's bias per chunk of the job (log2 units; 0 on the
+//               position's diagonal chunk; -inf where it did not route the chunk) into a ring of
+//               kRD jobs in shared memory, ahead of the softmax
+//   warp 3      idle after the set-up
+//   warps 4-19  softmax, two threads per row: tile u = (warp-4)/8 takes the 64-key half
+//               hf = ((warp-4)/4) % 2 of every job for the rows of TMEM lane quarter warp % 4.
+//               Per job: the half's maximum of the biased logits, exchanged with the other half
+//               through shared memory; the row's running maximum m moves only when the job
+//               exceeds it by more than 2^8 (O and the sums are then rescaled), otherwise the
+//               stale maximum is kept (values stay <= 2^8, exact in the final normalisation);
+//               p = 2^(s - m) as bf16 pairs into the half's 32 P columns of TMEM.
+// (The two halves' P columns lie inside each half's own S columns, so neither half writes where
+// the other still reads S.)
 // MASK = true reads the routed support from the bit-packed block mask (one bit per (position,
 // chunk), 32 chunks per word) instead of the ascending chunk lists; the biases are read in the
 // same ascending order, so both variants compute identical results.
-// Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
+// Every wait is bounded (mbarriers only, no named barriers between roles or halves); on time-out
+// the block records an error code and leaves.
 #include <climits>
 
 #include "dash_common.cuh"
@@ -44,17 +53,18 @@ constexpr int kRows = 128, kD = 128, kJK = 128;        // rows per tile, head di
 constexpr int kQBytes = kRows * kD * 2;                 // 32 KB per tile: two d-halves of [128 rows][64 d]
 constexpr int kKVHalf = kJK * 64 * 2;                   // 16 KB: [128 keys][64 d]
 constexpr int kKVBytes = 2 * kKVHalf;                   // 32 KB: K (or V) of one job
-constexpr int kKSlots = 2;                              // K ring; the V ring has VS = 2 or 3 slots
 constexpr int kOffQ = 0;
-constexpr int kOffK = 2 * kQBytes;                      // 64 KB
-constexpr int kOffV = kOffK + kKSlots * kKVBytes;       // 128 KB
-constexpr int kNumBars = 18;
-// after the V ring: barriers, misc (tmem base, abort, jobs, units), the pair's positions
-// (2 * 128 / g ints), the union units (uint16, ascending, padded to whole jobs)
-__host__ __device__ constexpr int off_bar(int vs) { return kOffV + vs * kKVBytes; }
-__host__ __device__ constexpr int off_misc(int vs) { return off_bar(vs) + kNumBars * 8; }
-__host__ __device__ constexpr int off_pos(int vs) { return off_misc(vs) + 32; }
-constexpr int kThreads = 320;
+constexpr int kOffK = 2 * kQBytes;                      // 64 KB: K ring, 2 slots
+constexpr int kOffV = kOffK + 2 * kKVBytes;             // 128 KB: V ring, 2 slots
+constexpr int kRD = 8;                                  // jobs of routing data prepared ahead
+constexpr int kNumBars = 1 + 2 * 4 + 2 * 5 + kRD + 1;
+constexpr int kOffBar = kOffV + 2 * kKVBytes;           // 192 KB
+constexpr int kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort, jobs, units
+constexpr int kOffX = kOffMisc + 32;                    // [2 job parity][2 tiles][2 halves][128 rows] maxima
+constexpr int kOffL = kOffX + 2 * 2 * 2 * kRows * 4;    // [2 tiles][2 halves][128 rows] row sums
+constexpr int kOffRB = kOffL + 2 * 2 * kRows * 4;       // route ring [kRD][J][2P] floats, then positions, units
+constexpr int kThreads = 640;
+constexpr int kMaxP2 = 64;                              // positions per pair: 2 * 128 / g, g >= 4
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, 128, false, false);
@@ -95,43 +105,50 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return d;
 }
 
-// K slot j % 2 holds K_j until S_0(j) and S_1(j) are done (k_free); V slot j % VS holds V_j until
-// PV_0(j) and PV_1(j) are done (v_free).  V is needed later than K (after both tiles' softmax of
-// the job), so a third V slot keeps the load of V_j in flight while PV_1(j-2) still reads its
-// predecessor.  Per tile u: s_full (S_u of a job is in TMEM), p_full (its 128 softmax threads
-// wrote P_u), pv_done (PV_u completed).
+// K slot j % 2 holds K_j until S_0(j) and S_1(j) are done (k_free); V slot j % 2 holds V_j until
+// PV_0(j) and PV_1(j) are done (v_free).  Per tile u: s_full (S_u of a job is in TMEM), xchg (the
+// tile's 256 softmax threads posted their half maxima), p_full (they wrote P_u), pv_done (PV_u
+// completed), lsum (the two halves' row sums are posted, at the end).  route[k]: the routing data
+// of job j (k = j % kRD) is in shared memory.
 struct Bars {
-    uint32_t q_full, k_full[2], v_full[3], k_free[2], v_free[3], s_full[2], p_full[2], pv_done[2], drain;
+    uint32_t q_full, k_full[2], v_full[2], k_free[2], v_free[2];
+    uint32_t s_full[2], xchg[2], p_full[2], pv_done[2], lsum[2];
+    uint32_t route[kRD], drain;
 };
 
-__device__ __forceinline__ Bars make_bars(uint32_t base, int vs)
+__device__ __forceinline__ Bars make_bars(uint32_t base)
 {
     Bars b;
-    uint32_t a = base + off_bar(vs);
+    uint32_t a = base + kOffBar;
     b.q_full = a; a += 8;
     for (int k = 0; k < 2; ++k) { b.k_full[k] = a; a += 8; }
-    for (int k = 0; k < 3; ++k) { b.v_full[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.v_full[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.k_free[k] = a; a += 8; }
-    for (int k = 0; k < 3; ++k) { b.v_free[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.v_free[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.s_full[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.xchg[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.p_full[k] = a; a += 8; }
     for (int k = 0; k < 2; ++k) { b.pv_done[k] = a; a += 8; }
+    for (int k = 0; k < 2; ++k) { b.lsum[k] = a; a += 8; }
+    for (int k = 0; k < kRD; ++k) { b.route[k] = a; a += 8; }
     b.drain = a;
     return b;
 }
 
-// The row's routed chunks in ascending order, four at a time ahead of use, from the chunk list
-// (MASK = false) or from the bit-packed mask (MASK = true); the bias of the k-th routed chunk is
-// the k-th entry of the row's bias list in both cases.
+// A position's routed chunks in ascending order with their biases, from the chunk list (MASK =
+// false) or from the bit-packed mask (MASK = true; the bias of the k-th routed chunk is the k-th
+// entry of the position's bias list in both cases).  Two banks of four entries: the current bank
+// is consumed while the next one's loads are in flight, and the banks swap only when the current
+// one is used up, so no instruction reads a register whose load was issued shortly before.
 template <bool MASK>
 struct RouteQueue {
-    int c[4];
-    float bs[4];
-    int cnt, next;         // routed chunks, entries fetched so far
+    int cc[4], nc[4];
+    float cb[4], nb[4];
+    int k, cnt, next;
     const int* li;
     const float* lb;
-    const uint32_t* mw;    // the row's mask words (MASK)
-    uint32_t word;         // bits of mask word `wi` not yet taken
+    const uint32_t* mw;
+    uint32_t word, word2;
     int wi, words;
 
     __device__ __forceinline__ int fetch_chunk()
@@ -139,7 +156,8 @@ struct RouteQueue {
         if constexpr (MASK) {
             while (word == 0u) {
                 if (++wi >= words) return INT_MAX;
-                word = mw[wi];
+                word = word2;
+                word2 = wi + 1 < words ? mw[wi + 1] : 0u;
             }
             const int b = __ffs(word) - 1;
             word &= word - 1u;
@@ -148,36 +166,42 @@ struct RouteQueue {
             return li[next];
         }
     }
-    __device__ __forceinline__ void load(int k)
+    __device__ __forceinline__ void fill_next()
     {
-        if (next < cnt) {
-            c[k] = fetch_chunk();
-            bs[k] = lb[next];
-            ++next;
-        } else {
-            c[k] = INT_MAX;
-            bs[k] = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (next < cnt) {
+                nc[q] = fetch_chunk();
+                nb[q] = lb[next];
+                ++next;
+            } else {
+                nc[q] = INT_MAX;
+                nb[q] = 0.f;
+            }
         }
+    }
+    __device__ __forceinline__ void swap_banks()
+    {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { cc[q] = nc[q]; cb[q] = nb[q]; }
+        k = 0;
+        fill_next();
     }
     __device__ __forceinline__ void init(const int* li_, const float* lb_, const uint32_t* mw_, int words_, int cnt_)
     {
-        li = li_; lb = lb_; mw = mw_; words = words_; cnt = cnt_; next = 0;
-        wi = 0;
+        li = li_; lb = lb_; mw = mw_; words = words_; cnt = cnt_; next = 0; wi = 0;
         word = (MASK && cnt > 0) ? mw[0] : 0u;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) load(k);
+        word2 = (MASK && cnt > 0 && words > 1) ? mw[1] : 0u;
+        fill_next();
+        swap_banks();
     }
-    __device__ __forceinline__ void pop()
-    {
-        c[0] = c[1]; bs[0] = bs[1];
-        c[1] = c[2]; bs[1] = bs[2];
-        c[2] = c[3]; bs[2] = bs[3];
-        load(3);
-    }
+    __device__ __forceinline__ int front() const { return k == 0 ? cc[0] : k == 1 ? cc[1] : k == 2 ? cc[2] : cc[3]; }
+    __device__ __forceinline__ float front_bias() const { return k == 0 ? cb[0] : k == 1 ? cb[1] : k == 2 ? cb[2] : cb[3]; }
+    __device__ __forceinline__ void pop() { if (++k == 4) swap_banks(); }
 };
 
 // J = chunks per 128-key job (128 / B).
-template <int J, bool MASK, int VS>
+template <int J, bool MASK>
 __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                   const __grid_constant__ CUtensorMap tmQ1,
                                                                   const __grid_constant__ CUtensorMap tmK,
@@ -190,17 +214,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
     extern __shared__ char smem_raw[];
     char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = tc::smem_addr(sm);
-    const Bars bar = make_bars(base, VS);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + off_misc(VS));
-    volatile int* abort = reinterpret_cast<volatile int*>(sm + off_misc(VS) + 4);
-    int* njobs_s = reinterpret_cast<int*>(sm + off_misc(VS) + 8);
-    int* nunits_s = reinterpret_cast<int*>(sm + off_misc(VS) + 12);
-    int* spos = reinterpret_cast<int*>(sm + off_pos(VS));
+    const Bars bar = make_bars(base);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+    int* njobs_s = reinterpret_cast<int*>(sm + kOffMisc + 8);
+    int* nunits_s = reinterpret_cast<int*>(sm + kOffMisc + 12);
+    float* xsh = reinterpret_cast<float*>(sm + kOffX);
+    float* lsh = reinterpret_cast<float*>(sm + kOffL);
     uint32_t* umask = reinterpret_cast<uint32_t*>(sm + kOffK);   // set-up scratch until the first TMA
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = s.g, P = kRows / G, P2 = 2 * P;
-    uint16_t* jobs = reinterpret_cast<uint16_t*>(sm + off_pos(VS) + 4 * P2);
+    float* rb = reinterpret_cast<float*>(sm + kOffRB);            // [kRD][J][P2]
+    int* spos = reinterpret_cast<int*>(sm + kOffRB + kRD * J * P2 * 4);
+    uint16_t* jobs = reinterpret_cast<uint16_t*>(sm + kOffRB + kRD * J * P2 * 4 + 4 * P2);
     const int nblk = (s.n + P - 1) / P;
     const int npairs = (nblk + 1) / 2;
     const int br = blockIdx.x % (s.batch * s.hkv);
@@ -216,17 +243,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
     // ---- set-up: barriers, TMEM, union of the pair's routed + diagonal chunks ------------------
     if (tid == 0) {
         tc::mbar_init(bar.q_full, 1);
-        for (int k = 0; k < VS; ++k) {
-            tc::mbar_init(bar.v_full[k], 1);
-            tc::mbar_init(bar.v_free[k], 1);
-        }
         for (int k = 0; k < 2; ++k) {
             tc::mbar_init(bar.k_full[k], 1);
+            tc::mbar_init(bar.v_full[k], 1);
             tc::mbar_init(bar.k_free[k], 1);
+            tc::mbar_init(bar.v_free[k], 1);
             tc::mbar_init(bar.s_full[k], 1);
-            tc::mbar_init(bar.p_full[k], 128);
+            tc::mbar_init(bar.xchg[k], 256);
+            tc::mbar_init(bar.p_full[k], 256);
             tc::mbar_init(bar.pv_done[k], 1);
+            tc::mbar_init(bar.lsum[k], 256);
         }
+        for (int k = 0; k < kRD; ++k) tc::mbar_init(bar.route[k], 1);
         tc::mbar_init(bar.drain, 1);
         *abort = 0;
         tc::mbar_fence_init();
@@ -258,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
         // the positions' list lengths and their prefix sums (scratch in the V ring), then every
         // list entry by a flat index, several independent loads per thread in flight
         int* pcnt = reinterpret_cast<int*>(sm + kOffV);
-        int* poff = pcnt + 2 * kRows;
+        int* poff = pcnt + kMaxP2;
         for (int p = tid; p < P2; p += blockDim.x) {
             const int i = spos[p];
             pcnt[p] = i < s.n ? counts[i] : 0;
@@ -329,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
         __syncwarp();
         // padding entries repeat the last unit (real keys, finite values); every row masks them
         const int nj = (basec + J - 1) / J;
-        if (lane < nj * J - basec) jobs[basec + lane] = basec > 0 ? jobs[basec - 1] : 0;
+        if (lane < nj * J - basec) jobs[basec + lane] = basec > 0 ? jobs[basec - 1] : (uint16_t)0;
         if (lane == 0) {
             *njobs_s = nj;
             *nunits_s = basec;
@@ -366,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
             }
             // loads in the order of first use: K_0, V_0, K_1, V_1, ...; slot j % 2 is refilled
             // once both tiles' MMAs of job j - 2 that read it have completed
-            int lastk[2] = {-1, -1}, lastv[3] = {-1, -1, -1};
+            int lastk[2] = {-1, -1}, lastv[2] = {-1, -1};
             for (int j = 0; j < njobs; ++j) {
                 const int slot = j & 1;
                 if (j >= 2 && !tc::mbar_wait(bar.k_free[slot], ((j >> 1) - 1) & 1, abort, err, 21)) break;
@@ -379,28 +407,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
                     tc::tma_load_4d(dst, &tmK, bar.k_full[slot], 0, r, key0, b);
                     tc::tma_load_4d(dst + kKVHalf, &tmK, bar.k_full[slot], 64, r, key0, b);
                 }
-                const int vsl = j % VS;
-                if (j >= VS && !tc::mbar_wait(bar.v_free[vsl], ((j / VS) - 1) & 1, abort, err, 22)) break;
-                lastv[vsl] = j;
-                tc::mbar_expect_tx(bar.v_full[vsl], kKVBytes);
+                if (j >= 2 && !tc::mbar_wait(bar.v_free[slot], ((j >> 1) - 1) & 1, abort, err, 22)) break;
+                lastv[slot] = j;
+                tc::mbar_expect_tx(bar.v_full[slot], kKVBytes);
 #pragma unroll
                 for (int sg = 0; sg < J; ++sg) {
                     const int key0 = jobs[j * J + sg] * SEG;
-                    const uint32_t dst = base + kOffV + vsl * kKVBytes + sg * SEG * 128;
-                    tc::tma_load_4d(dst, &tmV, bar.v_full[vsl], 0, r, key0, b);
-                    tc::tma_load_4d(dst + kKVHalf, &tmV, bar.v_full[vsl], 64, r, key0, b);
+                    const uint32_t dst = base + kOffV + slot * kKVBytes + sg * SEG * 128;
+                    tc::tma_load_4d(dst, &tmV, bar.v_full[slot], 0, r, key0, b);
+                    tc::tma_load_4d(dst + kKVHalf, &tmV, bar.v_full[slot], 64, r, key0, b);
                 }
             }
             if (*abort) {
                 // let this block's TMA copies still in flight land before its shared memory goes away
-                for (int k = 0; k < 2; ++k)
+                for (int k = 0; k < 2; ++k) {
                     if (lastk[k] >= 0)
                         for (long long it = 0; it < (1ll << 22); ++it)
                             if (tc::mbar_try(bar.k_full[k], (lastk[k] >> 1) & 1)) break;
-                for (int k = 0; k < VS; ++k)
                     if (lastv[k] >= 0)
                         for (long long it = 0; it < (1ll << 22); ++it)
-                            if (tc::mbar_try(bar.v_full[k], (lastv[k] / VS) & 1)) break;
+                            if (tc::mbar_try(bar.v_full[k], (lastv[k] >> 1) & 1)) break;
+                }
                 for (long long it = 0; it < (1ll << 22); ++it)
                     if (tc::mbar_try(bar.q_full, 0)) break;
             }
@@ -424,11 +451,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
                 tc::mma_commit(bar.s_full[u]);
             };
             auto issue_pv = [&](int u, int j) {
-                const uint64_t dv = dV0 + (uint64_t)(((j % VS) * kKVBytes) >> 4);
+                const uint64_t dv = dV0 + (uint64_t)(((j & 1) * kKVBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kJK / 16; ++kk)
-                    tc::mma_f16_ts(tmem + 256u * u + 128u, tmem + 256u * u + kk * 8, dv + (uint64_t)((kk * 2048) >> 4),
-                                   kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kJK / 16; ++kk)   // P of keys 16kk.. : columns 8kk (+32 for the upper half)
+                    tc::mma_f16_ts(tmem + 256u * u + 128u, tmem + 256u * u + kk * 8 + (kk >= 4 ? 32u : 0u),
+                                   dv + (uint64_t)((kk * 2048) >> 4), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(bar.pv_done[u]);
             };
             bool ok = tc::mbar_wait(bar.q_full, 0, abort, err, 23) && tc::mbar_wait(bar.k_full[0], 0, abort, err, 24);
@@ -441,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
             for (int j = 0; ok && j < njobs; ++j) {
                 const bool more = j + 1 < njobs;
                 if (!tc::mbar_wait(bar.p_full[0], j & 1, abort, err, 25) ||
-                    !tc::mbar_wait(bar.v_full[j % VS], (j / VS) & 1, abort, err, 26)) { ok = false; break; }
+                    !tc::mbar_wait(bar.v_full[j & 1], (j >> 1) & 1, abort, err, 26)) { ok = false; break; }
                 tc::fence_after_sync();
                 issue_pv(0, j);
                 if (more) {
@@ -452,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
                 if (!tc::mbar_wait(bar.p_full[1], j & 1, abort, err, 28)) { ok = false; break; }
                 tc::fence_after_sync();
                 issue_pv(1, j);
-                tc::mma_commit(bar.v_free[j % VS]);
+                tc::mma_commit(bar.v_free[j & 1]);
                 if (more) {
                     issue_s(1, j + 1);
                     tc::mma_commit(bar.k_free[(j + 1) & 1]);
@@ -465,76 +492,161 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
                     if (tc::mbar_try(bar.drain, 0)) break;
             }
         }
-    } else {
-        // ---- softmax: tile u, one thread per row ----------------------------------------------------
-        const int u = (warp - 2) >> 2;
-        const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
-        const int row = q4 * 32 + lane;
-        const int pl = row / G, h = row % G;
-        const int i = spos[u * P + pl];
-        const bool valid = i < s.n;
-        const int diag = valid ? i / s.B : -1;
-        const long long toff = valid ? tri_offset(i, s.B) : 0;
-        RouteQueue<MASK> rq;
-        rq.init(ridx + toff, rbias + toff, MASK ? rmask + (long long)(valid ? i : 0) * rt.words : nullptr, rt.words,
-                valid ? counts[i] : 0);
-        const float scale2 = kLog2e * rsqrtf((float)kD);
-        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + 256u * u;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
+    } else if (warp == 2) {
+        // ---- routing: lane = position (and position + 32 when the pair has 64) ------------------
+        constexpr int kPerLane = kMaxP2 / 32;
+        RouteQueue<MASK> rq[kPerLane];
+        int diag[kPerLane];
+        bool vld[kPerLane];
+#pragma unroll
+        for (int q = 0; q < kPerLane; ++q) {
+            const int p = lane + 32 * q;
+            const int i = p < P2 ? spos[p] : INT_MAX;
+            vld[q] = i < s.n;
+            diag[q] = vld[q] ? i / s.B : -1;
+            const long long toff = vld[q] ? tri_offset(i, s.B) : 0;
+            rq[q].init(ridx + toff, rbias + toff, MASK ? rmask + (long long)(vld[q] ? i : 0) * rt.words : nullptr,
+                       rt.words, vld[q] ? counts[i] : 0);
+        }
         for (int j = 0; j < njobs; ++j) {
-            // waits are made warp-uniform: the tcgen05 loads and stores below are .sync.aligned
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.s_full[u], j & 1, abort, err, 29))) { ok = false; break; }
-            tc::fence_after_sync();
-            float bias2[J];
-            bool dg[J];
+            const int slot = j % kRD;
+            // slot reuse: both tiles' softmax of job j - kRD has finished reading it
+            if (j >= kRD && !__all_sync(0xffffffffu, tc::mbar_wait(bar.p_full[0], (j - kRD) & 1, abort, err, 32) &&
+                                                         tc::mbar_wait(bar.p_full[1], (j - kRD) & 1, abort, err, 33)))
+                break;
+            float* dst = rb + slot * J * P2;
 #pragma unroll
             for (int sg = 0; sg < J; ++sg) {
                 const int e = j * J + sg;
                 const int unit = jobs[e];
-                bias2[sg] = -INFINITY;
-                dg[sg] = false;
-                if (valid && e < nunits) {
-                    if (rq.c[0] == unit) {
-                        bias2[sg] = rq.bs[0] * kLog2e;
-                        rq.pop();
-                    } else if (unit == diag) {
-                        bias2[sg] = 0.f;
-                        dg[sg] = true;
+#pragma unroll
+                for (int q = 0; q < kPerLane; ++q) {
+                    const int p = lane + 32 * q;
+                    float b2 = -INFINITY;
+                    if (vld[q] && e < nunits) {
+                        if (rq[q].front() == unit) {
+                            b2 = rq[q].front_bias() * kLog2e;
+                            rq[q].pop();
+                        } else if (unit == diag[q]) {
+                            b2 = 0.f;
+                        }
                     }
+                    if (p < P2) dst[sg * P2 + p] = b2;
                 }
             }
-            uint32_t pk[kJK / 2];
-            float js = 0.f;
-            // one pass over S against the reference maximum mref; returns the largest exponent
-            // 2^x it produced (x = s*scale2 + bias2 - mref), -inf when the row uses none of the job
-            auto attempt = [&](float mref) -> float {
-                const unsigned long long sc2 = f2(scale2, scale2);
-                unsigned long long ls2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-                float xm = -INFINITY;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar.route[slot]);
+        }
+    } else if (warp >= 4) {
+        // ---- softmax: tile u, key half hf, two threads per row ------------------------------------
+        const int w4 = warp - 4;
+        const int u = w4 >> 3, hf = (w4 >> 2) & 1;
+        const int q4 = warp & 3;                  // TMEM lane quarter this warp may access
+        const int row = q4 * 32 + lane;
+        const int pl = row / G, h = row % G;
+        const int pidx = u * P + pl;
+        const int i = spos[pidx];
+        const bool valid = i < s.n;
+        const int diag = valid ? i / s.B : -1;
+        const float scale2 = kLog2e * rsqrtf((float)kD);
+        const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + 256u * u;
+        // S of this half: columns 64 hf + [0, 64); its P (bf16 pairs) over the first 32 of them,
+        // which only this half reads; O of this half: 128 + 64 hf + [0, 64)
+        const uint32_t scol = 64u * hf, pcol = 64u * hf, ocol = 128u + 64u * hf;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < njobs; ++j) {
+            const int slot = j % kRD;
+            // waits are made warp-uniform: the tcgen05 loads and stores below are .sync.aligned
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.route[slot], (j / kRD) & 1, abort, err, 34) &&
+                                             tc::mbar_wait(bar.s_full[u], j & 1, abort, err, 29))) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            // this half's two 32-key blocks: bias (log2 units; -inf: not routed or padding) and
+            // the block's first key when it lies on the row's diagonal chunk (causal mask)
+            float b2[2];
+            int j0[2];
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    const int sg = (cb * 32) / SEG;
-                    if (__all_sync(0xffffffffu, bias2[sg] == -INFINITY)) {
+            for (int cb = 0; cb < 2; ++cb) {
+                const int kin = 64 * hf + 32 * cb;           // first key of the block within the job
+                const int sg = kin / SEG;
+                b2[cb] = rb[(slot * J + sg) * P2 + pidx];
+                const int unit = jobs[j * J + sg];
+                j0[cb] = unit == diag ? unit * SEG + kin % SEG : -1;
+            }
+            // pass 1: the half's maximum of the biased logits
+            float xm = -INFINITY;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[16 * cb + e] = 0u;
-                        continue;
+            for (int cb = 0; cb < 2; ++cb) {
+                if (__all_sync(0xffffffffu, b2[cb] == -INFINITY)) continue;
+                float v[32];
+                tc::tmem_ld32(tbase + scol + 32 * cb, v);
+                tc::tmem_wait_ld();
+                if (j0[cb] >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j0[cb] + e > i) v[e] = -INFINITY;
+                }
+                float a = fmax3(v[0], v[1], v[2]);
+#pragma unroll
+                for (int e = 3; e < 31; e += 2) a = fmax3(a, v[e], v[e + 1]);
+                a = fmaxf(a, v[31]);
+                if (b2[cb] != -INFINITY) xm = fmaxf(xm, fmaf(a, scale2, b2[cb]));
+            }
+            // the row's maximum over both halves (shared memory, per job parity)
+            float* xs = xsh + (((j & 1) * 2 + u) * 2) * kRows;
+            xs[hf * kRows + row] = xm;
+            tc::mbar_arrive(bar.xchg[u]);
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.xchg[u], j & 1, abort, err, 35))) { ok = false; break; }
+            const float xr = fmaxf(xs[row], xs[kRows + row]);
+            // the running maximum moves when the job exceeds it by more than 2^8 (or holds the
+            // row's first used key); O (this half's 64 columns) and l are rescaled
+            const bool need = xr != -INFINITY && (m == -INFINITY || xr > m + 8.f);
+            if (__any_sync(0xffffffffu, need)) {
+                const float f = need && m != -INFINITY ? ex2_approx(m - xr) : 1.f;
+                if (__any_sync(0xffffffffu, f != 1.f)) {
+                    // PV_u(j-1) has completed: it precedes S_u(j) on the tensor pipe
+                    if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[u], (j - 1) & 1, abort, err, 30))) {
+                        ok = false;
+                        break;
                     }
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int ob = 0; ob < 2; ++ob) {
+                        float o[32];
+                        tc::tmem_ld32(tbase + ocol + 32 * ob, o);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] *= f;
+                        tc::tmem_st32(tbase + ocol + 32 * ob, o);
+                    }
+                }
+                l *= f;
+                if (need) m = xr;
+            }
+            // pass 2: p = 2^(s*scale2 + bias2 - m), bf16 pairs into this half's 32 P columns; a
+            // block that no row of the warp uses is written as zeros without computing
+            const float mref = m == -INFINITY ? 0.f : m;
+            const unsigned long long sc2 = f2(scale2, scale2);
+            unsigned long long ls2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t pk[16];
+                if (__all_sync(0xffffffffu, b2[cb] == -INFINITY)) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                } else {
                     float v[32];
-                    tc::tmem_ld32(lane_base + cb * 32, v);
+                    tc::tmem_ld32(tbase + scol + 32 * cb, v);
                     tc::tmem_wait_ld();
-                    if (dg[sg]) {   // keys past the query on its diagonal chunk
-                        const int j0 = diag * SEG + (cb * 32) % SEG;
+                    if (j0[cb] >= 0) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if (j0 + e > i) v[e] = -INFINITY;
+                            if (j0[cb] + e > i) v[e] = -INFINITY;
                     }
-                    float a = fmax3(v[0], v[1], v[2]);
-#pragma unroll
-                    for (int e = 3; e < 31; e += 2) a = fmax3(a, v[e], v[e + 1]);
-                    a = fmaxf(a, v[31]);
-                    const float off = bias2[sg] - mref;
-                    if (bias2[sg] != -INFINITY) xm = fmaxf(xm, fmaf(a, scale2, off));
+                    const float off = b2[cb] - mref;
                     const unsigned long long off2 = f2(off, off);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -543,76 +655,50 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
                         const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         ls2[e & 1] = fadd2(ls2[e & 1], f2(p0, p1));
                         __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
-                        pk[16 * cb + e] = *reinterpret_cast<uint32_t*>(&t2);
+                        pk[e] = *reinterpret_cast<uint32_t*>(&t2);
                     }
                 }
-                float a0, a1, b0, b1;
-                unf2(ls2[0], a0, a1);
-                unf2(ls2[1], b0, b1);
-                js = (a0 + a1) + (b0 + b1);
-                return xm;
-            };
-            float xm = attempt(m == -INFINITY ? 0.f : m);
-            // the running maximum moves when the job exceeds it by more than 2^8 (or when it is
-            // the row's first job with a used key); O and l are rescaled, and the job is redone
-            const bool need = xm != -INFINITY && (m == -INFINITY || xm > 8.f);
-            if (__any_sync(0xffffffffu, need)) {
-                const float mnew = need ? (m == -INFINITY ? xm : m + xm) : m;
-                if (__any_sync(0xffffffffu, need && m != -INFINITY)) {
-                    // PV_u(j-1) has completed: it precedes S_u(j) on the tensor pipe
-                    if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[u], (j - 1) & 1, abort, err, 30))) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
-                    const float f = need && m != -INFINITY ? ex2_approx(m - mnew) : 1.f;
-                    l *= f;
-#pragma unroll
-                    for (int cb = 0; cb < 4; ++cb) {
-                        float o[32];
-                        tc::tmem_ld32(lane_base + 128 + cb * 32, o);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= f;
-                        tc::tmem_st32(lane_base + 128 + cb * 32, o);
-                    }
-                }
-                m = mnew;
-                attempt(m == -INFINITY ? 0.f : m);
+                tc::tmem_st16(tbase + pcol + 16 * cb, pk);
             }
-            l += js;
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tc::tmem_st16(lane_base + cb * 16, pk + 16 * cb);
+            float a0, a1, c0, c1;
+            unf2(ls2[0], a0, a1);
+            unf2(ls2[1], c0, c1);
+            l += (a0 + a1) + (c0 + c1);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(bar.p_full[u]);
         }
-        // ---- epilogue: O / l -> bf16 --------------------------------------------------------------
-        if (ok && njobs > 0 &&
-            __all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[u], (njobs - 1) & 1, abort, err, 31))) {
-            tc::fence_after_sync();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = valid ? O + (long long)b * s.os[0] + (long long)i * s.os[1] +
-                                              (long long)(r * G + h) * s.os[2]
-                                        : nullptr;
+        // ---- epilogue: the two halves' sums, O / l -> bf16 (each half writes its 64 columns) -----
+        if (ok && njobs > 0) {
+            lsh[(u * 2 + hf) * kRows + row] = l;
+            tc::mbar_arrive(bar.lsum[u]);
+            if (__all_sync(0xffffffffu, tc::mbar_wait(bar.lsum[u], 0, abort, err, 36) &&
+                                            tc::mbar_wait(bar.pv_done[u], (njobs - 1) & 1, abort, err, 31))) {
+                tc::fence_after_sync();
+                const float lt = lsh[(u * 2) * kRows + row] + lsh[(u * 2 + 1) * kRows + row];
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                __nv_bfloat16* orow = valid ? O + (long long)b * s.os[0] + (long long)i * s.os[1] +
+                                                  (long long)(r * G + h) * s.os[2] + 64 * hf
+                                            : nullptr;
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float o[32];
-                tc::tmem_ld32(lane_base + 128 + cb * 32, o);
-                tc::tmem_wait_ld();
-                if (orow) {
+                for (int ob = 0; ob < 2; ++ob) {
+                    float o[32];
+                    tc::tmem_ld32(tbase + ocol + 32 * ob, o);
+                    tc::tmem_wait_ld();
+                    if (orow) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 w4;
-                        __nv_bfloat162 a0 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
-                        __nv_bfloat162 a1 = __floats2bfloat162_rn(o[e + 2] * inv, o[e + 3] * inv);
-                        __nv_bfloat162 a2 = __floats2bfloat162_rn(o[e + 4] * inv, o[e + 5] * inv);
-                        __nv_bfloat162 a3 = __floats2bfloat162_rn(o[e + 6] * inv, o[e + 7] * inv);
-                        w4.x = *reinterpret_cast<uint32_t*>(&a0);
-                        w4.y = *reinterpret_cast<uint32_t*>(&a1);
-                        w4.z = *reinterpret_cast<uint32_t*>(&a2);
-                        w4.w = *reinterpret_cast<uint32_t*>(&a3);
-                        *reinterpret_cast<uint4*>(orow + cb * 32 + e) = w4;
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 w4;
+                            __nv_bfloat162 a0 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
+                            __nv_bfloat162 a1 = __floats2bfloat162_rn(o[e + 2] * inv, o[e + 3] * inv);
+                            __nv_bfloat162 a2 = __floats2bfloat162_rn(o[e + 4] * inv, o[e + 5] * inv);
+                            __nv_bfloat162 a3 = __floats2bfloat162_rn(o[e + 6] * inv, o[e + 7] * inv);
+                            w4.x = *reinterpret_cast<uint32_t*>(&a0);
+                            w4.y = *reinterpret_cast<uint32_t*>(&a1);
+                            w4.z = *reinterpret_cast<uint32_t*>(&a2);
+                            w4.w = *reinterpret_cast<uint32_t*>(&a3);
+                            *reinterpret_cast<uint4*>(orow + 32 * ob + e) = w4;
+                        }
                     }
                 }
             }
@@ -628,21 +714,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
     }
 }
 
-size_t pair_smem(const Shape& s, int vs)
+size_t pair_smem(const Shape& s)
 {
-    const int P2 = 2 * (kRows / s.g);
-    return 1024 + (size_t)off_pos(vs) + 4 * (size_t)P2 + 2 * (size_t)(s.T + 2 + 4);
+    const int P2 = 2 * (kRows / s.g), J = s.B >= kJK ? 1 : kJK / s.B;
+    return 1024 + (size_t)kOffRB + (size_t)kRD * J * P2 * 4 + 4 * (size_t)P2 + 2 * (size_t)(s.T + 2 + 4);
 }
 
-// three V slots when they fit in shared memory, two otherwise
-int pair_vslots(const Shape& s) { return pair_smem(s, 3) <= 227 * 1024 ? 3 : 2; }
-
-template <int J, bool MASK, int VS>
-cudaError_t launch_jv(const Shape& s, const CUtensorMap& mq, const CUtensorMap& mq1, const CUtensorMap& mk,
-                      const CUtensorMap& mv, const Routes& rt, void* O, int* err, const int* perm, cudaStream_t st)
+template <int J, bool MASK>
+cudaError_t launch_j(const Shape& s, const CUtensorMap& mq, const CUtensorMap& mq1, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const Routes& rt, void* O, int* err, const int* perm, cudaStream_t st)
 {
-    auto kern = attend_pair_kernel<J, MASK, VS>;
-    const size_t smem = pair_smem(s, VS);
+    auto kern = attend_pair_kernel<J, MASK>;
+    const size_t smem = pair_smem(s);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int P = kRows / s.g;
@@ -653,23 +736,7 @@ cudaError_t launch_jv(const Shape& s, const CUtensorMap& mq, const CUtensorMap& 
     return cudaGetLastError();
 }
 
-template <int J, bool MASK>
-cudaError_t launch_j(const Shape& s, const CUtensorMap& mq, const CUtensorMap& mq1, const CUtensorMap& mk,
-                     const CUtensorMap& mv, const Routes& rt, void* O, int* err, const int* perm, cudaStream_t st)
-{
-    return pair_vslots(s) == 3 ? launch_jv<J, MASK, 3>(s, mq, mq1, mk, mv, rt, O, err, perm, st)
-                               : launch_jv<J, MASK, 2>(s, mq, mq1, mk, mv, rt, O, err, perm, st);
-}
-
-}  // namespace
-
-bool attend_pair_supported(const Shape& s, int dtype)
-{
-    return dtype == DASH_BF16 && s.d == kD && (s.B == 32 || s.B == 64 || s.B == 128) && s.g >= 1 && s.g <= 16 &&
-           (kRows % s.g) == 0 && s.T + 8 < 65536 && s2_encode_available() && pair_smem(s, 2) <= 227 * 1024;
-}
-
-static cudaError_t launch_attend_prefill_pair_impl(const Shape& s, const void* Q, const void* K, const void* V, void* O,
+cudaError_t launch_attend_prefill_pair_impl(const Shape& s, const void* Q, const void* K, const void* V, void* O,
                                             const Routes& rt, int* perm, int* err, bool mask, cudaStream_t st)
 {
     const int P = kRows / s.g;
@@ -695,6 +762,15 @@ static cudaError_t launch_attend_prefill_pair_impl(const Shape& s, const void* Q
     case 64: return launch_j<2, false>(s, mq, mq1, mk, mv, rt, O, err, pm, st);
     default: return launch_j<1, false>(s, mq, mq1, mk, mv, rt, O, err, pm, st);
     }
+}
+
+}  // namespace
+
+bool attend_pair_supported(const Shape& s, int dtype)
+{
+    return dtype == DASH_BF16 && s.d == kD && (s.B == 32 || s.B == 64 || s.B == 128) &&
+           (s.g == 4 || s.g == 8 || s.g == 16) && s.T + 8 < 65536 && s2_encode_available() &&
+           pair_smem(s) <= 227 * 1024;
 }
 
 cudaError_t launch_attend_prefill_pair(const Shape& s, const void* Q, const void* K, const void* V, void* O,

@@ -156,9 +156,43 @@ __global__ void __launch_bounds__(1024) group_positions_kernel(Shape s, Routes r
     }
 }
 
+// A position's routed chunks in ascending order, from the ascending chunk list (MASK = false: the
+// k-th entry) or from the bit-packed block mask M_i (MASK = true: the k-th set bit, taken in order
+// by a scan over the position's mask words).  The bias of the k-th routed chunk is the k-th entry of
+// the bias list either way, so both sources give identical results.
+template <bool MASK>
+struct ChunkSource {
+    const int* li;
+    const uint32_t* mw;
+    uint32_t word;
+    int wi, words;
+    __device__ __forceinline__ void init(const int* li_, const uint32_t* mw_, int words_, bool any)
+    {
+        li = li_; mw = mw_; words = words_; wi = 0;
+        word = MASK && any ? mw[0] : 0u;
+    }
+    // chunk id of entry k; entries are requested in increasing order, one after the other
+    __device__ __forceinline__ int at(int k)
+    {
+        if constexpr (MASK) {
+            (void)k;
+            while (word == 0u) {
+                if (++wi >= words) return INT_MAX;
+                word = mw[wi];
+            }
+            const int b = __ffs(word) - 1;
+            word &= word - 1u;
+            return (wi << 5) + b;
+        } else {
+            return li[k];
+        }
+    }
+};
+
 // CPT = chunks per 64-key tile: 1 for chunks of 64 or 128 keys (a chunk is one or two jobs), 2 for
 // 32-key chunks (a job covers two neighbouring chunks, each row with its own bias per half).
-template <int CPT>
+// MASK = true: the routed support comes from the bit-packed block mask instead of the chunk lists.
+template <int CPT, bool MASK>
 __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                    const __grid_constant__ CUtensorMap tmQ1,
                                                                    const __grid_constant__ CUtensorMap tmK,
@@ -188,6 +222,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
     const int* counts = rt.counts + (long long)br * s.n;
     const int* ridx = rt.idx + (long long)br * rt.cap;
     const float* rbias = rt.bias + (long long)br * rt.cap;
+    const uint32_t* rmask = MASK ? rt.bitmask + (long long)br * s.n * rt.words : nullptr;
     const int W = (s.T + 32) >> 5;
     const int NH = CPT == 1 ? s.B / kKT : 1;   // jobs per union unit (chunk, or 64-key tile)
     const int UB = CPT == 1 ? s.B : kKT;       // keys per union unit
@@ -221,18 +256,37 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         spos[p] = perm && k < s.n ? perm[(long long)br * s.n + k] : k;
     }
     __syncthreads();
-    for (int p = 0; p < P; ++p) {
-        const int i = spos[p];
-        if (i >= s.n) continue;
-        const int cnt = counts[i];
-        const int* li = ridx + tri_offset(i, s.B);
-        for (int k = tid; k < cnt; k += blockDim.x) {
-            const int u = li[k] / CPT;
+    if constexpr (MASK) {
+        // union units from the positions' mask words (chunks; pairs of chunks when CPT = 2)
+        for (int e = tid; e < P * rt.words; e += blockDim.x) {
+            const int i = spos[e / rt.words];
+            if (i >= s.n) continue;
+            uint32_t w = rmask[(long long)i * rt.words + e % rt.words];
+            while (w) {
+                const int c = ((e % rt.words) << 5) + __ffs(w) - 1;
+                w &= w - 1u;
+                const int u = c / CPT;
+                atomicOr(&umask[u >> 5], 1u << (u & 31));
+            }
+        }
+        if (tid < P && spos[tid] < s.n) {
+            const int u = (spos[tid] / s.B) / CPT;
             atomicOr(&umask[u >> 5], 1u << (u & 31));
         }
-        if (tid == 0) {
-            const int u = (i / s.B) / CPT;
-            atomicOr(&umask[u >> 5], 1u << (u & 31));
+    } else {
+        for (int p = 0; p < P; ++p) {
+            const int i = spos[p];
+            if (i >= s.n) continue;
+            const int cnt = counts[i];
+            const int* li = ridx + tri_offset(i, s.B);
+            for (int k = tid; k < cnt; k += blockDim.x) {
+                const int u = li[k] / CPT;
+                atomicOr(&umask[u >> 5], 1u << (u & 31));
+            }
+            if (tid == 0) {
+                const int u = (i / s.B) / CPT;
+                atomicOr(&umask[u >> 5], 1u << (u & 31));
+            }
         }
     }
     __syncthreads();
@@ -383,18 +437,20 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         const int* li = ridx + (valid ? tri_offset(i, s.B) : 0);
         const float* lb = rbias + (valid ? tri_offset(i, s.B) : 0);
         const int cnt = valid ? counts[i] : 0;
+        ChunkSource<MASK> cs;
+        cs.init(li, MASK ? rmask + (long long)(valid ? i : 0) * rt.words : nullptr, rt.words, cnt > 0);
         // the row's next two routed chunks stay in registers, so the global load of an entry is
         // issued at least one tile before the entry is compared
         int cur = 0;
-        int nxt = cnt > 0 ? li[0] : INT_MAX;
+        int nxt = cnt > 0 ? cs.at(0) : INT_MAX;
         float nbias = cnt > 0 ? lb[0] : 0.f;
-        int nxt2 = cnt > 1 ? li[1] : INT_MAX;
+        int nxt2 = cnt > 1 ? cs.at(1) : INT_MAX;
         float nbias2 = cnt > 1 ? lb[1] : 0.f;
         // two chunks per job: entries cur+2, cur+3 as well, and the queue only shifts at the end
         // of a job, so no compare waits on a load issued in the same job
-        int nxt3 = CPT > 1 && cnt > 2 ? li[2] : INT_MAX;
+        int nxt3 = CPT > 1 && cnt > 2 ? cs.at(2) : INT_MAX;
         float nbias3 = CPT > 1 && cnt > 2 ? lb[2] : 0.f;
-        int nxt4 = CPT > 1 && cnt > 3 ? li[3] : INT_MAX;
+        int nxt4 = CPT > 1 && cnt > 3 ? cs.at(3) : INT_MAX;
         float nbias4 = CPT > 1 && cnt > 3 ? lb[3] : 0.f;
         const float scale2 = kLog2e * rsqrtf((float)kD);
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
@@ -529,7 +585,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                     ++cur;
                     nxt = nxt2;
                     nbias = nbias2;
-                    nxt2 = cur + 1 < cnt ? li[cur + 1] : INT_MAX;
+                    nxt2 = cur + 1 < cnt ? cs.at(cur + 1) : INT_MAX;
                     nbias2 = cur + 1 < cnt ? lb[cur + 1] : 0.f;
                 }
             } else if (adv == 1) {
@@ -537,15 +593,15 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 nxt = nxt2; nbias = nbias2;
                 nxt2 = nxt3; nbias2 = nbias3;
                 nxt3 = nxt4; nbias3 = nbias4;
-                nxt4 = cur + 3 < cnt ? li[cur + 3] : INT_MAX;
+                nxt4 = cur + 3 < cnt ? cs.at(cur + 3) : INT_MAX;
                 nbias4 = cur + 3 < cnt ? lb[cur + 3] : 0.f;
             } else if (adv == 2) {
                 cur += 2;
                 nxt = nxt3; nbias = nbias3;
                 nxt2 = nxt4; nbias2 = nbias4;
-                nxt3 = cur + 2 < cnt ? li[cur + 2] : INT_MAX;
+                nxt3 = cur + 2 < cnt ? cs.at(cur + 2) : INT_MAX;
                 nbias3 = cur + 2 < cnt ? lb[cur + 2] : 0.f;
-                nxt4 = cur + 3 < cnt ? li[cur + 3] : INT_MAX;
+                nxt4 = cur + 3 < cnt ? cs.at(cur + 3) : INT_MAX;
                 nbias4 = cur + 3 < cnt ? lb[cur + 3] : 0.f;
             }
         }
@@ -667,7 +723,7 @@ size_t attend_tc_smem(const Shape& s)
 }
 
 cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* K, const void* V, void* O,
-                                     const Routes& rt, int* perm, int* err, cudaStream_t st)
+                                     const Routes& rt, int* perm, int* err, cudaStream_t st, bool mask)
 {
     CUtensorMap mq, mq1, mk, mv;
     const int P = kRows / s.g;
@@ -682,7 +738,9 @@ cudaError_t launch_attend_prefill_tc(const Shape& s, const void* Q, const void* 
         !make_map(&mk, K, s.batch, s.n, s.hkv, s.ks, 1, kKT) || !make_map(&mv, V, s.batch, s.n, s.hkv, s.vs, 1, kKT))
         return cudaErrorInvalidValue;
     const size_t smem = attend_tc_smem(s);
-    auto kern = s.B >= kKT ? attend_prefill_tc_kernel<1> : attend_prefill_tc_kernel<2>;
+    if (mask && !rt.bitmask) return cudaErrorInvalidValue;
+    auto kern = s.B >= kKT ? (mask ? attend_prefill_tc_kernel<1, true> : attend_prefill_tc_kernel<1, false>)
+                           : (mask ? attend_prefill_tc_kernel<2, true> : attend_prefill_tc_kernel<2, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long nblk = (s.n + P - 1) / P;

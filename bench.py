@@ -33,16 +33,16 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # DRAM bytes per launch of a Stage 2 kernel (dram__bytes_read.sum + dram__bytes_write.sum from one
 # ncu capture of the current kernel on that workload), keyed by (kernel, workload); absent until
 # the current kernel has been captured.
-STAGE2_TRAFFIC = {}
+STAGE2_TRAFFIC = {("attend_prefill_tc_kernel (tcgen05, one tile per block)", "prefill_32k"): 314.7e6}
 
 
 def stage2_kernel_name():
     sel = os.environ.get("DASH_STAGE2", "")
     if sel.startswith("m"):
         return "attend_prefill_mma_kernel (mma.sync)"
-    if sel.startswith("t"):
-        return "attend_prefill_tc_kernel (tcgen05, one tile per block)"
-    return "attend_pair_kernel (tcgen05, two tiles per block)"
+    if sel.startswith("p"):
+        return "attend_pair_kernel (tcgen05, two tiles per block)"
+    return "attend_prefill_tc_kernel (tcgen05, one tile per block)"
 
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")

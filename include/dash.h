@@ -31,8 +31,9 @@
  * computes the same routes and outputs, only the kernels that produce them differ):
  *   DASH_STAGE2=mma       prefill Stage 1 / Stage 2 and decode Stage 2 on the warp-level mma.sync
  *                         kernels instead of the tcgen05 / TMA ones (paged decode keeps the TMA path)
- *   DASH_STAGE2=tile      prefill Stage 2 on the one-tile tcgen05 kernel (64-key jobs, two blocks
- *                         per SM) instead of the paired-tile kernel (128-key jobs shared by two tiles)
+ *   DASH_STAGE2=pair      prefill Stage 2 on the paired-tile tcgen05 kernel (two 128-row tiles per
+ *                         block share one walk of 128-key jobs; g in {4, 8, 16}) instead of the
+ *                         one-tile kernel (64-key jobs, two blocks per SM)
  *   DASH_CLUSTER=0        prefill Stage 2 forms its 128-row tiles from consecutive positions
  *                         instead of grouping positions with similar routes (the grouping changes
  *                         only the schedule: outputs are bit-identical)
@@ -121,8 +122,8 @@ int dash_prefill(const dash_params* p, const void* Q, const void* K, const void*
  * DASH_STAGE2_BITMASK is Stage 2 driven by the bit-packed block mask M_i (route->bitmask, written
  * by a stage-1 call that was given a bitmask output; the paper review's Stage 2 kernel walks the
  * active chunks of M) together with the bias lists, instead of the chunk-id lists; its output
- * equals DASH_STAGE2's bit for bit.  DASH_EINVAL without route->bitmask; DASH_EUNSUPPORTED unless
- * bf16, d_h = 128, chunk 32 / 64 / 128. */
+ * equals DASH_STAGE2's bit for bit (same tensor-core kernel, same schedule).  DASH_EINVAL without
+ * route->bitmask; DASH_EUNSUPPORTED unless bf16, d_h = 128, chunk 32 / 64 / 128. */
 enum { DASH_STAGE0 = 0, DASH_STAGE1 = 1, DASH_STAGE2 = 2, DASH_STAGE2_BITMASK = 3 };
 int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const void* K, const void* V,
                        const float* qbar, void* O, float* kbar_out, const dash_route_out* route,

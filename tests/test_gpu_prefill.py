@@ -253,7 +253,7 @@ np.save(sys.argv[2], O.view(torch.int16).cpu().numpy())
 @pytest.mark.parametrize("kernel", ["tile", "pair"])
 def test_position_grouping_changes_only_the_schedule(tmp_path, kernel):
     """Stage 2 orders a sparse window's positions by their first routed chunk before forming the
-    128-row tiles.  With the one-tile kernel (DASH_STAGE2=tile) a row's arithmetic does not depend
+    128-row tiles.  With the one-tile kernel (the default) a row's arithmetic does not depend
     on its tile-mates (a key tile the row does not route adds exact zeros to its sums, and every
     chunk is its own job), so the output equals the sequence-order run (DASH_CLUSTER=0) bit for
     bit.  The paired-tile kernel packs two union chunks into each 128-key job, so which chunks
@@ -265,8 +265,8 @@ def test_position_grouping_changes_only_the_schedule(tmp_path, kernel):
     for flag in ("1", "0"):
         f = tmp_path / f"o_{flag}.npy"
         env = dict(os.environ, DASH_CLUSTER=flag)
-        if kernel == "tile":
-            env["DASH_STAGE2"] = "tile"
+        if kernel == "pair":
+            env["DASH_STAGE2"] = "pair"
         r = subprocess.run([sys.executable, "-c", _GROUPING_CHILD, here, str(f)], env=env,
                            capture_output=True, text=True, timeout=600)
         assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
@@ -277,3 +277,65 @@ def test_position_grouping_changes_only_the_schedule(tmp_path, kernel):
         a, b = (torch.from_numpy(o).view(torch.bfloat16).float() for o in outs)
         err = (a - b).abs()
         assert err.max().item() <= 2e-2 and (err.mean() / b.abs().mean()).item() <= 1e-3
+
+
+@pytest.mark.parametrize("B", [32, 64, 128])
+def test_bitmask_driven_stage2_equals_list_stage2(B):
+    """Stage 2 driven by the bit-packed block mask (DASH_STAGE2_BITMASK: the support read from
+    M_i, the biases in ascending chunk order) reproduces the list-driven Stage 2 bit for bit on the
+    same tensor-core kernel; the list-driven output is checked against the oracle first."""
+    from adaptive_sparse_hierarchical_b200 import _lib as L
+    x = inputs.planted(15, 1, 3000, 16, 2, 128, B, dtype="bf16", chunk_frac=0.1, strength=2.0)
+    O, pf = run_prefill(x, chunk=B, alpha=1.5, gamma=8.0, bitmask=True)
+    compare(x, pf, O, chunk=B, alpha=1.5, gamma=8.0, positions=_sample_positions(3000, B, 200, 4))
+    O_list = O.clone()
+    pf.O.fill_(float("nan"))
+    pf.stage(L.DASH_STAGE2_BITMASK)
+    torch.cuda.synchronize()
+    assert pf.error_word() == 0
+    assert torch.equal(pf.O, O_list)
+
+
+def test_bitmask_stage2_needs_a_bitmask():
+    from adaptive_sparse_hierarchical_b200 import _lib as L
+    x = inputs.planted(16, 1, 300, 8, 2, 128, 64, dtype="bf16")
+    O, pf = run_prefill(x, chunk=64, alpha=1.5, gamma=6.0, bitmask=False)
+    with pytest.raises(L.DashError):
+        pf.stage(L.DASH_STAGE2_BITMASK)
+
+
+_PAIR_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import oracle
+import adaptive_sparse_hierarchical_b200 as D
+from adaptive_sparse_hierarchical_b200 import _lib as L
+from adaptive_sparse_hierarchical_b200 import inputs
+B, g = int(sys.argv[2]), int(sys.argv[3])
+x = inputs.planted(17, 1, 1500, 2 * g, 2, 128, B, dtype="bf16", chunk_frac=0.1, strength=2.0)
+Q, K, V = (torch.from_numpy(x[k]).cuda().to(torch.bfloat16) for k in ("Q", "K", "V"))
+pf = D.Prefill(Q, K, V, torch.from_numpy(x["qbar"]).cuda(), chunk=B, alpha=1.5, gamma=8.0, want_route=True,
+               bitmask=True)
+O = pf().clone()
+torch.cuda.synchronize()
+assert pf.error_word() == 0
+ref, _ = oracle.prefill(x["Q"], x["K"], x["V"], x["qbar"], chunk=B, alpha=1.5, gamma=8.0)
+err = np.abs(O.float().cpu().numpy() - ref)
+assert err.max() <= 2e-2 and err.mean() / np.abs(ref).mean() <= 1e-2, (err.max(), err.mean())
+pf.O.fill_(float("nan"))
+pf.stage(L.DASH_STAGE2_BITMASK)
+torch.cuda.synchronize()
+assert pf.error_word() == 0 and torch.equal(pf.O, O)
+print("ok", err.max())
+"""
+
+
+@pytest.mark.parametrize("B,g", [(32, 8), (64, 8), (128, 16), (64, 4)])
+def test_paired_tile_stage2_kernel_against_oracle(B, g):
+    """The paired-tile tcgen05 Stage 2 kernel (DASH_STAGE2=pair: two 128-row tiles per block share
+    one walk of 128-key jobs), a selectable path, against the oracle in a child process (the switch
+    is read once), with its bitmask-driven variant bit-identical to its list-driven one."""
+    here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _PAIR_CHILD, here, str(B), str(g)],
+                       env=dict(os.environ, DASH_STAGE2="pair"), capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
