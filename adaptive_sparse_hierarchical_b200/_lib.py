@@ -84,6 +84,8 @@ def load():
         lib.dash_backward.restype = ctypes.c_int
         lib.dash_status_string.argtypes = [ctypes.c_int]
         lib.dash_status_string.restype = ctypes.c_char_p
+        lib.dash_set_wait_limit.argtypes = [ctypes.c_longlong]
+        lib.dash_set_wait_limit.restype = ctypes.c_longlong
         _lib = lib
     return _lib
 
@@ -146,6 +148,12 @@ def dash_route_capacity(p: dash_params) -> int:
 
 def dash_status_string(rc: int) -> str:
     return load().dash_status_string(rc).decode()
+
+
+def dash_set_wait_limit(polls: int) -> int:
+    """Poll limit of the tensor-core Stage 2 kernels' bounded waits for later launches (a
+    diagnostic knob; 0 makes the first wait give up).  Returns the previous limit."""
+    return int(load().dash_set_wait_limit(int(polls)))
 
 
 def dash_prefill(p, Q, K, V, qbar, O, kbar_out=None, route=None, workspace=None, ws_bytes=None,

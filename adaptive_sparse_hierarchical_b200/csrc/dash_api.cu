@@ -13,7 +13,15 @@ bool pow2_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16;
 
 }  // namespace
 
+#include <atomic>
+
 namespace dash {
+
+namespace {
+std::atomic<long long> g_wait_limit{1ll << 23};
+}
+
+long long wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
 
 // Shape checks shared by every entry point.
 int check_params(const dash_params* p)
@@ -64,6 +72,7 @@ Shape make_shape(const dash_params* p)
     s.pt = nullptr;
     s.psz = s.pmax = s.npages = 0;
     s.kps = s.vps = 0;
+    s.polls = wait_limit();
     return s;
 }
 
@@ -372,6 +381,12 @@ int dash_decode_paged(const dash_params* p, const dash_paged_kv* pk, const void*
 {
     if (!pk) return DASH_EINVAL;
     return decode(p, pk, q, K_pool, V_pool, kbar_cache, seqlens, O, route, workspace, ws_bytes, stream);
+}
+
+long long dash_set_wait_limit(long long polls)
+{
+    if (polls < 0) return -1;
+    return g_wait_limit.exchange(polls);
 }
 
 const char* dash_status_string(int status)

@@ -22,7 +22,11 @@ struct Shape {
     const int* pt;                       // page table [batch][pmax]
     int psz, pmax, npages;               // page size (tokens), pages per sequence, pool pages
     long long kps, vps;                  // elements between pages of the K / V pools
+    long long polls;                     // poll limit of the bounded waits of the Stage 2 tcgen05 kernels
 };
+
+// Poll limit the next launches' Shapes carry (dash_set_wait_limit; the default is kWaitPolls).
+long long wait_limit();
 
 // Element offset of token t of sequence b, KV head r in a K (st = ks, ps = kps) or V cache; -1
 // when the token's page is unmapped (a page id outside [0, npages), or t beyond the table), so

@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             for (int k = 0; k < kNS; ++k) lastk[k] = lastv[k] = -1;
             auto load_k = [&](int k) -> bool {
                 const int slot = k % kNS;
-                if (k >= kNS && !tc::mbar_wait(bar.s_full[slot], ((k / kNS) - 1) & 1, abort, err, 1)) return false;
+                if (k >= kNS && !tc::mbar_wait(bar.s_full[slot], ((k / kNS) - 1) & 1, abort, err, 1, s.polls)) return false;
                 lastk[slot] = k;
                 const int key0 = jobs[k / NH] * UB + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot;
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             };
             auto load_v = [&](int k) -> bool {
                 const int slot = k % kNS;
-                if (k >= kNS && !tc::mbar_wait(bar.pv_done[slot], ((k / kNS) - 1) & 1, abort, err, 10)) return false;
+                if (k >= kNS && !tc::mbar_wait(bar.pv_done[slot], ((k / kNS) - 1) & 1, abort, err, 10, s.polls)) return false;
                 lastv[slot] = k;
                 const int key0 = jobs[k / NH] * UB + (k % NH) * kKT;
                 const uint32_t dst = base + kOffSlots + slot * kSlot + 2 * kKVHalf;
@@ -392,8 +392,8 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             const uint64_t dV0 = tc::sw128_desc(base + kOffSlots + 2 * kKVHalf, kKVHalf, 1024);
             auto issue_pv = [&](int j) -> bool {
                 const int pbuf = j & 1;
-                if (!tc::mbar_wait(bar.p_full[pbuf], (j >> 1) & 1, abort, err, 2)) return false;
-                if (!tc::mbar_wait(bar.v_full[j % kNS], (j / kNS) & 1, abort, err, 13)) return false;
+                if (!tc::mbar_wait(bar.p_full[pbuf], (j >> 1) & 1, abort, err, 2, s.polls)) return false;
+                if (!tc::mbar_wait(bar.v_full[j % kNS], (j / kNS) & 1, abort, err, 13, s.polls)) return false;
                 tc::fence_after_sync();
                 const uint64_t dv = dV0 + (uint64_t)(((j % kNS) * kSlot) >> 4);
                 // P_j (bf16, 2 per column) sits in the first 32 columns of S buffer pbuf
@@ -404,11 +404,11 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
                 tc::mma_commit(bar.pv_done[pbuf]);
                 return true;
             };
-            bool ok = tc::mbar_wait(bar.q_full, 0, abort, err, 3);
+            bool ok = tc::mbar_wait(bar.q_full, 0, abort, err, 3, s.polls);
             for (int k = 0; ok && k < njobs; ++k) {
                 const int slot = k % kNS, sb = k & 1;
-                if (!tc::mbar_wait(bar.k_full[slot], (k / kNS) & 1, abort, err, 4)) { ok = false; break; }
-                if (k >= 2 && !tc::mbar_wait(bar.s_free[sb], ((k - 2) >> 1) & 1, abort, err, 5)) { ok = false; break; }
+                if (!tc::mbar_wait(bar.k_full[slot], (k / kNS) & 1, abort, err, 4, s.polls)) { ok = false; break; }
+                if (k >= 2 && !tc::mbar_wait(bar.s_free[sb], ((k - 2) >> 1) & 1, abort, err, 5, s.polls)) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint64_t dk = dK0 + (uint64_t)((slot * kSlot) >> 4);
 #pragma unroll
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         for (int k = 0; k < njobs; ++k) {
             const int sb = k & 1;
             // waits are made warp-uniform: the tcgen05 loads and stores below are .sync.aligned
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.s_full[sb], (k >> 1) & 1, abort, err, 6))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.s_full[sb], (k >> 1) & 1, abort, err, 6, s.polls))) { ok = false; break; }
             tc::fence_after_sync();
             float v[64];
             tc::tmem_ld32(lane_base + sb * 64, v);
@@ -523,7 +523,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             if (m == -INFINITY) m = mt;
             if (__any_sync(0xffffffffu, need)) {
                 // rescale O: wait until the previous P V has landed
-                if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort, err, 7))) {
+                if (!__all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort, err, 7, s.polls))) {
                     ok = false;
                     break;
                 }
@@ -607,7 +607,7 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
         }
         // ---- epilogue: O / l -> bf16 --------------------------------------------------------
         if (ok && njobs > 0 &&
-            __all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[(njobs - 1) & 1], ((njobs - 1) >> 1) & 1, abort, err, 9))) {
+            __all_sync(0xffffffffu, tc::mbar_wait(bar.pv_done[(njobs - 1) & 1], ((njobs - 1) >> 1) & 1, abort, err, 9, s.polls))) {
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16* orow = valid ? O + (long long)b * s.os[0] + (long long)i * s.os[1] +

@@ -49,10 +49,13 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
 // try_wait itself suspends for a short hardware-defined time).  On time-out the shared abort
 // flag and the global error word are set and false is returned, so that every role of the block
 // leaves its loop and the block tears down normally.
+// `polls` overrides the limit (the tensor-core Stage 2 kernels take it from the launch's Shape, so
+// that a diagnostic setting can make their waits run out on purpose; see dash_set_wait_limit).
 constexpr long long kWaitPolls = 1ll << 23;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* err, int code)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* err, int code,
+                                          long long polls = kWaitPolls)
 {
-    for (long long it = 0; it < kWaitPolls; ++it) {
+    for (long long it = 0; it < polls; ++it) {
         if (mbar_try(bar, parity)) return true;
         if ((it & 255) == 255 && *abort) return false;
     }

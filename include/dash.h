@@ -230,6 +230,14 @@ int dash_backward(const dash_params* p, const void* Q, const void* K, const void
                   const void* dO, const float* kbar, const dash_route_out* route, float* dQ, float* dK, float* dV,
                   float* dqbar, void* workspace, size_t ws_bytes, void* stream);
 
+/* Diagnostic knob: the number of polls after which a bounded on-chip wait of the tensor-core
+ * Stage 2 prefill kernels gives up (the kernel then sets the workspace status word, drains its
+ * in-flight copies and MMAs, frees its tensor memory and returns; the output is not valid).  It
+ * applies to launches enqueued after the call; 0 makes the first wait give up at once (used by the
+ * tests of that failure path).  The default is 2^23.  Returns the previous limit, or -1 for a
+ * negative argument (nothing changed).  Not thread-safe with respect to concurrent launches. */
+long long dash_set_wait_limit(long long polls);
+
 /* Static text for a status code. */
 const char* dash_status_string(int status);
 

@@ -28,7 +28,7 @@ def test_header_symbols_exported():
     assert set(syms) == {"dash_workspace_size", "dash_route_capacity", "dash_prefill", "dash_prefill_stage",
                          "dash_summary_build", "dash_error_word_offset", "dash_decode_noalloc",
                          "dash_summary_append", "dash_decode", "dash_status_string", "dash_summary_build_paged",
-                         "dash_summary_append_paged", "dash_decode_paged", "dash_backward"}
+                         "dash_summary_append_paged", "dash_decode_paged", "dash_backward", "dash_set_wait_limit"}
     lib = D.load()
     for s in syms:
         assert hasattr(lib, s), s
@@ -145,3 +145,11 @@ def test_backward_arguments_rejected_before_launch():
     big = _p(seqlen=131072, h_q=32, h_kv=2, chunk=32, q_strides=(0, 32 * 128, 128), k_strides=(0, 256, 128),
              v_strides=(0, 256, 128), o_strides=(0, 32 * 128, 128))
     assert call(big, full, nbytes=1 << 50) == L.DASH_EUNSUPPORTED
+
+
+def test_wait_limit_knob_round_trips():
+    """The diagnostic poll limit: the previous value comes back, a negative one is refused."""
+    prev = L.dash_set_wait_limit(5)
+    assert prev == 1 << 23
+    assert L.dash_set_wait_limit(-1) == -1
+    assert L.dash_set_wait_limit(prev) == 5

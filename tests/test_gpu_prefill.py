@@ -339,3 +339,26 @@ def test_paired_tile_stage2_kernel_against_oracle(B, g):
     r = subprocess.run([sys.executable, "-c", _PAIR_CHILD, here, str(B), str(g)],
                        env=dict(os.environ, DASH_STAGE2="pair"), capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+
+
+def test_bounded_wait_timeout_sets_the_status_word_and_recovers():
+    """Failure path of the bounded on-chip waits, without a fault: with a poll limit of 0 the
+    tensor-core Stage 2 kernel's first wait gives up at once; the block sets the status word,
+    drains the copies and MMAs it has in flight, frees its tensor memory and returns.  The word
+    reads non-zero afterwards, and the next call with the default limit is clean and reproduces
+    the output bit for bit (the context stays usable)."""
+    from adaptive_sparse_hierarchical_b200 import _lib as L
+    x = inputs.planted(18, 1, 1200, 16, 2, 128, 64, dtype="bf16", chunk_frac=0.1, strength=2.0)
+    O, pf = run_prefill(x, chunk=64, alpha=1.5, gamma=8.0)
+    O_ref = O.clone()
+    prev = L.dash_set_wait_limit(0)
+    try:
+        pf.stage(2)
+        torch.cuda.synchronize()
+        assert pf.error_word() != 0
+    finally:
+        assert L.dash_set_wait_limit(prev) == 0
+    pf()   # Stage 0 of a full call clears the word
+    torch.cuda.synchronize()
+    assert pf.error_word() == 0
+    assert torch.equal(pf.O, O_ref)
