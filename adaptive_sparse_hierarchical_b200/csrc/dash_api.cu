@@ -108,7 +108,7 @@ long long route_cap(const dash_params* p)
     return tri_offset(p->seqlen, p->chunk);
 }
 
-struct PrefillLayout { size_t kbar, counts, idx, bias, err, planes, redo, perm, total; };
+struct PrefillLayout { size_t kbar, counts, idx, bias, err, knorm, planes, redo, perm, total; };
 PrefillLayout prefill_layout(const dash_params* p)
 {
     PrefillLayout L;
@@ -120,7 +120,8 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.idx = L.counts + up(bh * (size_t)p->seqlen * 4);
     L.bias = L.idx + up(bh * cap * 4);
     L.err = L.bias + up(bh * cap * 4);
-    L.planes = L.err + kAlign;
+    L.knorm = L.err + 16;   // the status word, then one float per (sequence, KV head)
+    L.planes = L.err + up(16 + bh * 4);
     L.redo = L.planes + up(bh * 3 * T * p->d_h * 2);
     L.perm = L.redo + up(bh * (size_t)p->seqlen);   // one flag per position block at most
     L.total = L.perm + up(bh * (size_t)p->seqlen * 4);
@@ -243,15 +244,19 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     // bf16: Stage 0 also writes the summaries as three exact bf16 planes for Stage 1's MMAs
     __nv_bfloat16* planes = p->dtype == DASH_BF16 ? reinterpret_cast<__nv_bfloat16*>(ws + L.planes) : nullptr;
     int* err = reinterpret_cast<int*>(ws + L.err);
+    float* knorm = reinterpret_cast<float*>(ws + L.knorm);
     if (stage == -1 || stage == DASH_STAGE0) {
-        // a prefill starts here: clear the status word of the bounded waits
-        if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return DASH_ELAUNCH;
-        rc = launch_status(launch_stage0(s, p->dtype, K, qbar, nullptr, kbar, s.T, nullptr, st, planes));
+        // a prefill starts here: clear the status word of the bounded waits and the per-(sequence,
+        // KV head) summary norms that Stage 0 raises
+        if (cudaMemsetAsync(err, 0, L.planes - L.err, st) != cudaSuccess) return DASH_ELAUNCH;
+        rc = launch_status(launch_stage0(s, p->dtype, K, qbar, nullptr, kbar, s.T, nullptr, st, planes,
+                                         planes ? knorm : nullptr));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE1) {
         unsigned char* redo = reinterpret_cast<unsigned char*>(ws + L.redo);
-        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, rt, redo, err, st));
+        rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, planes ? knorm : nullptr, rt, redo,
+                                                err, st));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE2)

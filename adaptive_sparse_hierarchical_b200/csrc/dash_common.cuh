@@ -153,15 +153,17 @@ int check_params(const dash_params* p);
 // planes (optional, bf16 [b][hkv][3][T][d]): each summary split exactly into hi + mid + lo.
 cudaError_t launch_stage0(const Shape& s, int dtype, const void* K, const float* qbar,
                           const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st,
-                          __nv_bfloat16* planes = nullptr);
+                          __nv_bfloat16* planes = nullptr, float* knorm = nullptr);
 cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const void* v_new,
                           const float* qbar, void* Kc, void* Vc, float* kbar, int kbar_T,
                           float* state, int* seqlens, cudaStream_t st);
 // Stage 1 for prefill: routes of every position.
 // redo: one byte per (sequence, KV head, position block) for the long-row kernel's overflow flags
+// knorm: per (sequence, KV head) the largest Euclidean norm of a summary (written by Stage 0
+// with the planes; the long-row kernel's hi-plane bound)
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const __nv_bfloat16* planes, const Routes& rt, unsigned char* redo, int* err,
-                                 cudaStream_t st);
+                                 const __nv_bfloat16* planes, const float* knorm, const Routes& rt,
+                                 unsigned char* redo, int* err, cudaStream_t st);
 // tcgen05 / TMEM variant of Stage 1 (bf16, d = 128, at most 512 complete chunks)
 bool route_tcgen05_supported(const Shape& s, int dtype);
 cudaError_t launch_route_prefill_tcgen05(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
@@ -172,8 +174,8 @@ size_t route_prefill_smem(const Shape& s, int* positions_per_block);
 // and writes nothing, and launch_route_prefill recomputes those blocks with the kernels above.
 bool route_long_supported(const Shape& s, int dtype);
 int route_long_positions(const Shape& s);
-cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
-                                      unsigned char* redo, int* err, cudaStream_t st);
+cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const float* knorm,
+                                      const Routes& rt, unsigned char* redo, int* err, cudaStream_t st);
 // Stage 2 for prefill.
 // perm: workspace of batch * h_kv * n ints (the tensor-core path's grouped position order)
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,

@@ -51,7 +51,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restrict__ K,
                                                      const float* __restrict__ qbar,
                                                      const int* __restrict__ len, float* kbar,
-                                                     int kbar_T, float* state, __nv_bfloat16* planes)
+                                                     int kbar_T, float* state, __nv_bfloat16* planes,
+                                                     float* knorm)
 {
     using L = KeyLanes<T, D>;
     __shared__ float wst[4][D + 2];
@@ -146,6 +147,20 @@ __global__ void __launch_bounds__(128) stage0_kernel(Shape s, const T* __restric
                 pl[2 * ps + e] = __float2bfloat16_rn(rem - __bfloat162float(mid));
             }
         }
+        if (knorm) {
+            // the largest Euclidean norm of a summary of this (sequence, KV head): non-negative
+            // floats order as their bit patterns, so an unsigned maximum of the bits
+            float ss = 0.f;
+            for (int e = 0; e < L::EPL; ++e) {
+                const float v = run.acc[e] * inv;
+                ss = fmaf(v, v, ss);
+            }
+            constexpr unsigned kGrp = L::LPK >= 32 ? 0xffffffffu : ((1u << L::LPK) - 1u);
+#pragma unroll
+            for (int o = L::LPK / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(kGrp, ss, o);
+            if (sub == 0)
+                atomicMax(reinterpret_cast<unsigned*>(knorm) + (b * s.hkv + r), __float_as_uint(sqrtf(ss)));
+        }
     } else {
         float* st = state + ((long long)b * s.hkv + r) * (D + 2);
         for (int e = 0; e < L::EPL; ++e) st[sub * L::EPL + e] = run.acc[e];
@@ -203,15 +218,15 @@ __global__ void append_kernel(Shape s, const T* __restrict__ k_new, const T* __r
 
 template <typename T>
 cudaError_t stage0_t(const Shape& s, const void* K, const float* qbar, const int* len, float* kbar,
-                     int kbar_T, float* state, __nv_bfloat16* planes, cudaStream_t st)
+                     int kbar_T, float* state, __nv_bfloat16* planes, float* knorm, cudaStream_t st)
 {
     const long long items = (long long)s.batch * s.hkv * (kbar_T + 1);
     const unsigned grid = (unsigned)items;
     if (grid == 0) return cudaSuccess;
     if (s.d == 128)
-        stage0_kernel<T, 128><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes);
+        stage0_kernel<T, 128><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes, knorm);
     else
-        stage0_kernel<T, 64><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes);
+        stage0_kernel<T, 64><<<grid, 128, 0, st>>>(s, (const T*)K, qbar, len, kbar, kbar_T, state, planes, knorm);
     return cudaGetLastError();
 }
 
@@ -233,10 +248,10 @@ cudaError_t append_t(const Shape& s, const void* kn, const void* vn, const float
 
 cudaError_t launch_stage0(const Shape& s, int dtype, const void* K, const float* qbar,
                           const int* len, float* kbar, int kbar_T, float* state, cudaStream_t st,
-                          __nv_bfloat16* planes)
+                          __nv_bfloat16* planes, float* knorm)
 {
-    return dtype == DASH_BF16 ? stage0_t<__nv_bfloat16>(s, K, qbar, len, kbar, kbar_T, state, planes, st)
-                              : stage0_t<float>(s, K, qbar, len, kbar, kbar_T, state, planes, st);
+    return dtype == DASH_BF16 ? stage0_t<__nv_bfloat16>(s, K, qbar, len, kbar, kbar_T, state, planes, knorm, st)
+                              : stage0_t<float>(s, K, qbar, len, kbar, kbar_T, state, planes, knorm, st);
 }
 
 cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const void* v_new,

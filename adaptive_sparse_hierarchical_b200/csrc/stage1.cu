@@ -10,10 +10,11 @@
 // group share one sparse support.
 //
 // Threshold tau: the mass f(t) = sum_c [x_c - t]_+^{1/(alpha-1)} is continuous and strictly
-// decreasing where positive; f(max x - 1) >= 1 and f(max x - nvis^{-(alpha-1)}) <= 1.  A fixed
-// number of bisection steps narrows that bracket to about 1e-6 of its width, then Newton steps
-// from the left end (the tangent of a convex decreasing function stays below it, so the steps
-// never pass the root) finish to float precision.
+// decreasing where positive; f(max x - 1) >= 1 and f(max x - nvis^{-(alpha-1)}) <= 1.  Newton
+// steps on f^(alpha-1) from the left end (the tangent of a convex decreasing function stays
+// below it, so the steps never pass the root) finish to float precision; for alpha = 2 and 1.5
+// the closed-form root on the current support ends the solve once the support is found
+// (entmax.cuh, ent_step).
 #include <cstdlib>
 
 #include "dash_common.cuh"
@@ -211,7 +212,7 @@ __device__ float warp_threshold_compact(const float (&xr)[NPL], int nv, float al
     __syncwarp();
     const float t = entmax_threshold(
         [&](auto fn) { for (int c = lane; c < m; c += 32) fn(scratch[c]); },
-        [](float& a, float& b) { a = warp_sum(a); b = warp_sum(b); }, mx, nv, alpha);
+        [](EntSums& S) { ent_warp_reduce(S); }, mx, nv, alpha);
     __syncwarp();   // scratch is reused by the warp's next row
     return t;
 }
@@ -229,7 +230,7 @@ __device__ float warp_threshold_reg(const float (&xr)[NPL], int nv, float alpha)
 #pragma unroll
             for (int k = 0; k < NPL; ++k) fn(xr[k]);
         },
-        [](float& a, float& b) { a = warp_sum(a); b = warp_sum(b); }, mx, nv, alpha);
+        [](EntSums& S) { ent_warp_reduce(S); }, mx, nv, alpha);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -543,7 +544,7 @@ cudaError_t route_tc_d(const Shape& s, const void* Q, const __nv_bfloat16* plane
 __global__ void __launch_bounds__(256) dec_tau_block_kernel(Shape s, int kbar_T, const int* __restrict__ seqlens,
                                                             float* X)
 {
-    __shared__ float red[2][8][2];
+    __shared__ float4 red[2][8];
     const int h = blockIdx.x, br = blockIdx.y, b = br / s.hkv;
     const int nv = min((seqlens[b] - 1) / s.B, kbar_T);
     if (nv <= 0) return;
@@ -557,14 +558,15 @@ __global__ void __launch_bounds__(256) dec_tau_block_kernel(Shape s, int kbar_T,
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int phase = 0;
-    auto bsum2 = [&](float& a, float& bb) {
-        a = warp_sum(a);
-        bb = warp_sum(bb);
-        if (lane == 0) { red[phase][warp][0] = a; red[phase][warp][1] = bb; }
+    auto bsum = [&](EntSums& S) {
+        ent_warp_reduce(S);
+        if (lane == 0) red[phase][warp] = make_float4(S.f, S.fd, S.n, S.um);
         __syncthreads();
-        a = 0.f;
-        bb = 0.f;
-        for (int w = 0; w < 8; ++w) { a += red[phase][w][0]; bb += red[phase][w][1]; }
+        S = ent_zero();
+        for (int w = 0; w < 8; ++w) {
+            const float4 v = red[phase][w];
+            ent_merge(S, EntSums{v.x, v.y, v.z, v.w});
+        }
         phase ^= 1;   // alternate buffers: the next reduction cannot overwrite values still being read
     };
     float mx = xr[0];
@@ -572,10 +574,10 @@ __global__ void __launch_bounds__(256) dec_tau_block_kernel(Shape s, int kbar_T,
     for (int k = 1; k < NPL; ++k) mx = fmaxf(mx, xr[k]);
     {
         const float m2 = warp_max(mx);
-        if (lane == 0) red[phase][warp][0] = m2;
+        if (lane == 0) red[phase][warp].x = m2;
         __syncthreads();
         mx = -INFINITY;
-        for (int w = 0; w < 8; ++w) mx = fmaxf(mx, red[phase][w][0]);
+        for (int w = 0; w < 8; ++w) mx = fmaxf(mx, red[phase][w].x);
         phase ^= 1;
     }
     const float tau = entmax_threshold(
@@ -583,7 +585,7 @@ __global__ void __launch_bounds__(256) dec_tau_block_kernel(Shape s, int kbar_T,
 #pragma unroll
             for (int k = 0; k < NPL; ++k) fn(xr[k]);
         },
-        bsum2, mx, nv, s.alpha);
+        bsum, mx, nv, s.alpha);
     const float p = 1.f / (s.alpha - 1.f);
     const int mode = ent_mode(s.alpha);
 #pragma unroll
@@ -704,8 +706,8 @@ static bool long_route_off()
 }
 
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
-                                 const __nv_bfloat16* planes, const Routes& rt, unsigned char* redo, int* err,
-                                 cudaStream_t st)
+                                 const __nv_bfloat16* planes, const float* knorm, const Routes& rt,
+                                 unsigned char* redo, int* err, cudaStream_t st)
 {
     if (planes && route_tcgen05_supported(s, dtype) && !legacy_stage2())
         return launch_route_prefill_tcgen05(s, Q, planes, rt, err, st);
@@ -713,8 +715,8 @@ cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const
     // the position blocks whose candidate lists overflowed
     const unsigned char* mask = nullptr;
     int mask_p = 1;
-    if (planes && redo && route_long_supported(s, dtype) && !legacy_stage2() && !long_route_off()) {
-        cudaError_t e = launch_route_prefill_long(s, Q, planes, rt, redo, err, st);
+    if (planes && knorm && redo && route_long_supported(s, dtype) && !legacy_stage2() && !long_route_off()) {
+        cudaError_t e = launch_route_prefill_long(s, Q, planes, knorm, rt, redo, err, st);
         if (e != cudaSuccess) return e;
         mask = redo;
         mask_p = route_long_positions(s);

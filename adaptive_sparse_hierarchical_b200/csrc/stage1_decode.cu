@@ -17,6 +17,7 @@
 #include <type_traits>
 
 #include "dash_common.cuh"
+#include "entmax.cuh"
 #include "stage2_mma.cuh"
 
 namespace cg = cooperative_groups;
@@ -28,15 +29,6 @@ constexpr int kRanks = 4;        // blocks per cluster (small clusters: all of t
 constexpr int kThr = 512;        // 16 warps: warp h owns head h in the per-head phases
 constexpr int kMaxG = 16;
 constexpr int kSlots = 16 / kRanks;   // heads each block solves (head h: block h % kRanks, slot h / kRanks)
-
-__device__ __forceinline__ float dpow(float u, float p, int mode)
-{
-    return mode == 1 ? u : mode == 2 ? u * u : exp2f(p * __log2f(u));
-}
-__device__ __forceinline__ float dpow1(float u, float p, int mode)
-{
-    return mode == 1 ? 1.f : mode == 2 ? u : exp2f((p - 1.f) * __log2f(u));
-}
 
 struct Cross {                   // per block, read by the other blocks of the cluster
     float mx[kMaxG];             // slice maximum of each head's logits
@@ -89,7 +81,7 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
     __shared__ float tau[kMaxG], gmax[kMaxG];
     __shared__ int wsum[kThr / 32 + 1];
     __shared__ float fsum[kThr / 32];
-    __shared__ float npart[2][kSlots * kRanks][2];   // Newton partial sums [step parity][slot, source]
+    __shared__ float4 npart[2][kSlots * kRanks];      // solve partial sums [step parity][slot, source]
     __shared__ int ndone[kSlots];
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -202,7 +194,7 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
     cl.sync();
     // ---- thresholds: block `rank` solves heads h = rank + kRanks slot on the pushed entries; warp
     // (slot, k) sums over source block k's entries, the partials are added in k order, and every
-    // thread of the slot takes the same Newton step on f^(alpha-1) from max - 1 ---------------
+    // thread of the slot takes the same step of the solve (entmax.cuh, ent_step) from max - 1 ---
     static_assert(kSlots * kRanks == kThr / 32, "one warp per (head slot, source block)");
     {
         const int slot = warp / kRanks, k = warp % kRanks, h = rank + kRanks * slot;
@@ -221,30 +213,17 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
             for (int j = 0; j < kSlots; ++j) all = all && ndone[j];
             if (all) break;
             const int ph = it & 1;
-            float f = 0.f, fd = 0.f;
-            for (int j = lane; j < nk; j += 32) {
-                const float u = gl[j] - t;
-                if (u > 0.f) { f += dpow(u, p, mode); fd += dpow1(u, p, mode); }
-            }
-            f = warp_sum(f);
-            fd = warp_sum(fd);
-            if (lane == 0) { npart[ph][slot * kRanks + k][0] = f; npart[ph][slot * kRanks + k][1] = fd; }
+            EntSums S = ent_zero();
+            for (int j = lane; j < nk; j += 32) ent_add(S, gl[j] - t, p, mode);
+            ent_warp_reduce(S);
+            if (lane == 0) npart[ph][slot * kRanks + k] = make_float4(S.f, S.fd, S.n, S.um);
             __syncthreads();   // a parity slot is rewritten two steps later, after the next barrier
-            float F = 0.f, FD = 0.f;
-            for (int kk = 0; kk < kRanks; ++kk) { F += npart[ph][slot * kRanks + kk][0]; FD += npart[ph][slot * kRanks + kk][1]; }
-            if (!dn) {
-                if (F >= 1.f) lo = t; else hi = t;
-                float tn = 0.5f * (lo + hi);
-                if (FD > 0.f && F > 0.f) {
-                    const float gg = mode == 2 ? sqrtf(F) : mode == 1 ? F : exp2f((s.alpha - 1.f) * __log2f(F));
-                    tn = t + (gg - 1.f) * F / (gg * FD);
-                }
-                if (fabsf(tn - t) <= 2e-7f * fmaxf(1.f, fabsf(t)) || fabsf(F - 1.f) <= 1e-6f) { t = tn; dn = true; }
-                else {
-                    if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
-                    t = tn;
-                }
+            S = ent_zero();
+            for (int kk = 0; kk < kRanks; ++kk) {
+                const float4 v = npart[ph][slot * kRanks + kk];
+                ent_merge(S, EntSums{v.x, v.y, v.z, v.w});
             }
+            if (!dn) dn = ent_step(S, t, lo, hi, s.alpha, mode);
             // every thread of a slot holds the same state; the slot's first warp reports it
             if (k == 0 && lane == 0) ndone[slot] = dn;
             __syncthreads();
@@ -263,7 +242,7 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
         float a = 0.f;
         for (int h = 0; h < G; ++h) {
             const float u = xsm[h * per + c] - tau[h];
-            a += u > 0.f ? dpow(u, p, mode) : 0.f;
+            a += u > 0.f ? ent_pow(u, p, mode) : 0.f;
         }
         const float w = a * inv_g;
         xsm[c] = w;   // row 0 is only read by this thread from here on

@@ -25,6 +25,7 @@
 #include <cudaTypedefs.h>
 
 #include "dash_common.cuh"
+#include "entmax.cuh"
 #include "tc_ptx.cuh"
 
 namespace dash {
@@ -38,17 +39,8 @@ constexpr int kStage = 3 * 2 * kPlaneHalf;      // three planes x two d-halves =
 constexpr int kOffQ1 = 0, kOffRing = kQB, kOffW = kOffRing + 2 * kStage;
 constexpr int kCand = 48;   // candidate list length per row and warp: 16 x 32 x 48 floats fill the ring
 static_assert(16 * 32 * kCand * 4 <= 2 * kStage && kCand % 4 == 0, "candidate lists must fit the ring");
-constexpr int kMisc = 128 + 3 * 4 * kR * 8;     // barriers, TMEM slot, abort flag, reduction slots
+constexpr int kMisc = 128 + 3 * 4 * kR * 16;    // barriers, TMEM slot, abort flag, reduction slots
 constexpr uint32_t kIdescX = tc::idesc_bf16(128, 64, false, false);
-
-__device__ __forceinline__ float pw(float u, float p, int mode)
-{
-    return mode == 1 ? u : mode == 2 ? u * u : exp2f(p * __log2f(u));
-}
-__device__ __forceinline__ float dpw(float u, float p, int mode)
-{
-    return mode == 1 ? 1.f : mode == 2 ? u : exp2f((p - 1.f) * __log2f(u));
-}
 
 // Sum over the g neighbouring lanes of a position of 32 values, reduce-scattered: afterwards
 // lane (h = lane % g) holds the sums of the 32/g columns starting at *off.
@@ -86,7 +78,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
     constexpr int P = kR / G;
     float* wbuf = reinterpret_cast<float*>(sm + kOffW);            // [P][Tw] group sums of the head weights
     char* misc = sm + kOffW + P * Tw * 4;
-    float2* red = reinterpret_cast<float2*>(misc + 128);          // [3][4][kR] partial (f, f') / max
+    float4* red = reinterpret_cast<float4*>(misc + 128);          // [3][4][kR] partial solve sums / max
     const uint32_t bar0 = tc::smem_addr(misc);
     const uint32_t q_full = bar0, x_ready = bar0 + 8;
     const uint32_t full0 = bar0 + 16, empty0 = bar0 + 32;          // [2] each
@@ -258,58 +250,45 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
             const bool listed = __all_sync(0xffffffffu, m <= kCand);
             const int m4 = (m + 3) >> 2;
             for (int k = m; k < 4 * m4 && k < kCand; ++k) cl[k * 32] = -INFINITY;
-            // Newton on g(t) = f(t)^(alpha-1) from t = max - 1 (see stage1.cu); every lane keeps
-            // stepping until the whole warp has converged
+            // the solve from t = max - 1 (entmax.cuh, ent_step: Newton on f^(alpha-1), closed-form
+            // finish for alpha = 2 and 1.5); every lane keeps stepping until the whole warp is done
             float hi = nv > 0 ? mx - exp2f(-(s.alpha - 1.f) * __log2f((float)nv)) : 0.f;
             float t = lo;
             bool done = nv == 0;
             for (int it = 0; it < 32 && !__all_sync(0xffffffffu, done); ++it) {
-                float f = 0.f, fd = 0.f;
+                EntSums S = ent_zero();
                 if (listed && mode == 2) {
 #pragma unroll 2
                     for (int k = 0; k < m4; ++k) {
-                        const float u0 = fmaxf(cl[(4 * k) * 32] - t, 0.f), u1 = fmaxf(cl[(4 * k + 1) * 32] - t, 0.f);
-                        const float u2 = fmaxf(cl[(4 * k + 2) * 32] - t, 0.f), u3 = fmaxf(cl[(4 * k + 3) * 32] - t, 0.f);
-                        f += u0 * u0 + u1 * u1 + u2 * u2 + u3 * u3;
-                        fd += (u0 + u1) + (u2 + u3);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float u = cl[(4 * k + j) * 32] - t;
+                            const float up = fmaxf(u, 0.f);
+                            S.f = fmaf(up, up, S.f);
+                            S.fd += up;
+                            S.n += u > 0.f ? 1.f : 0.f;
+                            S.um = fminf(S.um, u > 0.f ? u : INFINITY);
+                        }
                     }
                 } else if (listed) {
-                    for (int k = 0; k < 4 * m4; ++k) {
-                        const float u = cl[k * 32] - t;
-                        if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
-                    }
+                    for (int k = 0; k < 4 * m4; ++k) ent_add(S, cl[k * 32] - t, p, mode);
                 } else {
                     for (int pc = cq; pc < npieces; pc += 4) {
                         float v[32];
                         load_piece(pc, v);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float u = v[e] - t;
-                            if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
-                        }
+                        for (int e = 0; e < 32; ++e) ent_add(S, v[e] - t, p, mode);
                     }
                 }
-                float2* slot = red + (it & 1) * 4 * kR;
-                slot[cq * kR + row] = make_float2(f, fd);
+                float4* slot = red + (it & 1) * 4 * kR;
+                slot[cq * kR + row] = make_float4(S.f, S.fd, S.n, S.um);
                 group_sync();
-                const float2 r0 = slot[row], r1 = slot[kR + row], r2 = slot[2 * kR + row], r3 = slot[3 * kR + row];
-                f = (r0.x + r1.x) + (r2.x + r3.x);
-                fd = (r0.y + r1.y) + (r2.y + r3.y);
-                if (!done) {
-                    // g = f^(alpha-1) has g' = -(alpha-1) f^(alpha-2) p sum u^(p-1) = -f^(alpha-2) fd,
-                    // so the Newton step (g - 1) / -g' is (g - 1) f / (g fd)
-                    if (f >= 1.f) lo = t; else hi = t;
-                    float tn = 0.5f * (lo + hi);
-                    if (fd > 0.f && f > 0.f) {
-                        const float gg = mode == 2 ? sqrtf(f) : mode == 1 ? f : exp2f((s.alpha - 1.f) * __log2f(f));
-                        tn = t + (gg - 1.f) * f / (gg * fd);
-                    }
-                    if (fabsf(tn - t) <= 2e-7f * fmaxf(1.f, fabsf(t)) || fabsf(f - 1.f) <= 1e-6f) { t = tn; done = true; }
-                    else {
-                        if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
-                        t = tn;
-                    }
-                }
+                const float4 r0 = slot[row], r1 = slot[kR + row], r2 = slot[2 * kR + row], r3 = slot[3 * kR + row];
+                S.f = (r0.x + r1.x) + (r2.x + r3.x);
+                S.fd = (r0.y + r1.y) + (r2.y + r3.y);
+                S.n = (r0.z + r1.z) + (r2.z + r3.z);
+                S.um = fminf(fminf(r0.w, r1.w), fminf(r2.w, r3.w));
+                if (!done) done = ent_step(S, t, lo, hi, s.alpha, mode);
             }
             // head weights of this warp's pieces, summed over the position's g lanes, into wbuf
             for (int pc = cq; pc < npieces; pc += 4) {
@@ -318,7 +297,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const float u = v[e] - t;
-                    v[e] = u > 0.f ? pw(u, p, mode) : 0.f;
+                    v[e] = u > 0.f ? ent_pow(u, p, mode) : 0.f;
                 }
                 int off;
                 group_reduce_scatter<G>(v, lane, &off);

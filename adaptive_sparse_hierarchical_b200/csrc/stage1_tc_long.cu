@@ -7,15 +7,19 @@
 //   bias_c = (log w_c - mean_R log w)/sigma.
 //
 // One block = 128 query rows = (128/g positions) x (g heads) of one (sequence, KV head).  The
-// logits X = Q k̄^T stream through two 256-column halves of TMEM in blocks of 256 chunks
-// (three exact bf16 planes of k̄, TMA-staged), three times: pass 0 takes each row's maximum,
-// pass 1 copies the entries above (max - 1) -- the only ones the support can reach -- into
-// per-thread lists in shared memory, Newton on f^(alpha-1) then runs on the lists, and pass 2
-// forms the head weights, sums them over the g heads of each position and writes the block's
-// routed chunks (ascending) with log w; the bias is fixed up with the mean once all blocks are
-// written.  The MMAs of one block overlap the processing of the previous one.  A block whose
-// lists overflow flags its tile in `redo` and writes nothing; the per-shape routing kernels
-// then recompute the flagged tiles.
+// logits X = Q k̄^T stream through two 192-column halves of TMEM in blocks of 192 chunks,
+// TMA-staged bf16 planes of k̄ (hi + mid + lo = k̄ exactly).  Pass 0 takes each row's maximum
+// from the hi plane alone: |x - x_hi| <= xs 2^-8 |q| |k̄_c| (bf16 rounding of k̄, plus a margin
+// for the fp32 accumulation), so with the largest |k̄_c| of the (sequence, KV head) from Stage 0
+// that maximum less the bound is a lower bound on the exact one.  Pass 1 (all three planes)
+// copies the entries above (that bound - 1) -- a superset of the only ones the support can
+// reach, tau >= max - 1 -- with their chunk indices into per-thread lists in shared memory; the
+// threshold is solved on the lists, and the head weights, their sums over the g heads of each
+// position and the routed chunks (ascending, with log w) all come from the lists, window by
+// window; the bias is fixed up with the mean once every window is written.  The MMAs of one
+// block overlap the processing of the previous one.  A block whose lists overflow flags its
+// tile in `redo` and writes nothing; the per-shape routing kernels then recompute the flagged
+// tiles.
 // Roles (18 warps): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, warps 2-17 four
 // warps per TMEM lane quarter (32 rows), each reading every fourth 32-column piece of a block.
 // Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
@@ -23,50 +27,48 @@
 #include <cudaTypedefs.h>
 
 #include "dash_common.cuh"
+#include "entmax.cuh"
 #include "tc_ptx.cuh"
 
 namespace dash {
 
 namespace {
 
-constexpr int kR = 128, kCT = 64, kDd = 128;
-constexpr int kPlaneHalf = kCT * 64 * 2;        // [64 chunks][64 d] bf16 = 8 KB
-constexpr int kStage = 2 * kPlaneHalf;          // one plane of a tile, two d-halves = 16 KB
-constexpr int kNS = 4;                          // ring stages
-constexpr int kBW = 192;                        // chunks per block = columns of a TMEM half
-constexpr int kTPB = kBW / kCT;                 // 64-chunk tiles per block
+constexpr int kR = 128, kDd = 128;
+constexpr int kBW = 192;                        // chunks per block = columns of a TMEM half = MMA N
+constexpr int kStage = kBW * 64 * 2;            // ring stage: [192 chunks][64 d] bf16 of one plane = 24 KB
+constexpr int kNS = 2;                          // ring stages
 constexpr int kPieces = kBW / 32;               // 32-column pieces per block
-// TMEM: X halves at columns [0, 192) and [192, 384); the Q tile (the MMAs' A operand, 128 rows x
-// 128 bf16, two per 32-bit column) at [384, 448)
-constexpr int kColQ = 2 * kBW;
+// TMEM: X halves at columns [0, 192) and [256, 448); the Q tile (the MMAs' A operand, 128 rows x
+// 128 bf16, two per 32-bit column) at [448, 512)
+constexpr int kHalfCol = 256;
+constexpr int kColQ = 448;
 constexpr int kOffRing = 0, kOffLists = kOffRing + kNS * kStage;
-constexpr uint32_t kIdescX = tc::idesc_bf16(128, 64, false, false);
+// one MMA per (block, plane, 16-wide k step): M = 128 rows, N = 192 chunks.  Narrow N = 64 MMAs
+// accumulating into one tile form a dependent chain that runs at a fraction of the tensor rate.
+constexpr uint32_t kIdescX = tc::idesc_bf16(128, kBW, false, false);
 // after every pass but the first the workers post whether another pass over the blocks follows
 // (kPlanGo) or not (kPlanStop); at most kMaxExtract extraction passes per set of rows in play
 constexpr int kPlanStop = 0, kPlanGo = 1;
 constexpr int kMaxExtract = 2;
 
-// candidate list entries per (worker warp, lane); the lists also hold the weights buffer
-// [P][kBW] of the emission pass (the lists are dead by then)
-constexpr int kCap = 72;
-constexpr int kOffMisc = kOffLists + 16 * 32 * kCap * 4;
-// misc: barriers (kBarBytes), tmem slot / abort / overflow / plan (16 B), red [3][4][kR] float2
-// (12 KB), per position: running log-sum, count, list base (3 x 32 words)
+// candidate list entries per (worker warp, lane): a logit (fp32) and its chunk index (16 bits);
+// the emission's head-weight buffer [kR rows][kWin chunks] reuses the plane ring (idle by then)
+constexpr int kWin = 96;
+constexpr int kCap = 52;
+constexpr int kOffIdx = kOffLists + 16 * 32 * kCap * 4;
+constexpr int kOffMisc = kOffIdx + 16 * 32 * kCap * 2;
+// misc: barriers (kBarBytes), tmem slot / abort / overflow / plan (16 B), red [2][4][kR] float4
+// (16 KB), per position: running log-sum, count, list base (3 x 32 words), per row |q| (kR)
 constexpr int kBarBytes = 8 * (1 + 2 * kNS + 2 + 2 + 2);   // q_full, full/empty ring, x_ready/x_free, drain, dec
 constexpr int kMiscBase = (kBarBytes + 15) / 16 * 16;
-constexpr int kMiscBytes = kMiscBase + 16 + 3 * 4 * kR * 8 + 3 * 32 * 4;
+constexpr int kMiscBytes = kMiscBase + 16 + 2 * 4 * kR * 16 + 3 * 32 * 4 + kR * 4;
 constexpr size_t kLongSmem = 1024 + kOffMisc + kMiscBytes;
 static_assert(kLongSmem <= 227 * 1024, "shared memory of the long-row routing kernel");
-static_assert((kR / 4) * kBW * 4 <= 16 * 32 * kCap * 4, "weights buffer inside the lists");
-
-__device__ __forceinline__ float pw(float u, float p, int mode)
-{
-    return mode == 1 ? u : mode == 2 ? u * u : exp2f(p * __log2f(u));
-}
-__device__ __forceinline__ float dpw(float u, float p, int mode)
-{
-    return mode == 1 ? 1.f : mode == 2 ? u : exp2f((p - 1.f) * __log2f(u));
-}
+static_assert(kR * kWin * 4 <= kNS * kStage, "head-weight buffer inside the plane ring");
+static_assert(kCap % 4 == 0, "lists are padded to a multiple of four entries");
+// |x - x_hi| <= xs (2^-8 |q| |k̄_c|  +  fp32 accumulation error): coefficient of xs |q| max|k̄_c|
+constexpr float kHiPlaneBound = 0.00390625f + 0.0009765625f;
 
 // Lower bound on the root of f_S(t) = sum_{x in S} [x - t]_+^p = 1 over a subset S of a row's
 // logits: this thread's list (entry k at cl[32 k], m entries) and three more values (the other
@@ -82,13 +84,13 @@ __device__ __noinline__ float subset_bound(const float* cl, int m, float om0, fl
         float f = 0.f, fd = 0.f;
         for (int k = 0; k < m; ++k) {
             const float u = cl[32 * k] - t;
-            if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
+            if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
         }
         const float om[3] = {om0, om1, om2};
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
             const float u = om[j] - t;
-            if (u > 0.f) { f += pw(u, p, mode); fd += dpw(u, p, mode); }
+            if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
         }
         if (f < 1.f) return it == 0 ? -INFINITY : t;
         if (!(fd > 0.f)) break;
@@ -128,15 +130,16 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane, i
 template <int G>
 __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid_constant__ CUtensorMap tmP,
                                                                     const __nv_bfloat16* __restrict__ Q,
-                                                                    Shape s, Routes rt, unsigned char* redo,
-                                                                    int* err)
+                                                                    const float* __restrict__ knorm, Shape s,
+                                                                    Routes rt, unsigned char* redo, int* err)
 {
     extern __shared__ char smem_raw[];
     char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = tc::smem_addr(sm);
     constexpr int P = kR / G, CAP = kCap;
     float* lists = reinterpret_cast<float*>(sm + kOffLists);            // [16 warps][CAP][32 lanes]
-    float* wbuf = lists;                                                // [P][kBW] group sums of one block
+    unsigned short* lidx = reinterpret_cast<unsigned short*>(sm + kOffIdx);   // chunk index of each entry
+    float* wbuf = reinterpret_cast<float*>(sm + kOffRing);              // [kR][kWin] head weights of a window
     char* misc = sm + kOffMisc;
     const uint32_t bar0 = tc::smem_addr(misc);
     const uint32_t q_full = bar0, full0 = bar0 + 8, empty0 = full0 + 8 * kNS;   // ring [kNS] each
@@ -147,9 +150,10 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
     volatile int* abort = reinterpret_cast<volatile int*>(misc + kMiscBase + 4);
     int* overflow = reinterpret_cast<int*>(misc + kMiscBase + 8);
     volatile int* plan_word = reinterpret_cast<volatile int*>(misc + kMiscBase + 12);
-    float2* red = reinterpret_cast<float2*>(misc + kMiscBase + 16);                  // [3][4][kR]
-    float* pslog = reinterpret_cast<float*>(misc + kMiscBase + 16 + 3 * 4 * kR * 8);  // [P] log-sum so far
+    float4* red = reinterpret_cast<float4*>(misc + kMiscBase + 16);                  // [2][4][kR]
+    float* pslog = reinterpret_cast<float*>(misc + kMiscBase + 16 + 2 * 4 * kR * 16);  // [P] log-sum so far
     int* pcnt = reinterpret_cast<int*>(pslog + 32);                        // [P] entries so far
+    float* qnorm = pslog + 3 * 32;                                         // [kR] |q| of each row
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntile128 = (s.n + P - 1) / P;
@@ -172,8 +176,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                 if (i0 + k / rt.words < s.n) bm[(long long)i0 * rt.words + k] = 0u;
         return;
     }
-    const int ntiles = (nvmax + kCT - 1) / kCT;
-    const int nbk = (ntiles + kTPB - 1) / kTPB;   // 256-chunk blocks
+    const int nbk = (nvmax + kBW - 1) / kBW;   // 192-chunk blocks
 
     if (tid == 0) {
         tc::mbar_init(q_full, 128);   // the four warps that write the Q rows into TMEM
@@ -208,18 +211,19 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
             int last[kNS];
 #pragma unroll
             for (int j = 0; j < kNS; ++j) last[j] = -1;
-            int gs = 0;   // ring stage counter: one stage per (tile, plane)
+            int gs = 0;   // ring stage counter: one stage per (block, plane, d-half)
             bool pok = true;
             for (int k = 0; pok; ++k) {
-                for (int t = 0; pok && t < ntiles; ++t) {
-                    for (int pl = 0; pl < 3; ++pl, ++gs) {
+                const int npl = k == 0 ? 1 : 3;   // the row-maximum pass reads the hi plane alone
+                for (int kb = 0; pok && kb < nbk; ++kb) {
+                    for (int j = 0; j < 2 * npl; ++j, ++gs) {
                         const int st = gs % kNS;
                         if (gs >= kNS && !tc::mbar_wait(empty0 + 8 * st, ((gs / kNS) - 1) & 1, abort, err, 31)) { pok = false; break; }
                         last[st] = gs;
                         const uint32_t dst = base + kOffRing + st * kStage, fb = full0 + 8 * st;
                         tc::mbar_expect_tx(fb, kStage);
-                        tc::tma_load_4d(dst, &tmP, fb, 0, t * kCT, br * 3 + pl, 0);
-                        tc::tma_load_4d(dst + kPlaneHalf, &tmP, fb, 64, t * kCT, br * 3 + pl, 0);
+                        // chunks past T read as zeros (their columns are never used)
+                        tc::tma_load_4d(dst, &tmP, fb, 64 * (j & 1), kb * kBW, br * 3 + (j >> 1), 0);
                     }
                 }
                 if (!pok || k == 0) continue;
@@ -241,24 +245,23 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
             bool ok = tc::mbar_wait(q_full, 0, abort, err, 32);
             int gs = 0, u = 0;
             for (int k = 0; ok; ++k) {
+                const int npl = k == 0 ? 1 : 3;
                 for (int kb = 0; ok && kb < nbk; ++kb, ++u) {
                     const int hlf = u & 1;
                     // the half's previous use (u - 2) has been read by every worker
                     if (u >= 2 && !tc::mbar_wait(x_free0 + 8 * hlf, ((u >> 1) - 1) & 1, abort, err, 33)) { ok = false; break; }
-                    for (int t = kb * kTPB; ok && t < min(ntiles, (kb + 1) * kTPB); ++t) {
-                        const uint32_t xd = tmem + hlf * kBW + (t - kb * kTPB) * kCT;
-                        for (int pl = 0; pl < 3; ++pl, ++gs) {
-                            const int st = gs % kNS;
-                            if (!tc::mbar_wait(full0 + 8 * st, (gs / kNS) & 1, abort, err, 34)) { ok = false; break; }
-                            tc::fence_after_sync();
-                            const uint64_t dp = dP0 + (uint64_t)((st * kStage) >> 4);
+                    const uint32_t xd = tmem + hlf * kHalfCol;
+                    for (int j = 0; j < 2 * npl; ++j, ++gs) {
+                        // stage j: plane j / 2, d-half j % 2 (k steps 4 (j % 2) .. + 3)
+                        const int st = gs % kNS;
+                        if (!tc::mbar_wait(full0 + 8 * st, (gs / kNS) & 1, abort, err, 34)) { ok = false; break; }
+                        tc::fence_after_sync();
+                        const uint64_t dp = dP0 + (uint64_t)((st * kStage) >> 4);
 #pragma unroll
-                            for (int kk = 0; kk < kDd / 16; ++kk)
-                                tc::mma_f16_ts(xd, tmem + kColQ + kk * 8,
-                                               dp + (uint64_t)(((kk >> 2) * kPlaneHalf + (kk & 3) * 32) >> 4),
-                                               kIdescX, (pl > 0 || kk > 0) ? 1u : 0u);
-                            tc::mma_commit(empty0 + 8 * st);
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_f16_ts(xd, tmem + kColQ + (4 * (j & 1) + kk) * 8, dp + (uint64_t)((kk * 32) >> 4),
+                                           kIdescX, (j > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_commit(empty0 + 8 * st);
                     }
                     if (ok) tc::mma_commit(x_ready0 + 8 * hlf);
                 }
@@ -304,31 +307,45 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
         // its idle partner's region (capacity 2 CAP).
         if (cq == 0) {
             // row (position i0 + row / g, head r g + row % g) of the Q tile into this lane of TMEM
-            // columns [kColQ, kColQ + 64): the row's bf16 pairs are already the 32-bit columns
+            // columns [kColQ, kColQ + 64): the row's bf16 pairs are already the 32-bit columns;
+            // its Euclidean norm for the hi-plane bound
             uint4 qw[16];
             const __nv_bfloat16* qrow = Q + (long long)b * s.qs[0] + (long long)i * s.qs[1] + (long long)(r * G + row % G) * s.qs[2];
 #pragma unroll
             for (int k = 0; k < 16; ++k)
                 qw[k] = i < s.n ? __ldg(reinterpret_cast<const uint4*>(qrow) + k) : make_uint4(0u, 0u, 0u, 0u);
+            float qq = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const uint32_t w4[4] = {qw[k].x, qw[k].y, qw[k].z, qw[k].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float lo16 = __uint_as_float(w4[j] << 16), hi16 = __uint_as_float(w4[j] & 0xffff0000u);
+                    qq = fmaf(lo16, lo16, fmaf(hi16, hi16, qq));
+                }
+            }
+            qnorm[row] = sqrtf(qq);
 #pragma unroll
             for (int k = 0; k < 4; ++k) tc::tmem_st16(lane_base + kColQ + 16 * k, reinterpret_cast<const uint32_t*>(qw + 4 * k));
             tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(q_full);
         }
-        float* const own_list = lists + ((cq * 2 + (q4 & 1)) * 2 + (q4 >> 1)) * CAP * 32 + lane;
-        float* const pair_list = lists + ((cq * 2 + (q4 & 1)) * 2) * CAP * 32 + lane;
-        float* cl = own_list;   // this thread's list, entry k at cl[32 k]
+        const int own_off = ((cq * 2 + (q4 & 1)) * 2 + (q4 >> 1)) * CAP * 32 + lane;
+        const int pair_off = ((cq * 2 + (q4 & 1)) * 2) * CAP * 32 + lane;
+        float* cl = lists + own_off;            // this thread's list, entry k at cl[32 k]
+        unsigned short* ci = lidx + own_off;    // and its chunk index at ci[32 k]
         int cap = CAP;
         float mx = -INFINITY, lo = 0.f, t = 0.f;
         float hi = 0.f;
-        float om[3] = {-INFINITY, -INFINITY, -INFINITY};   // the other three column sets' row maxima
+        float om[3] = {-INFINITY, -INFINITY, -INFINITY};   // lower bounds on the other column sets' maxima
         float lo_t = 0.f;   // this thread's list cut: lo, raised by its own subset bounds
         int m = 0;
         bool ok = true, emitted = false, redo_me = false;
-        int kind = 0;   // pass kind: 0 row maximum, 1 candidate extraction, 2 weights and emission
+        int kind = 0;   // pass kind: 0 row maximum (hi plane), 1 candidate extraction
         int half = -1;  // rows in play: all (-1), or the quarters q4 >> 1 == half
         int nextract = 0;
+        const float kmax = __ldg(knorm + br);   // largest |k̄_c| of this (sequence, KV head)
         for (int k = 0, u = 0;; ++k) {
             const bool active = half < 0 || (q4 >> 1) == half;
             for (int kb = 0; kb < nbk; ++kb, ++u) {
@@ -341,23 +358,27 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                     // column = kb * kBW + 32 lp + e
                     for (int lp = 0; lp < kPieces; ++lp) {
                         if ((kb * kPieces + lp) % 4 != cq) continue;
-                        const int c0 = kb * kBW + lp * 32;
                         // columns past every row of the warp: never read (the g rows of a position
-                        // sit in one warp, and the emission stops at the position's own bound)
-                        if (c0 >= nvw) continue;
-                        float v[32];
-                        tc::tmem_ld32(lane_base + hlf * kBW + lp * 32, v);
-                        tc::tmem_wait_ld();
+                        // sit in one warp, and the emission stops at the position's own bound);
+                        // 16 columns per TMEM load keep the register footprint low
+#pragma unroll 1
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int c0 = kb * kBW + lp * 32 + 16 * hh;
+                            if (c0 >= nvw) break;
+                            float v[16];
+                            tc::tmem_ld16(lane_base + hlf * kHalfCol + lp * 32 + 16 * hh, v);
+                            tc::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = c0 + e < nv ? v[e] * xs : -INFINITY;
-                        if (kind == 0) {
+                            for (int e = 0; e < 16; ++e) v[e] = c0 + e < nv ? v[e] * xs : -INFINITY;
+                            if (kind == 0) {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
-                        } else if (kind == 1) {
+                                for (int e = 0; e < 16; ++e) mx = fmaxf(mx, v[e]);
+                                continue;
+                            }
                             // entries above the cut, compacted by prefix popcount (no serial chain)
                             uint32_t mask = 0u;
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) mask |= (v[e] > lo_t ? 1u : 0u) << e;
+                            for (int e = 0; e < 16; ++e) mask |= (v[e] > lo_t ? 1u : 0u) << e;
                             if (m + __popc(mask) > cap && m <= cap) {
                                 // list full: raise the cut to this thread's subset bound on tau
                                 // (less the margin below) and drop the entries under it
@@ -368,57 +389,154 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                                     int j = 0;
                                     for (int kk = 0; kk < m; ++kk) {
                                         const float x = cl[32 * kk];
-                                        if (x > cut) cl[32 * j++] = x;
+                                        if (x > cut) {
+                                            ci[32 * j] = ci[32 * kk];
+                                            cl[32 * j++] = x;
+                                        }
                                     }
                                     m = j;
                                     mask = 0u;
 #pragma unroll
-                                    for (int e = 0; e < 32; ++e) mask |= (v[e] > lo_t ? 1u : 0u) << e;
+                                    for (int e = 0; e < 16; ++e) mask |= (v[e] > lo_t ? 1u : 0u) << e;
                                 }
                             }
                             if (mask) {
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) {
+                                for (int e = 0; e < 16; ++e) {
                                     const int kk = m + __popc(mask & ((1u << e) - 1u));
-                                    if (((mask >> e) & 1u) && kk < cap) cl[kk * 32] = v[e];
+                                    if (((mask >> e) & 1u) && kk < cap) {
+                                        cl[kk * 32] = v[e];
+                                        ci[kk * 32] = (unsigned short)(c0 + e);
+                                    }
                                 }
                                 m += __popc(mask);
                             }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const float uu = v[e] - t;
-                                v[e] = uu > 0.f ? pw(uu, p, mode) : 0.f;
-                            }
-                            int off;
-                            group_reduce_scatter<G>(v, lane, &off);
-#pragma unroll
-                            for (int j = 0; j < 32 / G; ++j) wbuf[pl * kBW + lp * 32 + off + j] = v[j];
                         }
                     }
                 }
                 // TMEM half read: the MMAs of use u + 2 may overwrite it
                 tc::fence_before_sync();
                 tc::mbar_arrive(x_free0 + 8 * hlf);
-
-                if (kind == 2 && ok) {
-                    // ---- this block's routed chunks of each position in play: warp per position,
-                    // ascending, log w for now (the bias needs the mean over all blocks) ---------
+            }
+            if (kind == 0) {
+                // row maximum over the four warps of the rows, from the hi plane: less the bound on
+                // |x - x_hi| it is a lower bound on the exact maximum, so the lists start at that
+                // value - 1 (tau >= max - 1: the largest entry alone gives f(max - 1) >= 1)
+                red[cq * kR + row].x = mx;
+                group_sync();
+#pragma unroll
+                for (int j = 0; j < 3; ++j) om[j] = red[((cq + 1 + j) & 3) * kR + row].x;
+                mx = fmaxf(fmaxf(mx, om[0]), fmaxf(om[1], om[2]));
+                const float eb = xs * kHiPlaneBound * qnorm[row] * kmax + 1e-6f * fmaxf(1.f, fabsf(mx));
+#pragma unroll
+                for (int j = 0; j < 3; ++j) om[j] -= eb;
+                lo = mx - eb - 1.f;
+                lo_t = lo;
+                hi = nv > 0 ? mx + eb - exp2f(-(s.alpha - 1.f) * __log2f((float)nv)) : 0.f;
+                kind = 1;
+                continue;   // an extraction pass always follows
+            }
+            // ---- after an extraction pass: threshold on the lists.  A list that overflowed
+            // dropped entries, and the root on the entries kept is then a lower bound on tau
+            // (a subset's f is smaller everywhere) from which the next extraction starts ----------
+            if (active && m > cap) atomicOr(overflow, 1);
+            workers_sync();   // also orders the reads of the maxima before the slots are reused
+            const bool over = *overflow != 0;
+            ++nextract;
+            if (ok && active) {
+                const int mm = min(m, cap);
+                const int m4 = (mm + 3) >> 2;
+                for (int kk = mm; kk < 4 * m4; ++kk) cl[kk * 32] = -INFINITY;
+                // every list holds all of its column set's entries above the largest of the
+                // four cuts (each cut is at most tau), so the solve starts there
+                red[(4 + cq) * kR + row].y = lo_t;
+                group_sync();
+                lo = fmaxf(fmaxf(red[(4 + 0) * kR + row].y, red[(4 + 1) * kR + row].y),
+                           fmaxf(red[(4 + 2) * kR + row].y, red[(4 + 3) * kR + row].y));
+                // the solve from t = lo (entmax.cuh, ent_step), the four warps' partial sums
+                // combined in a fixed order; every row of the quarter steps until all are done
+                // (the group barriers stay matched).  Iteration 0 writes slot 0, read last before
+                // the barrier above; slot 1 (the cuts) is rewritten only after iteration 0's barrier.
+                float lo_n = lo, hi_n = hi;
+                t = lo;
+                bool done = nv == 0;
+                for (int it = 0; it < 32 && !__all_sync(0xffffffffu, done); ++it) {
+                    EntSums S = ent_zero();
+                    if (mode == 2) {
+                        for (int kk = 0; kk < m4; ++kk) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float uu = cl[(4 * kk + j) * 32] - t;
+                                const float up = fmaxf(uu, 0.f);
+                                S.f = fmaf(up, up, S.f);
+                                S.fd += up;
+                                S.n += uu > 0.f ? 1.f : 0.f;
+                                S.um = fminf(S.um, uu > 0.f ? uu : INFINITY);
+                            }
+                        }
+                    } else {
+                        for (int kk = 0; kk < 4 * m4; ++kk) ent_add(S, cl[kk * 32] - t, p, mode);
+                    }
+                    float4* slot = red + (it & 1) * 4 * kR;
+                    slot[cq * kR + row] = make_float4(S.f, S.fd, S.n, S.um);
+                    group_sync();
+                    const float4 r0 = slot[row], r1 = slot[kR + row], r2 = slot[2 * kR + row], r3 = slot[3 * kR + row];
+                    S.f = (r0.x + r1.x) + (r2.x + r3.x);
+                    S.fd = (r0.y + r1.y) + (r2.y + r3.y);
+                    S.n = (r0.z + r1.z) + (r2.z + r3.z);
+                    S.um = fminf(fminf(r0.w, r1.w), fminf(r2.w, r3.w));
+                    if (!done) done = ent_step(S, t, lo_n, hi_n, s.alpha, mode);
+                }
+                if (over) {
+                    // the next lists keep the entries above the bound, less a margin far
+                    // above the solve's rounding (f' at the root is at least 1/(alpha-1))
+                    lo = fmaxf(lo, t - 1e-3f * fmaxf(1.f, fabsf(t)));
+                }
+            }
+            bool stop = false;
+            if (!ok) stop = true;
+            else if (!over) {
+                // ---- every list holds its column set's whole support: head weights, their sums
+                // over the g heads of each position and the route lists, window by window (kWin
+                // chunks).  Each thread writes its own row's weights of the window into wh (one
+                // row per TMEM lane, zero elsewhere); the position's warp then sums its g rows in
+                // head order: a fixed order, no atomics ---------------------------------------------
+                const int mm = min(m, cap);
+                int cur = 0;
+                const int nwin = (nvmax + kWin - 1) / kWin;
+                for (int wi = 0; wi < nwin; ++wi) {
+                    const int c0 = wi * kWin;
+                    float4* z4 = reinterpret_cast<float4*>(wbuf);
+                    for (int e = tid - 64; e < kR * kWin / 4; e += 512) z4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
                     workers_sync();
+                    if (active) {
+                        for (; cur < mm; ++cur) {
+                            const int c = ci[cur * 32];
+                            if (c >= c0 + kWin) break;
+                            const float uu = cl[cur * 32] - t;
+                            if (uu > 0.f) wbuf[row * kWin + (c - c0)] = ent_pow(uu, p, mode);
+                        }
+                    }
+                    workers_sync();
+                    // this window's routed chunks of each position in play: warp per position,
+                    // ascending, log w for now (the bias needs the mean over all windows)
                     for (int pp = warp - 2; pp < P; pp += 16) {
                         const int ip = i0 + pp;
                         if (ip >= s.n || (half >= 0 && ((pp * G) >> 6) != half)) continue;
                         const int nvp = min(ip / s.B, s.T);
-                        const float* Wp = wbuf + pp * kBW;
+                        const float* Wp = wbuf + pp * G * kWin;
                         const float inv_g = 1.f / G;
                         const long long toff = tri_offset(ip, s.B);
                         uint32_t* mrow = bm ? bm + (long long)ip * rt.words : nullptr;
                         int basec = pcnt[pp];
                         float slog = 0.f;
-                        for (int j0 = 0; j0 < kBW; j0 += 32) {
-                            const int c = kb * kBW + j0 + lane;
-                            if (kb * kBW + j0 >= nvp) break;
-                            const float w = c < nvp ? Wp[j0 + lane] * inv_g : 0.f;
+                        for (int j0 = 0; j0 < kWin; j0 += 32) {
+                            const int c = c0 + j0 + lane;
+                            if (c0 + j0 >= nvp) break;
+                            float a = 0.f;
+#pragma unroll
+                            for (int h = 0; h < G; ++h) a += Wp[h * kWin + j0 + lane];
+                            const float w = c < nvp ? a * inv_g : 0.f;
                             const bool on = w > 0.f;
                             const uint32_t msk = __ballot_sync(0xffffffffu, on);
                             if (on) {
@@ -436,107 +554,37 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                         if (lane == 0) { pslog[pp] += slog; pcnt[pp] = basec; }
                         __syncwarp();
                     }
-                    workers_sync();   // wbuf is rewritten by the next block
+                    workers_sync();   // wbuf is rewritten by the next window
                 }
-            }
-            if (kind == 0) {
-                // row maximum over the four warps of the rows; the first lists start at max - 1
-                // (tau >= max - 1: the largest entry alone already gives f(max - 1) >= 1)
-                red[(2 * 4 + cq) * kR + row].x = mx;
-                group_sync();
-#pragma unroll
-                for (int j = 0; j < 3; ++j) om[j] = red[(2 * 4 + ((cq + 1 + j) & 3)) * kR + row].x;
-                mx = fmaxf(fmaxf(mx, om[0]), fmaxf(om[1], om[2]));
-                lo = mx - 1.f;
-                lo_t = lo;
-                hi = nv > 0 ? mx - exp2f(-(s.alpha - 1.f) * __log2f((float)nv)) : 0.f;
-                kind = 1;
-                continue;   // an extraction pass always follows
-            }
-            bool stop = false;
-            if (kind == 1) {
-                // ---- after an extraction pass: threshold on the lists.  A list that overflowed
-                // dropped entries, and the root on the entries kept is then a lower bound on tau
-                // (a subset's f is smaller everywhere) from which the next extraction starts ------
-                if (active && m > cap) atomicOr(overflow, 1);
-                workers_sync();
-                const bool over = *overflow != 0;
-                ++nextract;
-                if (ok && active) {
-                    const int mm = min(m, cap);
-                    const int m4 = (mm + 3) >> 2;
-                    for (int kk = mm; kk < 4 * m4; ++kk) cl[kk * 32] = -INFINITY;
-                    // every list holds all of its column set's entries above the largest of the
-                    // four cuts (each cut is at most tau), so the solve starts there
-                    red[(2 * 4 + cq) * kR + row].y = lo_t;
-                    group_sync();
-                    lo = fmaxf(fmaxf(red[(2 * 4 + 0) * kR + row].y, red[(2 * 4 + 1) * kR + row].y),
-                               fmaxf(red[(2 * 4 + 2) * kR + row].y, red[(2 * 4 + 3) * kR + row].y));
-                    // Newton on g(t) = f(t)^(alpha-1) from t = lo (see stage1.cu), the four warps'
-                    // partial sums combined in a fixed order; every row of the quarter steps until
-                    // all have converged (the group barriers stay matched)
-                    float lo_n = lo, hi_n = hi;
-                    t = lo;
-                    bool done = nv == 0;
-                    for (int it = 0; it < 32 && !__all_sync(0xffffffffu, done); ++it) {
-                        float f = 0.f, fd = 0.f;
-                        if (mode == 2) {
-                            for (int kk = 0; kk < m4; ++kk) {
-                                const float u0 = fmaxf(cl[(4 * kk) * 32] - t, 0.f), u1 = fmaxf(cl[(4 * kk + 1) * 32] - t, 0.f);
-                                const float u2 = fmaxf(cl[(4 * kk + 2) * 32] - t, 0.f), u3 = fmaxf(cl[(4 * kk + 3) * 32] - t, 0.f);
-                                f += u0 * u0 + u1 * u1 + u2 * u2 + u3 * u3;
-                                fd += (u0 + u1) + (u2 + u3);
-                            }
-                        } else {
-                            for (int kk = 0; kk < 4 * m4; ++kk) {
-                                const float uu = cl[kk * 32] - t;
-                                if (uu > 0.f) { f += pw(uu, p, mode); fd += dpw(uu, p, mode); }
-                            }
-                        }
-                        float2* slot = red + (it & 1) * 4 * kR;
-                        slot[cq * kR + row] = make_float2(f, fd);
-                        group_sync();
-                        const float2 r0 = slot[row], r1 = slot[kR + row], r2 = slot[2 * kR + row], r3 = slot[3 * kR + row];
-                        f = (r0.x + r1.x) + (r2.x + r3.x);
-                        fd = (r0.y + r1.y) + (r2.y + r3.y);
-                        if (!done) {
-                            if (f >= 1.f) lo_n = t; else hi_n = t;
-                            float tn = 0.5f * (lo_n + hi_n);
-                            if (fd > 0.f && f > 0.f) {
-                                const float gg = mode == 2 ? sqrtf(f) : mode == 1 ? f : exp2f((s.alpha - 1.f) * __log2f(f));
-                                tn = t + (gg - 1.f) * f / (gg * fd);
-                            }
-                            if (fabsf(tn - t) <= 2e-7f * fmaxf(1.f, fabsf(t)) || fabsf(f - 1.f) <= 1e-6f) { t = tn; done = true; }
-                            else {
-                                if (!(tn > lo_n && tn < hi_n)) tn = 0.5f * (lo_n + hi_n);
-                                t = tn;
-                            }
-                        }
-                    }
-                    if (over) {
-                        // the next lists keep the entries above the bound, less a margin far
-                        // above the solve's rounding (f' at the root is at least 1/(alpha-1))
-                        lo = fmaxf(lo, t - 1e-3f * fmaxf(1.f, fabsf(t)));
-                    }
-                }
-                if (!ok) stop = true;
-                else if (!over) kind = 2;
-                else if (nextract < kMaxExtract) { lo_t = lo; m = 0; }
-                else if (half < 0) {
-                    // a column set holds more of the support than its list: redo the rows in two
-                    // halves, each thread of the half in play taking its idle partner's list too
-                    half = 0;
+                // the ring is written by TMA again only after this pass's decision; order this
+                // thread's generic accesses to it before those asynchronous-proxy writes
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (half == 0) {
+                    // the second half of the rows: extraction passes of its own
+                    half = 1;
                     nextract = 0;
                     lo_t = lo;
                     m = 0;
-                    cl = pair_list;
-                    cap = 2 * CAP;
-                } else { stop = true; redo_me = true; }
+                } else {
+                    stop = true;
+                    emitted = true;
+                }
+            } else if (nextract < kMaxExtract) {
+                lo_t = lo;
+                m = 0;
+            } else if (half < 0) {
+                // a column set holds more of the support than its list: redo the rows in two
+                // halves, each thread of the half in play taking its idle partner's list too
+                half = 0;
+                nextract = 0;
+                lo_t = lo;
+                m = 0;
+                cl = lists + pair_off;
+                ci = lidx + pair_off;
+                cap = 2 * CAP;
             } else {
-                // ---- after a weights pass
-                if (!ok) stop = true;
-                else if (half == 0) { half = 1; kind = 1; nextract = 0; lo_t = lo; m = 0; }
-                else { stop = true; emitted = true; }
+                stop = true;
+                redo_me = true;
             }
             workers_sync();   // every worker has read the overflow word
             if (tid == 64) {
@@ -589,8 +637,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_l()
 }
 
 template <int G>
-cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
-                          unsigned char* redo, int* err, cudaStream_t st)
+cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* planes, const float* knorm,
+                          const Routes& rt, unsigned char* redo, int* err, cudaStream_t st)
 {
     auto fn = encode_fn_l();
     if (!fn) return cudaErrorInvalidValue;
@@ -600,7 +648,7 @@ cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* pl
         // planes [b*hkv*3][T][128] viewed as (d, chunk, plane-row, 1)
         cuuint64_t dims[4] = {128, (cuuint64_t)s.T, (cuuint64_t)s.batch * s.hkv * 3, 1};
         cuuint64_t strides[3] = {128 * 2, (cuuint64_t)s.T * 128 * 2, (cuuint64_t)s.T * 128 * 2 * s.batch * s.hkv * 3};
-        cuuint32_t box[4] = {64, (cuuint32_t)kCT, 1, 1};
+        cuuint32_t box[4] = {64, (cuuint32_t)kBW, 1, 1};
         cuuint32_t es[4] = {1, 1, 1, 1};
         if (fn(&mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(planes), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -614,7 +662,7 @@ cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* pl
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 576, smem, st>>>(mp, static_cast<const __nv_bfloat16*>(Q), s, rt, redo, err);
+    k<<<grid, 576, smem, st>>>(mp, static_cast<const __nv_bfloat16*>(Q), knorm, s, rt, redo, err);
     return cudaGetLastError();
 }
 
@@ -629,13 +677,13 @@ bool route_long_supported(const Shape& s, int dtype)
 
 int route_long_positions(const Shape& s) { return kR / s.g; }
 
-cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
-                                      unsigned char* redo, int* err, cudaStream_t st)
+cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const float* knorm,
+                                      const Routes& rt, unsigned char* redo, int* err, cudaStream_t st)
 {
     switch (s.g) {
-    case 4: return launch_long_g<4>(s, Q, planes, rt, redo, err, st);
-    case 8: return launch_long_g<8>(s, Q, planes, rt, redo, err, st);
-    default: return launch_long_g<16>(s, Q, planes, rt, redo, err, st);
+    case 4: return launch_long_g<4>(s, Q, planes, knorm, rt, redo, err, st);
+    case 8: return launch_long_g<8>(s, Q, planes, knorm, rt, redo, err, st);
+    default: return launch_long_g<16>(s, Q, planes, knorm, rt, redo, err, st);
     }
 }
 

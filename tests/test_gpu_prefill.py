@@ -158,15 +158,16 @@ def test_gamma_zero_is_dense_causal_attention():
     assert np.array_equal(cnt, np.broadcast_to(np.arange(1536) // 64, cnt.shape))
 
 
-def test_bitmask_matches_lists():
-    x = inputs.planted(14, 1, 2048, 8, 2, 128, 32, dtype="bf16")
-    O, pf = run_prefill(x, chunk=32, alpha=1.5, gamma=8.0, bitmask=True)
+@pytest.mark.parametrize("n,B", [(2048, 32), (9000, 16)], ids=["T64", "T562_long_rows"])
+def test_bitmask_matches_lists(n, B):
+    x = inputs.planted(14, 1, n, 8, 2, 128, B, dtype="bf16")
+    O, pf = run_prefill(x, chunk=B, alpha=1.5, gamma=8.0, bitmask=True)
     bm = pf.bitmask.cpu().numpy().view(np.uint32)
     cnt, idx = pf.counts.cpu().numpy(), pf.chunk_idx.cpu().numpy()
     from parity import tri_offset
     for r in range(2):
-        for i in range(0, 2048, 37):
-            off = tri_offset(i, 32)
+        for i in range(0, n, 37):
+            off = tri_offset(i, B)
             lst = idx[0, r, off:off + cnt[0, r, i]]
             bits = np.unpackbits(bm[0, r, i].view(np.uint8), bitorder="little")
             assert np.array_equal(np.nonzero(bits)[0], lst)
