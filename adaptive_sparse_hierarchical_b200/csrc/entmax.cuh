@@ -62,6 +62,7 @@ __device__ __forceinline__ void ent_merge(EntSums& a, const EntSums& b)
 //    decreasing, and linear while the support is fixed, so from t = max x - 1 (where f >= 1) the
 //    iterates rise monotonically to the root; g' = -f^(alpha-2) fd, so the step (g - 1)/(-g')
 //    is (g - 1) f / (g fd).  A step that leaves the bracket falls back to bisection.
+// Sums with n = 0 (a caller that leaves out the count and the minimum) take Newton steps only.
 __device__ __forceinline__ bool ent_step(const EntSums& S, float& t, float& lo, float& hi, float alpha, int mode)
 {
     if (S.f >= 1.f) lo = t; else hi = t;

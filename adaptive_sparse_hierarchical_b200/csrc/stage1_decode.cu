@@ -81,7 +81,7 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
     __shared__ float tau[kMaxG], gmax[kMaxG];
     __shared__ int wsum[kThr / 32 + 1];
     __shared__ float fsum[kThr / 32];
-    __shared__ float4 npart[2][kSlots * kRanks];      // solve partial sums [step parity][slot, source]
+    __shared__ float2 npart[2][kSlots * kRanks];      // Newton partial sums [step parity][slot, source]
     __shared__ int ndone[kSlots];
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -194,7 +194,9 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
     cl.sync();
     // ---- thresholds: block `rank` solves heads h = rank + kRanks slot on the pushed entries; warp
     // (slot, k) sums over source block k's entries, the partials are added in k order, and every
-    // thread of the slot takes the same step of the solve (entmax.cuh, ent_step) from max - 1 ---
+    // thread of the slot takes the same Newton step (entmax.cuh, ent_step; the closed-form finish
+    // is left out here: its count and minimum reductions cost more on these ~700-entry lists than
+    // the steps they save) from max - 1 -----------------------------------------------------------
     static_assert(kSlots * kRanks == kThr / 32, "one warp per (head slot, source block)");
     {
         const int slot = warp / kRanks, k = warp % kRanks, h = rank + kRanks * slot;
@@ -213,16 +215,17 @@ __global__ void __cluster_dims__(kRanks, 1, 1) __launch_bounds__(kThr, 1)
             for (int j = 0; j < kSlots; ++j) all = all && ndone[j];
             if (all) break;
             const int ph = it & 1;
-            EntSums S = ent_zero();
-            for (int j = lane; j < nk; j += 32) ent_add(S, gl[j] - t, p, mode);
-            ent_warp_reduce(S);
-            if (lane == 0) npart[ph][slot * kRanks + k] = make_float4(S.f, S.fd, S.n, S.um);
-            __syncthreads();   // a parity slot is rewritten two steps later, after the next barrier
-            S = ent_zero();
-            for (int kk = 0; kk < kRanks; ++kk) {
-                const float4 v = npart[ph][slot * kRanks + kk];
-                ent_merge(S, EntSums{v.x, v.y, v.z, v.w});
+            float f = 0.f, fd = 0.f;
+            for (int j = lane; j < nk; j += 32) {
+                const float u = gl[j] - t;
+                if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
             }
+            f = warp_sum(f);
+            fd = warp_sum(fd);
+            if (lane == 0) npart[ph][slot * kRanks + k] = make_float2(f, fd);
+            __syncthreads();   // a parity slot is rewritten two steps later, after the next barrier
+            EntSums S = ent_zero();   // n = 0: Newton steps only
+            for (int kk = 0; kk < kRanks; ++kk) { S.f += npart[ph][slot * kRanks + kk].x; S.fd += npart[ph][slot * kRanks + kk].y; }
             if (!dn) dn = ent_step(S, t, lo, hi, s.alpha, mode);
             // every thread of a slot holds the same state; the slot's first warp reports it
             if (k == 0 && lane == 0) ndone[slot] = dn;

@@ -8,10 +8,10 @@
 //   bias_c = (log w_c - mean_{c' in R} log w_c') / sigma                       (Prop. 4.1)
 //
 // One block = 128 query rows = (128/g positions) x (g heads) of one (sequence, KV head).
-//   warp 0     TMA: the Q tile once, then 64-chunk tiles of the three exact bf16 planes of the
-//              summaries (hi + mid + lo = kbar) into a 2-stage ring
+//   warp 0     TMA: the Q tile once, then 128-chunk tiles of the three exact bf16 planes of the
+//              summaries (hi + mid + lo = kbar) into a 3-stage ring, one plane per stage
 //   warp 1     allocates TMEM and issues, from one thread, X[:, tile] += Q . plane^T for the
-//              three planes (M=128, N=64, K=16 steps), so X holds the fp32 logits of every
+//              three planes (M=128, N=128, K=16 steps), so X holds the fp32 logits of every
 //              visible chunk, one row per TMEM lane
 //   warps 2-17 four warps per TMEM lane quarter (32 rows), each reading every fourth 32-column
 //              piece of its rows: max, Newton steps on f(t)^(alpha-1) and the head weights, the
@@ -32,15 +32,19 @@ namespace dash {
 
 namespace {
 
-constexpr int kR = 128, kCT = 64, kDd = 128;
+constexpr int kR = 128, kCT = 128, kDd = 128;
 constexpr int kQB = kR * kDd * 2;               // Q tile, two 16 KB d-halves
-constexpr int kPlaneHalf = kCT * 64 * 2;        // [64 chunks][64 d] bf16 = 8 KB
-constexpr int kStage = 3 * 2 * kPlaneHalf;      // three planes x two d-halves = 48 KB
-constexpr int kOffQ1 = 0, kOffRing = kQB, kOffW = kOffRing + 2 * kStage;
+constexpr int kPlaneHalf = kCT * 64 * 2;        // [128 chunks][64 d] bf16 = 16 KB
+constexpr int kStage = 2 * kPlaneHalf;          // one plane of a tile, two d-halves = 32 KB
+constexpr int kNS = 3;                          // ring stages
+constexpr int kOffQ1 = 0, kOffRing = kQB, kOffW = kOffRing + kNS * kStage;
 constexpr int kCand = 48;   // candidate list length per row and warp: 16 x 32 x 48 floats fill the ring
-static_assert(16 * 32 * kCand * 4 <= 2 * kStage && kCand % 4 == 0, "candidate lists must fit the ring");
+static_assert(16 * 32 * kCand * 4 <= kNS * kStage && kCand % 4 == 0, "candidate lists must fit the ring");
+static_assert(16 + 16 * kNS + 8 <= 96, "barriers below the TMEM slot");
 constexpr int kMisc = 128 + 3 * 4 * kR * 16;    // barriers, TMEM slot, abort flag, reduction slots
-constexpr uint32_t kIdescX = tc::idesc_bf16(128, 64, false, false);
+// one M = 128, N = 128 MMA per (tile, plane, 16-wide k step): narrower MMAs accumulating into one
+// tile form dependent chains that run well below the tensor rate
+constexpr uint32_t kIdescX = tc::idesc_bf16(128, kCT, false, false);
 
 // Sum over the g neighbouring lanes of a position of 32 values, reduce-scattered: afterwards
 // lane (h = lane % g) holds the sums of the 32/g columns starting at *off.
@@ -81,10 +85,10 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
     float4* red = reinterpret_cast<float4*>(misc + 128);          // [3][4][kR] partial solve sums / max
     const uint32_t bar0 = tc::smem_addr(misc);
     const uint32_t q_full = bar0, x_ready = bar0 + 8;
-    const uint32_t full0 = bar0 + 16, empty0 = bar0 + 32;          // [2] each
-    const uint32_t drain = bar0 + 48;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 64);
-    volatile int* abort = reinterpret_cast<volatile int*>(misc + 68);
+    const uint32_t full0 = bar0 + 16, empty0 = bar0 + 16 + 8 * kNS;   // [kNS] each
+    const uint32_t drain = bar0 + 16 + 16 * kNS;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 96);
+    volatile int* abort = reinterpret_cast<volatile int*>(misc + 100);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nblk = (s.n + P - 1) / P;
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
     if (tid == 0) {
         tc::mbar_init(q_full, 1);
         tc::mbar_init(x_ready, 1);
-        for (int k = 0; k < 2; ++k) { tc::mbar_init(full0 + 8 * k, 1); tc::mbar_init(empty0 + 8 * k, 1); }
+        for (int k = 0; k < kNS; ++k) { tc::mbar_init(full0 + 8 * k, 1); tc::mbar_init(empty0 + 8 * k, 1); }
         tc::mbar_init(drain, 1);
         *abort = 0;
         tc::mbar_fence_init();
@@ -133,24 +137,25 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
             tc::mbar_expect_tx(q_full, kQB);
             tc::tma_load_4d(base + kOffQ1, &tmQ, q_full, 0, r * G, i0, b);
             tc::tma_load_4d(base + kOffQ1 + kQB / 2, &tmQ, q_full, 64, r * G, i0, b);
-            int last[2] = {-1, -1};
-            for (int t = 0; t < ntiles; ++t) {
-                const int st = t & 1;
-                if (t >= 2 && !tc::mbar_wait(empty0 + 8 * st, ((t >> 1) - 1) & 1, abort, err, 21)) break;
-                last[st] = t;
+            int last[kNS];
+#pragma unroll
+            for (int k = 0; k < kNS; ++k) last[k] = -1;
+            bool pok = true;
+            // one ring stage per (tile, plane); chunks past T read as zeros (never used)
+            for (int gs = 0; pok && gs < 3 * ntiles; ++gs) {
+                const int st = gs % kNS, t = gs / 3, pl = gs % 3;
+                if (gs >= kNS && !tc::mbar_wait(empty0 + 8 * st, ((gs / kNS) - 1) & 1, abort, err, 21)) { pok = false; break; }
+                last[st] = gs;
                 const uint32_t dst = base + kOffRing + st * kStage, fb = full0 + 8 * st;
                 tc::mbar_expect_tx(fb, kStage);
-#pragma unroll
-                for (int pl = 0; pl < 3; ++pl) {
-                    tc::tma_load_4d(dst + (2 * pl) * kPlaneHalf, &tmP, fb, 0, t * kCT, br * 3 + pl, 0);
-                    tc::tma_load_4d(dst + (2 * pl + 1) * kPlaneHalf, &tmP, fb, 64, t * kCT, br * 3 + pl, 0);
-                }
+                tc::tma_load_4d(dst, &tmP, fb, 0, t * kCT, br * 3 + pl, 0);
+                tc::tma_load_4d(dst + kPlaneHalf, &tmP, fb, 64, t * kCT, br * 3 + pl, 0);
             }
             if (*abort) {
-                for (int k = 0; k < 2; ++k)
+                for (int k = 0; k < kNS; ++k)
                     if (last[k] >= 0)
                         for (long long it = 0; it < (1ll << 22); ++it)
-                            if (tc::mbar_try(full0 + 8 * k, (last[k] >> 1) & 1)) break;
+                            if (tc::mbar_try(full0 + 8 * k, (last[k] / kNS) & 1)) break;
                 for (long long it = 0; it < (1ll << 22); ++it)
                     if (tc::mbar_try(q_full, 0)) break;
             }
@@ -162,19 +167,17 @@ __global__ void __launch_bounds__(576, 1) route_prefill_tcgen05_kernel(const __g
             const uint64_t dQ = tc::sw128_desc(base + kOffQ1, 16, 1024);
             const uint64_t dP0 = tc::sw128_desc(base + kOffRing, 16, 1024);
             bool ok = tc::mbar_wait(q_full, 0, abort, err, 22);
-            for (int t = 0; ok && t < ntiles; ++t) {
-                const int st = t & 1;
-                if (!tc::mbar_wait(full0 + 8 * st, (t >> 1) & 1, abort, err, 23)) { ok = false; break; }
+            for (int gs = 0; ok && gs < 3 * ntiles; ++gs) {
+                const int st = gs % kNS, t = gs / 3, pl = gs % 3;
+                if (!tc::mbar_wait(full0 + 8 * st, (gs / kNS) & 1, abort, err, 23)) { ok = false; break; }
                 tc::fence_after_sync();
                 const uint64_t dp = dP0 + (uint64_t)((st * kStage) >> 4);
                 const uint32_t xd = tmem + t * kCT;
 #pragma unroll
-                for (int pl = 0; pl < 3; ++pl)
-#pragma unroll
-                    for (int kk = 0; kk < kDd / 16; ++kk)
-                        tc::mma_f16_ss(xd, dQ + (uint64_t)(((kk >> 2) * (kQB / 2) + (kk & 3) * 32) >> 4),
-                                       dp + (uint64_t)(((2 * pl + (kk >> 2)) * kPlaneHalf + (kk & 3) * 32) >> 4), kIdescX,
-                                       (pl > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kDd / 16; ++kk)
+                    tc::mma_f16_ss(xd, dQ + (uint64_t)(((kk >> 2) * (kQB / 2) + (kk & 3) * 32) >> 4),
+                                   dp + (uint64_t)(((kk >> 2) * kPlaneHalf + (kk & 3) * 32) >> 4), kIdescX,
+                                   (pl > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(empty0 + 8 * st);
             }
             if (ok) tc::mma_commit(x_ready);
@@ -391,7 +394,7 @@ cudaError_t launch_g(const Shape& s, const void* Q, const __nv_bfloat16* planes,
         // planes [b*hkv*3][T][128] viewed as (d, chunk, plane-row, 1)
         cuuint64_t dims[4] = {128, (cuuint64_t)s.T, (cuuint64_t)s.batch * s.hkv * 3, 1};
         cuuint64_t strides[3] = {128 * 2, (cuuint64_t)s.T * 128 * 2, (cuuint64_t)s.T * 128 * 2 * s.batch * s.hkv * 3};
-        cuuint32_t box[4] = {64, (cuuint32_t)kCT, 1, 1};
+        cuuint32_t box[4] = {64, (cuuint32_t)kCT, 1, 1};   // 128 chunks x 64 d
         cuuint32_t es[4] = {1, 1, 1, 1};
         if (fn(&mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(planes), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
