@@ -274,16 +274,20 @@ __global__ void __launch_bounds__(192, 2) attend_prefill_tc_kernel(const __grid_
             atomicOr(&umask[u >> 5], 1u << (u & 31));
         }
     } else {
-        for (int p = 0; p < P; ++p) {
+        // union units from the positions' lists: blockDim / P threads per position, all positions
+        // at once (one round trip for the counts, one for the entries)
+        const int tpp = max(1, (int)blockDim.x / P);
+        for (int p = tid / tpp; p < P; p += (int)blockDim.x / tpp) {
+            const int sub = tid % tpp;
             const int i = spos[p];
             if (i >= s.n) continue;
             const int cnt = counts[i];
             const int* li = ridx + tri_offset(i, s.B);
-            for (int k = tid; k < cnt; k += blockDim.x) {
+            for (int k = sub; k < cnt; k += tpp) {
                 const int u = li[k] / CPT;
                 atomicOr(&umask[u >> 5], 1u << (u & 31));
             }
-            if (tid == 0) {
+            if (sub == 0) {
                 const int u = (i / s.B) / CPT;
                 atomicOr(&umask[u >> 5], 1u << (u & 31));
             }
