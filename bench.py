@@ -33,7 +33,7 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # DRAM bytes per launch of a Stage 2 kernel (dram__bytes_read.sum + dram__bytes_write.sum from one
 # ncu capture of the current kernel on that workload), keyed by (kernel, workload); absent until
 # the current kernel has been captured.
-STAGE2_TRAFFIC = {("attend_prefill_tc_kernel (tcgen05, one tile per block)", "prefill_32k"): 314.7e6}
+STAGE2_TRAFFIC = {("attend_prefill_tc_kernel (tcgen05, one tile per block)", "prefill_32k"): 314.5e6}
 
 
 def stage2_kernel_name():
