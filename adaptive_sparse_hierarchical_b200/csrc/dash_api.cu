@@ -124,7 +124,9 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.planes = L.err + up(16 + bh * 4);
     L.redo = L.planes + up(bh * 3 * T * p->d_h * 2);
     L.perm = L.redo + up(bh * (size_t)p->seqlen);   // one flag per position block at most
-    L.total = L.perm + up(bh * (size_t)p->seqlen * 4);
+    // Stage 2's position order; before Stage 2 rewrites it, Stage 1's list of position blocks to
+    // recompute (one count + one int per block at most)
+    L.total = L.perm + up(bh * (size_t)p->seqlen * 4 + 16);
     return L;
 }
 
@@ -256,7 +258,7 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     if (stage == -1 || stage == DASH_STAGE1) {
         unsigned char* redo = reinterpret_cast<unsigned char*>(ws + L.redo);
         rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, planes ? knorm : nullptr, rt, redo,
-                                                err, st));
+                                                reinterpret_cast<int*>(ws + L.perm), err, st));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE2)

@@ -161,9 +161,10 @@ cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const vo
 // redo: one byte per (sequence, KV head, position block) for the long-row kernel's overflow flags
 // knorm: per (sequence, KV head) the largest Euclidean norm of a summary (written by Stage 0
 // with the planes; the long-row kernel's hi-plane bound)
+// redo_list: scratch of 1 + batch * h_kv * n ints for the list of position blocks to recompute
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
                                  const __nv_bfloat16* planes, const float* knorm, const Routes& rt,
-                                 unsigned char* redo, int* err, cudaStream_t st);
+                                 unsigned char* redo, int* redo_list, int* err, cudaStream_t st);
 // tcgen05 / TMEM variant of Stage 1 (bf16, d = 128, at most 512 complete chunks)
 bool route_tcgen05_supported(const Shape& s, int dtype);
 cudaError_t launch_route_prefill_tcgen05(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,

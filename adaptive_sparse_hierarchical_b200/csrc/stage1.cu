@@ -15,6 +15,7 @@
 // below it, so the steps never pass the root) finish to float precision; for alpha = 2 and 1.5
 // the closed-form root on the current support ends the solve once the support is found
 // (entmax.cuh, ent_step).
+#include <algorithm>
 #include <cstdlib>
 
 #include "dash_common.cuh"
@@ -76,10 +77,8 @@ __device__ __forceinline__ bool redo_wanted(const unsigned char* redo, int redo_
 // Shared memory: scaled query rows [rows][D], one summary tile [32][D+4], logits [rows][Ts].
 // ------------------------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __restrict__ Q,
-                                                            const float* __restrict__ kbar,
-                                                            Routes rt, int P, int Ts,
-                                                            const unsigned char* redo, int redo_p)
+__device__ void route_prefill_block(Shape s, const T* __restrict__ Q, const float* __restrict__ kbar, Routes rt,
+                                    int P, int Ts, const unsigned char* redo, int redo_p, int blk)
 {
     extern __shared__ float4 smem4[];
     float* qsm = reinterpret_cast<float*>(smem4);
@@ -87,8 +86,8 @@ __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __
     float* S = ktile + 32 * (D + 4);
     const int rows = P * s.g;
     const int nblk = (s.n + P - 1) / P;
-    const int br = blockIdx.x % (s.batch * s.hkv);
-    const int pb = nblk - 1 - blockIdx.x / (s.batch * s.hkv);   // heaviest blocks first
+    const int br = blk % (s.batch * s.hkv);
+    const int pb = nblk - 1 - blk / (s.batch * s.hkv);   // heaviest blocks first
     const int b = br / s.hkv, r = br % s.hkv;
     const int i0 = pb * P;
     const int ilast = min(i0 + P, s.n) - 1;
@@ -189,6 +188,25 @@ __global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __
     }
 }
 
+// Block number blk of the launch order above; with a list (list[0] entries from list[1] on), a
+// fixed grid walks the listed block numbers instead of one block per position block.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) route_prefill_kernel(Shape s, const T* __restrict__ Q,
+                                                            const float* __restrict__ kbar,
+                                                            Routes rt, int P, int Ts,
+                                                            const unsigned char* redo, int redo_p, const int* list)
+{
+    if (!list) {
+        route_prefill_block<T, D>(s, Q, kbar, rt, P, Ts, redo, redo_p, blockIdx.x);
+        return;
+    }
+    const int nl = list[0];
+    for (int w = blockIdx.x; w < nl; w += gridDim.x) {
+        route_prefill_block<T, D>(s, Q, kbar, rt, P, Ts, nullptr, 1, list[1 + w]);
+        __syncthreads();   // shared memory is reused by the next listed block
+    }
+}
+
 // Threshold from a compacted candidate list: tau >= max x - 1, so entries at or below max - 1
 // never enter the support and never contribute to the mass; the warp copies the others (about a
 // sixth of a typical row) to its scratch list once and takes the Newton passes over that list.
@@ -243,10 +261,9 @@ __device__ float warp_threshold_reg(const float (&xr)[NPL], int nv, float alpha)
 // threshold from registers.
 // ------------------------------------------------------------------------------------------
 template <int D, int RG>
-__global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __nv_bfloat16* __restrict__ Q,
-                                                               const __nv_bfloat16* __restrict__ planes,
-                                                               Routes rt, int Ts,
-                                                               const unsigned char* redo, int redo_p)
+__device__ void route_prefill_tc_block(Shape s, const __nv_bfloat16* __restrict__ Q,
+                                       const __nv_bfloat16* __restrict__ planes, Routes rt, int Ts,
+                                       const unsigned char* redo, int redo_p, int blk)
 {
     constexpr int ROWS = 16 * RG;
     constexpr int TCH = 32;                    // chunks per staged tile
@@ -257,8 +274,8 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
     float* scratch = S + ROWS * Ts + (threadIdx.x >> 5) * 512;   // per-warp candidate list
     const int G = s.g, P = ROWS / G;
     const int nblk = (s.n + P - 1) / P;
-    const int br = blockIdx.x % (s.batch * s.hkv);
-    const int pb = nblk - 1 - blockIdx.x / (s.batch * s.hkv);   // heaviest blocks first
+    const int br = blk % (s.batch * s.hkv);
+    const int pb = nblk - 1 - blk / (s.batch * s.hkv);   // heaviest blocks first
     const int b = br / s.hkv, r = br % s.hkv;
     const int i0 = pb * P;
     const int ilast = min(i0 + P, s.n) - 1;
@@ -370,6 +387,57 @@ __global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __
 // the cached summaries of chunks c < floor((L_b - 1)/B).
 // (a) logits: one block per (32-chunk tile, sequence, KV head), all g heads of the group.
 // ------------------------------------------------------------------------------------------
+template <int D, int RG>
+__global__ void __launch_bounds__(256) route_prefill_tc_kernel(Shape s, const __nv_bfloat16* __restrict__ Q,
+                                                               const __nv_bfloat16* __restrict__ planes,
+                                                               Routes rt, int Ts,
+                                                               const unsigned char* redo, int redo_p, const int* list)
+{
+    if (!list) {
+        route_prefill_tc_block<D, RG>(s, Q, planes, rt, Ts, redo, redo_p, blockIdx.x);
+        return;
+    }
+    const int nl = list[0];
+    for (int w = blockIdx.x; w < nl; w += gridDim.x) {
+        route_prefill_tc_block<D, RG>(s, Q, planes, rt, Ts, nullptr, 1, list[1 + w]);
+        __syncthreads();   // shared memory is reused by the next listed block
+    }
+}
+
+// The block numbers (launch order of the two kernels above, P positions per block) whose
+// positions overlap a position block that the long-row kernel flagged: appended to list[1..],
+// list[0] counting them (zero on entry).  The order of the list does not matter.
+__global__ void __launch_bounds__(256) redo_compact_kernel(Shape s, int P, const unsigned char* __restrict__ redo,
+                                                           int redo_p, int* list)
+{
+    const int nblk = (s.n + P - 1) / P;
+    const long long total = (long long)nblk * s.batch * s.hkv;
+    const long long f = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (f >= total) return;
+    const int br = (int)(f % (s.batch * s.hkv));
+    const int pb = nblk - 1 - (int)(f / (s.batch * s.hkv));
+    const int i0 = pb * P, ilast = min(i0 + P, s.n) - 1;
+    if (redo_wanted(redo, redo_p, s, br, i0, ilast)) list[1 + atomicAdd(list, 1)] = (int)f;
+}
+
+// Launch of a routing kernel over every position block (redo == null), or over the blocks that
+// overlap a flagged one: compacted into redo_list first, then a fixed grid of a few blocks per SM.
+template <typename Launch>
+cudaError_t launch_redo(const Shape& s, int P, long long grid, const unsigned char* redo, int redo_p, int* redo_list,
+                        cudaStream_t st, Launch launch)
+{
+    if (grid <= 0) return cudaSuccess;
+    if (!redo || !redo_list) return launch((unsigned)grid, redo, (const int*)nullptr);
+    if (cudaMemsetAsync(redo_list, 0, sizeof(int), st) != cudaSuccess) return cudaErrorUnknown;
+    redo_compact_kernel<<<(unsigned)((grid + 255) / 256), 256, 0, st>>>(s, P, redo, redo_p, redo_list);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        nsm = 148;
+    return launch((unsigned)std::min<long long>(grid, 2LL * nsm), (const unsigned char*)nullptr, (const int*)redo_list);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) dec_logits_kernel(Shape s, const T* __restrict__ q,
                                                          const float* __restrict__ kbar, int kbar_T,
@@ -487,7 +555,7 @@ __global__ void __launch_bounds__(512) dec_route_kernel(Shape s, int kbar_T, con
 
 template <typename T, int D>
 cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, const Routes& rt,
-                            cudaStream_t st, const unsigned char* redo = nullptr, int redo_p = 1)
+                            cudaStream_t st, const unsigned char* redo = nullptr, int redo_p = 1, int* redo_list = nullptr)
 {
     int P = 0;
     const size_t smem = route_prefill_smem(s, &P);
@@ -497,10 +565,11 @@ cudaError_t route_prefill_t(const Shape& s, const void* Q, const float* kbar, co
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long nblk = (s.n + P - 1) / P;
-    const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
-    if (grid == 0) return cudaSuccess;
-    k<<<grid, 256, smem, st>>>(s, (const T*)Q, kbar, rt, P, Ts, redo, redo_p);
-    return cudaGetLastError();
+    return launch_redo(s, P, nblk * s.batch * s.hkv, redo, redo_p, redo_list, st,
+                       [&](unsigned grid, const unsigned char* rd, const int* list) {
+                           k<<<grid, 256, smem, st>>>(s, (const T*)Q, kbar, rt, P, Ts, rd, redo_p, list);
+                           return cudaGetLastError();
+                       });
 }
 
 // Shared memory of the tensor-core routing kernel for RG row groups.
@@ -512,7 +581,7 @@ size_t route_tc_smem(const Shape& s, int RG)
 
 template <int D, int RG>
 cudaError_t route_tc_t(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt, cudaStream_t st,
-                       const unsigned char* redo, int redo_p)
+                       const unsigned char* redo, int redo_p, int* redo_list)
 {
     const size_t smem = route_tc_smem(s, RG);
     const int Ts = (s.T + 31) / 32 * 32 + 8;
@@ -521,20 +590,22 @@ cudaError_t route_tc_t(const Shape& s, const void* Q, const __nv_bfloat16* plane
     if (e != cudaSuccess) return e;
     const int P = 16 * RG / s.g;
     const long long nblk = (s.n + P - 1) / P;
-    const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
-    if (grid == 0) return cudaSuccess;
-    k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, planes, rt, Ts, redo, redo_p);
-    return cudaGetLastError();
+    return launch_redo(s, P, nblk * s.batch * s.hkv, redo, redo_p, redo_list, st,
+                       [&](unsigned grid, const unsigned char* rd, const int* list) {
+                           k<<<grid, 256, smem, st>>>(s, (const __nv_bfloat16*)Q, planes, rt, Ts, rd, redo_p, list);
+                           return cudaGetLastError();
+                       });
 }
 
 template <int D>
 cudaError_t route_tc_d(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
-                       cudaStream_t st, bool* used, const unsigned char* redo = nullptr, int redo_p = 1)
+                       cudaStream_t st, bool* used, const unsigned char* redo = nullptr, int redo_p = 1,
+                       int* redo_list = nullptr)
 {
     constexpr size_t kLimit = 225 * 1024;
     *used = true;
-    if (32 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, planes, rt, st, redo, redo_p);
-    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, planes, rt, st, redo, redo_p);
+    if (32 >= s.g && route_tc_smem(s, 2) <= kLimit) return route_tc_t<D, 2>(s, Q, planes, rt, st, redo, redo_p, redo_list);
+    if (16 >= s.g && route_tc_smem(s, 1) <= kLimit) return route_tc_t<D, 1>(s, Q, planes, rt, st, redo, redo_p, redo_list);
     *used = false;
     return cudaSuccess;
 }
@@ -707,7 +778,7 @@ static bool long_route_off()
 
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
                                  const __nv_bfloat16* planes, const float* knorm, const Routes& rt,
-                                 unsigned char* redo, int* err, cudaStream_t st)
+                                 unsigned char* redo, int* redo_list, int* err, cudaStream_t st)
 {
     if (planes && route_tcgen05_supported(s, dtype) && !legacy_stage2())
         return launch_route_prefill_tcgen05(s, Q, planes, rt, err, st);
@@ -723,12 +794,13 @@ cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const
     }
     if (dtype == DASH_BF16 && planes) {
         bool used = false;
-        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, planes, rt, st, &used, mask, mask_p)
-                                   : route_tc_d<64>(s, Q, planes, rt, st, &used, mask, mask_p);
+        int* list = mask ? redo_list : nullptr;
+        cudaError_t e = s.d == 128 ? route_tc_d<128>(s, Q, planes, rt, st, &used, mask, mask_p, list)
+                                   : route_tc_d<64>(s, Q, planes, rt, st, &used, mask, mask_p, list);
         if (used) return e;
         // very long rows (T * 16 rows of logits beyond shared memory): CUDA-core variant
-        return s.d == 128 ? route_prefill_t<__nv_bfloat16, 128>(s, Q, kbar, rt, st, mask, mask_p)
-                          : route_prefill_t<__nv_bfloat16, 64>(s, Q, kbar, rt, st, mask, mask_p);
+        return s.d == 128 ? route_prefill_t<__nv_bfloat16, 128>(s, Q, kbar, rt, st, mask, mask_p, list)
+                          : route_prefill_t<__nv_bfloat16, 64>(s, Q, kbar, rt, st, mask, mask_p, list);
     }
     return s.d == 128 ? route_prefill_t<float, 128>(s, Q, kbar, rt, st)
                       : route_prefill_t<float, 64>(s, Q, kbar, rt, st);
