@@ -61,6 +61,8 @@ def load():
         lib.dash_workspace_size.restype = sz
         lib.dash_error_word_offset.argtypes = [P, ctypes.c_int]
         lib.dash_error_word_offset.restype = ctypes.c_longlong
+        lib.dash_prefill_order_offset.argtypes = [P]
+        lib.dash_prefill_order_offset.restype = ctypes.c_longlong
         lib.dash_route_capacity.argtypes = [P]
         lib.dash_route_capacity.restype = ctypes.c_longlong
         lib.dash_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, R, vp, sz, vp]
@@ -140,6 +142,10 @@ def dash_workspace_size(p: dash_params, op: int) -> int:
 
 def dash_error_word_offset(p: dash_params, op: int) -> int:
     return int(load().dash_error_word_offset(ctypes.byref(p), op))
+
+
+def dash_prefill_order_offset(p: dash_params) -> int:
+    return int(load().dash_prefill_order_offset(ctypes.byref(p)))
 
 
 def dash_route_capacity(p: dash_params) -> int:

@@ -194,6 +194,14 @@ long long dash_error_word_offset(const dash_params* p, int op)
     return -1;
 }
 
+long long dash_prefill_order_offset(const dash_params* p)
+{
+    if (check_params(p) != DASH_OK) return -1;
+    const Shape s = make_shape(p);
+    if (!attend_tc_supported(s, p->dtype) || legacy_stage2() || pair_stage2() || !s2_grouping_enabled(s)) return -1;
+    return (long long)prefill_layout(p).perm;
+}
+
 long long dash_route_capacity(const dash_params* p)
 {
     if (check_params(p) != DASH_OK) return 0;

@@ -112,6 +112,7 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         if (lane == 0) {
             tc::prefetch_tmap(&tmK);
             tc::prefetch_tmap(&tmV);
+            const uint64_t pol = tc::l2_evict_first_policy();
             int last[kNSd];
             for (int k = 0; k < kNSd; ++k) last[k] = -1;
             int x = seg_of(j_lo);
@@ -134,10 +135,12 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 }
                 const uint32_t dst = base + slot * kSlotB, fb = bar_full + 8 * slot;
                 tc::mbar_expect_tx(fb, kSlotB);
-                tc::tma_load_4d(dst, &tmK, fb, 0, r, c2, c3);
-                tc::tma_load_4d(dst + kHalf, &tmK, fb, 64, r, c2, c3);
-                tc::tma_load_4d(dst + 2 * kHalf, &tmV, fb, 0, r, c2, c3);
-                tc::tma_load_4d(dst + 3 * kHalf, &tmV, fb, 64, r, c2, c3);
+                // the routed K/V tiles are a stream of several times L2 read once per step: evict
+                // them first, so the chunk summaries that the next step's routing reads stay in L2
+                tc::tma_load_4d_hint(dst, &tmK, fb, 0, r, c2, c3, pol);
+                tc::tma_load_4d_hint(dst + kHalf, &tmK, fb, 64, r, c2, c3, pol);
+                tc::tma_load_4d_hint(dst + 2 * kHalf, &tmV, fb, 0, r, c2, c3, pol);
+                tc::tma_load_4d_hint(dst + 3 * kHalf, &tmV, fb, 64, r, c2, c3, pol);
             }
             if (*abort)   // let copies still in flight land before the block's shared memory goes away
                 for (int k = 0; k < kNSd; ++k)

@@ -172,6 +172,44 @@ def stage2_routed_flops(counts, n, B, g, d, hq):
     return 4.0 * d * (float(counts.sum()) * B * g + counts.shape[0] * hq * diag)
 
 
+def stage2_executed_flops(pf, wl, counts):
+    """FLOPs the tensor-core Stage 2 executes: a tile of 128 query rows (128/g positions, in the
+    order Stage 2 tiled them) walks the union of its positions' routed chunks and diagonal chunks,
+    and every walked unit of keys costs 4 d flops per (row, key) for all 128 rows.  None when
+    the default Stage 2 is not the grouped tensor-core kernel for this shape."""
+    import torch
+    from adaptive_sparse_hierarchical_b200 import _lib as L
+
+    g, B, n, d = wl.h_q // wl.h_kv, wl.chunk, wl.n, wl.d
+    if wl.dtype != "bf16" or d != 128 or B not in (32, 64, 128) or 128 % g:
+        return None
+    off = L.dash_prefill_order_offset(pf.p)
+    P, CPT = 128 // g, (2 if B == 32 else 1)
+    nb = wl.batch * wl.h_kv
+    if off >= 0:
+        order = pf.workspace[off: off + nb * n * 4].view(torch.int32).cpu().numpy().reshape(nb, n)
+    else:
+        order = np.broadcast_to(np.arange(n, dtype=np.int64), (nb, n))
+    idx = pf.chunk_idx.cpu().numpy().reshape(nb, -1)
+    cnt = counts.reshape(nb, n).astype(np.int64)
+    pos = np.arange(n, dtype=np.int64)
+    c = pos // B
+    tri = B * c * (c - 1) // 2 + (pos - c * B) * c
+    units = (n // B + CPT) // CPT + 1
+    total = 0
+    for x in range(nb):
+        inv = np.empty(n, dtype=np.int64)
+        inv[order[x]] = pos
+        tile = inv // P
+        tot = int(cnt[x].sum())
+        rep_pos = np.repeat(pos, cnt[x])
+        start = np.repeat(np.cumsum(cnt[x]) - cnt[x], cnt[x])
+        ent = idx[x][np.repeat(tri, cnt[x]) + (np.arange(tot) - start)].astype(np.int64)
+        keys = np.concatenate([tile[rep_pos] * units + ent // CPT, tile * units + c // CPT])
+        total += np.unique(keys).size
+    return 4.0 * d * 128 * B * CPT * total
+
+
 def prefill_launches(wl):
     """Kernels of this library one prefill step launches: Stage 0, Stage 1, Stage 2, plus the
     position grouping ahead of the tensor-core Stage 2 (g = 8 or 16) and, for rows of more than
@@ -244,6 +282,16 @@ def run_prefill(wl, steps, warmup, ranks, pk, pk_kind, x=None, lite=False):
         "clocks": clk.summary(),
         "gpu_launches": prefill_launches(wl) * steps,
     }
+    try:
+        ex = stage2_executed_flops(pf, wl, counts)
+    except Exception as e:   # a diagnostic: reported, not fatal
+        ex, out["stage2_work_error"] = None, f"{type(e).__name__}: {e}"[:200]
+    if ex:
+        out["stage2_work"] = {"routed_tflop": flops / 1e12, "executed_tflop": ex / 1e12,
+                              "executed_over_routed": ex / flops,
+                              "executed_tflops": ex / t2 / 1e12, "executed_frac": ex / t2 / 1e12 / peak,
+                              "note": "executed: every 128-row tile's union of its positions' routed and "
+                                      "diagonal chunks, all 128 rows, in the order Stage 2 tiled them"}
     if lite:   # sweep mode: the device-timed step and the per-row support only
         c = counts.reshape(-1, wl.n)[:, wl.chunk:].astype("float64")
         vis = (np.arange(wl.n) // wl.chunk)[wl.chunk:].astype("float64")
@@ -709,6 +757,7 @@ def run_sweep(args, ranks, pk, pk_kind, steps=None, decode_steps=None, emit=True
         r = run_prefill(wl, steps, args.warmup, ranks, pk, pk_kind, x=cache[key], lite=True)
         line = {"sweep": name, "metric": "prefill Mtok/s", "value": r["value"], "unit": "Mtok/s",
                 "ms_per_step": r["ms_per_step"], "stages_ms": r["stages_ms"], "routed_fraction": r["routed_fraction"],
+                "stage2_work": r.get("stage2_work"),
                 "stage2_roofline_frac": r["roofline"]["frac"], "stage2_routed_tflops": r["roofline"]["achieved"],
                 "support_fraction_deciles": r["support_fraction_deciles"],
                 "support_chunks_deciles": r["support_chunks_deciles"],
@@ -771,7 +820,7 @@ def main():
             "config": config_of(wl, args), "roofline": pre["roofline"], "e2e": pre["e2e"],
             "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "stages_ms": pre["stages_ms"],
             "routed_fraction": pre["routed_fraction"], "dense_causal": pre["dense_causal"],
-            "stage2_list_vs_bitmask": pre["stage2_list_vs_bitmask"]}
+            "stage2_list_vs_bitmask": pre["stage2_list_vs_bitmask"], "stage2_work": pre.get("stage2_work")}
     if not args.no_decode:
         line["decode"] = run_decode(args.decode_steps, args.warmup, ranks, pk, pk_kind)
         line["gpu_launches"] += line["decode"]["gpu_launches"]

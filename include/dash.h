@@ -104,6 +104,16 @@ size_t dash_workspace_size(const dash_params* p, int op);
  * an op without such a word. */
 long long dash_error_word_offset(const dash_params* p, int op);
 
+/* Byte offset inside the prefill workspace of the order in which the tensor-core Stage 2 (the
+ * DashAttention review's Stage 2 kernel row) tiles the positions: int32 [batch][h_kv][n], entry k of
+ * (b, r) the position in slot k; the tile of 128 query rows numbered t takes the slots
+ * t*128/g .. (t+1)*128/g - 1.  Valid after a prefill's Stage 2 has run on the stream (read it after
+ * the stream has finished).  -1 when the default Stage 2 keeps the positions in sequence order for
+ * these params (no grouping: g other than 8 or 16, another Stage 2 kernel, DASH_CLUSTER=0) or for
+ * invalid params.  A diagnostic: it tells which positions shared a tile, i.e. how much work beyond
+ * the routed pairs a tile executed. */
+long long dash_prefill_order_offset(const dash_params* p);
+
 /* Routing-list entries per (batch, KV head) for prefill: sum over positions of floor(i/B). */
 long long dash_route_capacity(const dash_params* p);
 

@@ -26,7 +26,7 @@ def _p(**kw):
 def test_header_symbols_exported():
     syms = L.header_symbols()
     assert set(syms) == {"dash_workspace_size", "dash_route_capacity", "dash_prefill", "dash_prefill_stage",
-                         "dash_summary_build", "dash_error_word_offset", "dash_decode_noalloc",
+                         "dash_summary_build", "dash_error_word_offset", "dash_decode_noalloc", "dash_prefill_order_offset",
                          "dash_summary_append", "dash_decode", "dash_status_string", "dash_summary_build_paged",
                          "dash_summary_append_paged", "dash_decode_paged", "dash_backward", "dash_set_wait_limit"}
     lib = D.load()
