@@ -363,3 +363,23 @@ def test_bounded_wait_timeout_sets_the_status_word_and_recovers():
     torch.cuda.synchronize()
     assert pf.error_word() == 0
     assert torch.equal(pf.O, O_ref)
+
+
+def test_stage2_position_order_is_a_permutation():
+    """dash_prefill_order_offset: after a prefill with g = 8 the workspace holds the order in which
+    the tensor-core Stage 2 tiled the positions, a permutation of 0..n-1 per (sequence, KV head)
+    (here a workload whose windows take the grouped order), and the bench's executed-work count
+    reads it; g = 2 keeps sequence order (-1)."""
+    from adaptive_sparse_hierarchical_b200 import _lib as L
+    x = inputs.mixture(5, 2, 4096, 16, 2, 128)
+    O, pf = run_prefill(x, chunk=32, alpha=1.5, gamma=1.0)
+    off = L.dash_prefill_order_offset(pf.p)
+    assert off >= 0
+    n = 4096
+    order = pf.workspace[off:off + 2 * 2 * n * 4].view(torch.int32).cpu().numpy().reshape(4, n)
+    for row in order:
+        assert np.array_equal(np.sort(row), np.arange(n))
+    assert any(not np.array_equal(row, np.arange(n)) for row in order)
+    y = inputs.planted(12, 1, 256, 4, 2, 128, 64, dtype="bf16")
+    _, pf2 = run_prefill(y, chunk=64, alpha=1.5, gamma=6.0)
+    assert L.dash_prefill_order_offset(pf2.p) == -1
