@@ -15,8 +15,8 @@
 // copies the entries above (that bound - 1) -- a superset of the only ones the support can
 // reach, tau >= max - 1 -- with their chunk indices into per-thread lists in shared memory; the
 // threshold is solved on the lists, and the head weights, their sums over the g heads of each
-// position and the routed chunks (ascending, with log w) all come from the lists, window by
-// window; the bias is fixed up with the mean once every window is written.  The MMAs of one
+// position and the routed chunks (ascending, with log w) all come from the lists: one warp per
+// position merges the position's 4 g ascending lists; the bias is fixed up with the mean after.  The MMAs of one
 // block overlap the processing of the previous one.  A block whose lists overflow flags its
 // tile in `redo` and writes nothing; the per-shape routing kernels then recompute the flagged
 // tiles.
@@ -52,9 +52,7 @@ constexpr uint32_t kIdescX = tc::idesc_bf16(128, kBW, false, false);
 constexpr int kPlanStop = 0, kPlanGo = 1;
 constexpr int kMaxExtract = 2;
 
-// candidate list entries per (worker warp, lane): a logit (fp32) and its chunk index (16 bits);
-// the emission's head-weight buffer [kR rows][kWin chunks] reuses the plane ring (idle by then)
-constexpr int kWin = 96;
+// candidate list entries per (worker warp, lane): a logit (fp32) and its chunk index (16 bits)
 constexpr int kCap = 52;
 constexpr int kOffIdx = kOffLists + 16 * 32 * kCap * 4;
 constexpr int kOffMisc = kOffIdx + 16 * 32 * kCap * 2;
@@ -65,7 +63,7 @@ constexpr int kMiscBase = (kBarBytes + 15) / 16 * 16;
 constexpr int kMiscBytes = kMiscBase + 16 + 2 * 4 * kR * 16 + 3 * 32 * 4 + kR * 4;
 constexpr size_t kLongSmem = 1024 + kOffMisc + kMiscBytes;
 static_assert(kLongSmem <= 227 * 1024, "shared memory of the long-row routing kernel");
-static_assert(kR * kWin * 4 <= kNS * kStage, "head-weight buffer inside the plane ring");
+static_assert(kR * 4 * 9 <= kNS * kStage, "published list bases, lengths and thresholds inside the plane ring");
 static_assert(kCap % 4 == 0, "lists are padded to a multiple of four entries");
 // |x - x_hi| <= xs (2^-8 |q| |k̄_c|  +  fp32 accumulation error): coefficient of xs |q| max|k̄_c|
 constexpr float kHiPlaneBound = 0.00390625f + 0.0009765625f;
@@ -139,7 +137,6 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
     constexpr int P = kR / G, CAP = kCap;
     float* lists = reinterpret_cast<float*>(sm + kOffLists);            // [16 warps][CAP][32 lanes]
     unsigned short* lidx = reinterpret_cast<unsigned short*>(sm + kOffIdx);   // chunk index of each entry
-    float* wbuf = reinterpret_cast<float*>(sm + kOffRing);              // [kR][kWin] head weights of a window
     char* misc = sm + kOffMisc;
     const uint32_t bar0 = tc::smem_addr(misc);
     const uint32_t q_full = bar0, full0 = bar0 + 8, empty0 = full0 + 8 * kNS;   // ring [kNS] each
@@ -496,66 +493,101 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
             bool stop = false;
             if (!ok) stop = true;
             else if (!over) {
-                // ---- every list holds its column set's whole support: head weights, their sums
-                // over the g heads of each position and the route lists, window by window (kWin
-                // chunks).  Each thread writes its own row's weights of the window into wh (one
-                // row per TMEM lane, zero elsewhere); the position's warp then sums its g rows in
-                // head order: a fixed order, no atomics ---------------------------------------------
-                const int mm = min(m, cap);
-                int cur = 0;
-                const int nwin = (nvmax + kWin - 1) / kWin;
-                for (int wi = 0; wi < nwin; ++wi) {
-                    const int c0 = wi * kWin;
-                    float4* z4 = reinterpret_cast<float4*>(wbuf);
-                    for (int e = tid - 64; e < kR * kWin / 4; e += 512) z4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    workers_sync();
-                    if (active) {
-                        for (; cur < mm; ++cur) {
-                            const int c = ci[cur * 32];
-                            if (c >= c0 + kWin) break;
-                            const float uu = cl[cur * 32] - t;
-                            if (uu > 0.f) wbuf[row * kWin + (c - c0)] = ent_pow(uu, p, mode);
-                        }
-                    }
-                    workers_sync();
-                    // this window's routed chunks of each position in play: warp per position,
-                    // ascending, log w for now (the bias needs the mean over all windows)
-                    for (int pp = warp - 2; pp < P; pp += 16) {
-                        const int ip = i0 + pp;
-                        if (ip >= s.n || (half >= 0 && ((pp * G) >> 6) != half)) continue;
-                        const int nvp = min(ip / s.B, s.T);
-                        const float* Wp = wbuf + pp * G * kWin;
-                        const float inv_g = 1.f / G;
-                        const long long toff = tri_offset(ip, s.B);
-                        uint32_t* mrow = bm ? bm + (long long)ip * rt.words : nullptr;
-                        int basec = pcnt[pp];
-                        float slog = 0.f;
-                        for (int j0 = 0; j0 < kWin; j0 += 32) {
-                            const int c = c0 + j0 + lane;
-                            if (c0 + j0 >= nvp) break;
-                            float a = 0.f;
-#pragma unroll
-                            for (int h = 0; h < G; ++h) a += Wp[h * kWin + j0 + lane];
-                            const float w = c < nvp ? a * inv_g : 0.f;
-                            const bool on = w > 0.f;
-                            const uint32_t msk = __ballot_sync(0xffffffffu, on);
-                            if (on) {
-                                const int kk = basec + __popc(msk & ((1u << lane) - 1u));
-                                const float lw = __logf(w);
-                                idx[toff + kk] = c;
-                                bias[toff + kk] = lw;
-                                slog += lw;
-                            }
-                            if (mrow && lane == 0) mrow[c >> 5] = msk;
-                            basec += __popc(msk);
-                        }
-                        slog = warp_sum(slog);
-                        __syncwarp();
-                        if (lane == 0) { pslog[pp] += slog; pcnt[pp] = basec; }
-                        __syncwarp();
-                    }
-                    workers_sync();   // wbuf is rewritten by the next window
+                // ---- every list holds its column set's whole support: the route lists come from
+                // a merge of each position's 4 g lists (4 column sets x g heads, each ascending in
+                // chunk index).  One warp per position: every step takes the smallest chunk any
+                // list shows (a warp minimum), sums the head weights of the lists that show it in
+                // a fixed butterfly order (deterministic), writes the entry and advances those
+                // lists.  Entries at or below their row's threshold are skipped.  The lists' bases,
+                // lengths and thresholds are published in the (idle) plane ring.
+                float* pub_tau = reinterpret_cast<float*>(sm + kOffRing);   // [kR]
+                int* pub_len = reinterpret_cast<int*>(pub_tau + kR);        // [4][kR]
+                int* pub_off = pub_len + 4 * kR;                            // [4][kR] list base (entries)
+                if (active) {
+                    if (cq == 0) pub_tau[row] = t;
+                    pub_len[cq * kR + row] = min(m, cap);
+                    pub_off[cq * kR + row] = (int)(cl - lists);
                 }
+                workers_sync();
+                for (int pp = warp - 2; pp < P; pp += 16) {
+                    const int ip = i0 + pp;
+                    if (ip >= s.n || (half >= 0 && ((pp * G) >> 6) != half)) continue;
+                    const int nvp = min(ip / s.B, s.T);
+                    constexpr int NL = (4 * G + 31) / 32;   // lists per lane
+                    int lcur[NL] = {}, llen[NL] = {}, loff[NL] = {}, lc[NL] = {};
+                    float ltau[NL] = {}, lx[NL] = {};
+                    auto advance = [&](int j) {
+                        lc[j] = INT_MAX;
+                        while (lcur[j] < llen[j]) {
+                            const int e = loff[j] + 32 * lcur[j]++;
+                            const float x = lists[e];
+                            if (x > ltau[j]) { lc[j] = lidx[e]; lx[j] = x; break; }
+                        }
+                    };
+#pragma unroll
+                    for (int j = 0; j < NL; ++j) {
+                        const int li = lane + 32 * j;        // list li: column set li / G, head li % G
+                        const bool has = li < 4 * G;
+                        const int rr = pp * G + (has ? li % G : 0), cs = has ? li / G : 0;
+                        lcur[j] = 0;
+                        llen[j] = has ? pub_len[cs * kR + rr] : 0;
+                        loff[j] = has ? pub_off[cs * kR + rr] : 0;
+                        ltau[j] = has ? pub_tau[rr] : 0.f;
+                        advance(j);
+                    }
+                    const float inv_g = 1.f / G;
+                    const long long toff = tri_offset(ip, s.B);
+                    uint32_t* mrow = bm ? bm + (long long)ip * rt.words : nullptr;
+                    if (mrow) {
+                        for (int wd = lane; wd < rt.words; wd += 32) mrow[wd] = 0u;
+                        __syncwarp();
+                    }
+                    int kk = 0, wcur = -1;
+                    uint32_t wbits = 0u;
+                    float slog = 0.f;
+                    for (;;) {
+                        int c = lc[0];
+#pragma unroll
+                        for (int j = 1; j < NL; ++j) c = min(c, lc[j]);
+                        const int cmin = __reduce_min_sync(0xffffffffu, c);
+                        if (cmin == INT_MAX || cmin >= nvp) break;
+                        float w = 0.f;
+#pragma unroll
+                        for (int j = 0; j < NL; ++j)
+                            if (lc[j] == cmin) {
+                                w += ent_pow(lx[j] - ltau[j], p, mode);
+                                advance(j);
+                            }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+                        if (!(w > 0.f)) continue;   // weights that underflow route nothing
+                        // the sum of log w for the mean: lane kk % 32 takes entry kk, and the 32
+                        // partial sums are added in a tree at the end (few roundings per term)
+                        const float lw = __logf(w * inv_g);
+                        if (lane == (kk & 31)) slog += lw;
+                        if (lane == 0) {
+                            idx[toff + kk] = cmin;
+                            bias[toff + kk] = lw;
+                            if (mrow) {
+                                if ((cmin >> 5) != wcur) {
+                                    if (wcur >= 0) mrow[wcur] = wbits;
+                                    wcur = cmin >> 5;
+                                    wbits = 0u;
+                                }
+                                wbits |= 1u << (cmin & 31);
+                            }
+                        }
+                        ++kk;
+                    }
+                    slog = warp_sum(slog);
+                    if (lane == 0) {
+                        if (mrow && wcur >= 0) mrow[wcur] = wbits;
+                        pslog[pp] = slog;
+                        pcnt[pp] = kk;
+                    }
+                    __syncwarp();
+                }
+                workers_sync();   // the published lists are read; the ring may be refilled
                 // the ring is written by TMA again only after this pass's decision; order this
                 // thread's generic accesses to it before those asynchronous-proxy writes
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
