@@ -16,10 +16,10 @@
 // reach, tau >= max - 1 -- with their chunk indices into per-thread lists in shared memory; the
 // threshold is solved on the lists, and the head weights, their sums over the g heads of each
 // position and the routed chunks (ascending, with log w) all come from the lists: one warp per
-// position merges the position's 4 g ascending lists; the bias is fixed up with the mean after.  The MMAs of one
-// block overlap the processing of the previous one.  A block whose lists overflow flags its
-// tile in `redo` and writes nothing; the per-shape routing kernels then recompute the flagged
-// tiles.
+// position merges the position's 4 g ascending lists; the bias is fixed up with the mean after.
+// The MMAs of one block overlap the processing of the previous one.  A block whose lists
+// overflow flags its tile in `redo` and writes nothing; the per-shape routing kernels then
+// recompute the flagged tiles.
 // Roles (18 warps): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, warps 2-17 four
 // warps per TMEM lane quarter (32 rows), each reading every fourth 32-column piece of a block.
 // Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
@@ -57,7 +57,7 @@ constexpr int kCap = 52;
 constexpr int kOffIdx = kOffLists + 16 * 32 * kCap * 4;
 constexpr int kOffMisc = kOffIdx + 16 * 32 * kCap * 2;
 // misc: barriers (kBarBytes), tmem slot / abort / overflow / plan (16 B), red [2][4][kR] float4
-// (16 KB), per position: running log-sum, count, list base (3 x 32 words), per row |q| (kR)
+// (16 KB), per position: log-sum and count (2 x 32 words, then 32 spare), per row |q| (kR)
 constexpr int kBarBytes = 8 * (1 + 2 * kNS + 2 + 2 + 2);   // q_full, full/empty ring, x_ready/x_free, drain, dec
 constexpr int kMiscBase = (kBarBytes + 15) / 16 * 16;
 constexpr int kMiscBytes = kMiscBase + 16 + 2 * 4 * kR * 16 + 3 * 32 * 4 + kR * 4;
