@@ -500,12 +500,20 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                 // a fixed butterfly order (deterministic), writes the entry and advances those
                 // lists.  Entries at or below their row's threshold are skipped.  The lists' bases,
                 // lengths and thresholds are published in the (idle) plane ring.
-                float* pub_tau = reinterpret_cast<float*>(sm + kOffRing);   // [kR]
-                int* pub_len = reinterpret_cast<int*>(pub_tau + kR);        // [4][kR]
+                int* pub_len = reinterpret_cast<int*>(sm + kOffRing);      // [4][kR]
                 int* pub_off = pub_len + 4 * kR;                            // [4][kR] list base (entries)
                 if (active) {
-                    if (cq == 0) pub_tau[row] = t;
-                    pub_len[cq * kR + row] = min(m, cap);
+                    // the list in place becomes the support alone, each entry its head weight
+                    const int mm = min(m, cap);
+                    int j = 0;
+                    for (int k = 0; k < mm; ++k) {
+                        const float uu = cl[32 * k] - t;
+                        if (uu > 0.f) {
+                            ci[32 * j] = ci[32 * k];
+                            cl[32 * j++] = ent_pow(uu, p, mode);
+                        }
+                    }
+                    pub_len[cq * kR + row] = j;
                     pub_off[cq * kR + row] = (int)(cl - lists);
                 }
                 workers_sync();
@@ -513,26 +521,30 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                     const int ip = i0 + pp;
                     if (ip >= s.n || (half >= 0 && ((pp * G) >> 6) != half)) continue;
                     const int nvp = min(ip / s.B, s.T);
+                    // lane l holds list l (and l + 32 when 4 g = 64): column set li / G, head li % G.
+                    // A chunk lies in one column set, so the lists showing it are the G lanes
+                    // (li / G) * G .. + G - 1 of one group, summed by a butterfly inside the group.
                     constexpr int NL = (4 * G + 31) / 32;   // lists per lane
+                    constexpr int GW = G < 32 ? G : 32;     // lanes of a group
                     int lcur[NL] = {}, llen[NL] = {}, loff[NL] = {}, lc[NL] = {};
-                    float ltau[NL] = {}, lx[NL] = {};
+                    float lx[NL] = {};
                     auto advance = [&](int j) {
-                        lc[j] = INT_MAX;
-                        while (lcur[j] < llen[j]) {
+                        if (lcur[j] < llen[j]) {
                             const int e = loff[j] + 32 * lcur[j]++;
-                            const float x = lists[e];
-                            if (x > ltau[j]) { lc[j] = lidx[e]; lx[j] = x; break; }
+                            lc[j] = lidx[e];
+                            lx[j] = lists[e];
+                        } else {
+                            lc[j] = INT_MAX;
                         }
                     };
 #pragma unroll
                     for (int j = 0; j < NL; ++j) {
-                        const int li = lane + 32 * j;        // list li: column set li / G, head li % G
+                        const int li = lane + 32 * j;
                         const bool has = li < 4 * G;
                         const int rr = pp * G + (has ? li % G : 0), cs = has ? li / G : 0;
                         lcur[j] = 0;
                         llen[j] = has ? pub_len[cs * kR + rr] : 0;
                         loff[j] = has ? pub_off[cs * kR + rr] : 0;
-                        ltau[j] = has ? pub_tau[rr] : 0.f;
                         advance(j);
                     }
                     const float inv_g = 1.f / G;
@@ -555,11 +567,14 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
 #pragma unroll
                         for (int j = 0; j < NL; ++j)
                             if (lc[j] == cmin) {
-                                w += ent_pow(lx[j] - ltau[j], p, mode);
+                                w += lx[j];
                                 advance(j);
                             }
+                        const uint32_t on = __ballot_sync(0xffffffffu, w != 0.f);
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+                        for (int o = GW / 2; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+                        const int src = on ? ((__ffs(on) - 1) / GW) * GW : 0;
+                        w = __shfl_sync(0xffffffffu, w, src);
                         if (!(w > 0.f)) continue;   // weights that underflow route nothing
                         // the sum of log w for the mean: lane kk % 32 takes entry kk, and the 32
                         // partial sums are added in a tree at the end (few roundings per term)

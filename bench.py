@@ -655,8 +655,8 @@ def decode_kernel_split(st, qn, kn, vn, reset, dev, sm_mhz, nk=20):
     for e in prof.events():
         if e.device_type != torch.autograd.DeviceType.CUDA:
             continue
-        name = e.name.split("(")[0].replace("void ", "").replace("dash::(anonymous namespace)::", "")
-        name = name.replace("dash::<unnamed>::", "")[:60]
+        name = e.name.replace("void ", "").replace("(anonymous namespace)::", "").replace("<unnamed>::", "")
+        name = name.replace("dash::", "").split("(")[0][:60]
         t, n = per.get(name, (0.0, 0))
         per[name] = (t + e.device_time_total, n + 1)
     out = {}
@@ -665,8 +665,12 @@ def decode_kernel_split(st, qn, kn, vn, reset, dev, sm_mhz, nk=20):
         out[name] = {"us_per_step": us, "launches_per_step": n / nk}
         if sm_mhz:
             out[name]["kcycles_per_step"] = us * sm_mhz / 1e3
+    tot = sum(v["us_per_step"] for v in out.values()) or 1.0
+    for v in out.values():
+        v["share"] = v["us_per_step"] / tot
     return {"eager_steps": nk, "per_kernel": out,
-            "note": "eager steps, CUDA profiler kernel records; the graph step overlaps launches"}
+            "note": "eager steps under the CUDA profiler (its instrumentation lengthens them: compare the "
+                    "shares); the timed graph step overlaps the launches"}
 
 
 def paged_decode(wl, st, qn, kn, vn, prefix, nst, reset, stream, bps, pk, pk_kind, ranks):
