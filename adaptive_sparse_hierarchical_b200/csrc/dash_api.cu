@@ -108,7 +108,7 @@ long long route_cap(const dash_params* p)
     return tri_offset(p->seqlen, p->chunk);
 }
 
-struct PrefillLayout { size_t kbar, counts, idx, bias, err, knorm, planes, redo, perm, total; };
+struct PrefillLayout { size_t kbar, counts, idx, bias, err, knorm, planes, redo, perm, spill, total; };
 PrefillLayout prefill_layout(const dash_params* p)
 {
     PrefillLayout L;
@@ -126,7 +126,11 @@ PrefillLayout prefill_layout(const dash_params* p)
     L.perm = L.redo + up(bh * (size_t)p->seqlen);   // one flag per position block at most
     // Stage 2's position order; before Stage 2 rewrites it, Stage 1's list of position blocks to
     // recompute (one count + one int per block at most)
-    L.total = L.perm + up(bh * (size_t)p->seqlen * 4 + 16);
+    L.spill = L.perm + up(bh * (size_t)p->seqlen * 4 + 16);
+    // the long-row Stage 1 kernel's candidate-list spill areas (shapes it can serve)
+    const int g = p->h_kv > 0 ? p->h_q / p->h_kv : 0;
+    const bool long_rows = p->dtype == DASH_BF16 && p->d_h == 128 && T > 512 && (g == 4 || g == 8 || g == 16);
+    L.total = L.spill + (long_rows ? up(route_long_spill_bytes(make_shape(p))) : 0);
     return L;
 }
 
@@ -265,8 +269,9 @@ int dash_prefill_stage(const dash_params* p, int stage, const void* Q, const voi
     }
     if (stage == -1 || stage == DASH_STAGE1) {
         unsigned char* redo = reinterpret_cast<unsigned char*>(ws + L.redo);
+        void* spill = L.total > L.spill ? ws + L.spill : nullptr;
         rc = launch_status(launch_route_prefill(s, p->dtype, Q, kbar, planes, planes ? knorm : nullptr, rt, redo,
-                                                reinterpret_cast<int*>(ws + L.perm), err, st));
+                                                reinterpret_cast<int*>(ws + L.perm), spill, err, st));
         if (rc != DASH_OK) return rc;
     }
     if (stage == -1 || stage == DASH_STAGE2)

@@ -162,9 +162,10 @@ cudaError_t launch_append(const Shape& s, int dtype, const void* k_new, const vo
 // knorm: per (sequence, KV head) the largest Euclidean norm of a summary (written by Stage 0
 // with the planes; the long-row kernel's hi-plane bound)
 // redo_list: scratch of 1 + batch * h_kv * n ints for the list of position blocks to recompute
+// spill: route_long_spill_bytes(s) of scratch for the long-row kernel's candidate lists (or null)
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
                                  const __nv_bfloat16* planes, const float* knorm, const Routes& rt,
-                                 unsigned char* redo, int* redo_list, int* err, cudaStream_t st);
+                                 unsigned char* redo, int* redo_list, void* spill, int* err, cudaStream_t st);
 // tcgen05 / TMEM variant of Stage 1 (bf16, d = 128, at most 512 complete chunks)
 bool route_tcgen05_supported(const Shape& s, int dtype);
 cudaError_t launch_route_prefill_tcgen05(const Shape& s, const void* Q, const __nv_bfloat16* planes, const Routes& rt,
@@ -176,7 +177,10 @@ size_t route_prefill_smem(const Shape& s, int* positions_per_block);
 bool route_long_supported(const Shape& s, int dtype);
 int route_long_positions(const Shape& s);
 cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const float* knorm,
-                                      const Routes& rt, unsigned char* redo, int* err, cudaStream_t st);
+                                      const Routes& rt, unsigned char* redo, int* err, void* spill, cudaStream_t st);
+// per-thread spill entries of the long-row kernel's candidate lists and the bytes of their areas
+int route_long_spill_entries(const Shape& s);
+size_t route_long_spill_bytes(const Shape& s);
 // Stage 2 for prefill.
 // perm: workspace of batch * h_kv * n ints (the tensor-core path's grouped position order)
 cudaError_t launch_attend_prefill(const Shape& s, int dtype, const void* Q, const void* K,

@@ -778,7 +778,7 @@ static bool long_route_off()
 
 cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const float* kbar,
                                  const __nv_bfloat16* planes, const float* knorm, const Routes& rt,
-                                 unsigned char* redo, int* redo_list, int* err, cudaStream_t st)
+                                 unsigned char* redo, int* redo_list, void* spill, int* err, cudaStream_t st)
 {
     if (planes && route_tcgen05_supported(s, dtype) && !legacy_stage2())
         return launch_route_prefill_tcgen05(s, Q, planes, rt, err, st);
@@ -787,7 +787,7 @@ cudaError_t launch_route_prefill(const Shape& s, int dtype, const void* Q, const
     const unsigned char* mask = nullptr;
     int mask_p = 1;
     if (planes && knorm && redo && route_long_supported(s, dtype) && !legacy_stage2() && !long_route_off()) {
-        cudaError_t e = launch_route_prefill_long(s, Q, planes, knorm, rt, redo, err, st);
+        cudaError_t e = launch_route_prefill_long(s, Q, planes, knorm, rt, redo, err, spill, st);
         if (e != cudaSuccess) return e;
         mask = redo;
         mask_p = route_long_positions(s);

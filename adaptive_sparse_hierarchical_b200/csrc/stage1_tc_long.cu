@@ -23,6 +23,7 @@
 // Roles (18 warps): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, warps 2-17 four
 // warps per TMEM lane quarter (32 rows), each reading every fourth 32-column piece of a block.
 // Every mbarrier wait is bounded; on time-out the block records an error code and leaves.
+#include <algorithm>
 #include <climits>
 #include <cudaTypedefs.h>
 
@@ -63,7 +64,9 @@ constexpr int kMiscBase = (kBarBytes + 15) / 16 * 16;
 constexpr int kMiscBytes = kMiscBase + 16 + 2 * 4 * kR * 16 + 3 * 32 * 4 + kR * 4;
 constexpr size_t kLongSmem = 1024 + kOffMisc + kMiscBytes;
 static_assert(kLongSmem <= 227 * 1024, "shared memory of the long-row routing kernel");
-static_assert(kR * 4 * 9 <= kNS * kStage, "published list bases, lengths and thresholds inside the plane ring");
+static_assert(4 * 4 * kR * 4 <= kNS * kStage, "published list lengths, bases, capacities and spill columns inside the plane ring");
+// spill areas in global memory: one per SM id below kSpillAreas (one block per SM)
+constexpr int kSpillAreas = 160;
 static_assert(kCap % 4 == 0, "lists are padded to a multiple of four entries");
 // |x - x_hi| <= xs (2^-8 |q| |k̄_c|  +  fp32 accumulation error): coefficient of xs |q| max|k̄_c|
 constexpr float kHiPlaneBound = 0.00390625f + 0.0009765625f;
@@ -74,14 +77,15 @@ constexpr float kHiPlaneBound = 0.00390625f + 0.0009765625f;
 // tau.  g = f_S^(alpha-1) is convex and decreasing (a p-norm of the [x - t]_+), so Newton steps
 // on g taken from a point left of its root stay left of it: three steps from t0 (where f_S >= 1)
 // give a bound good enough to cut a list; -inf when f_S(t0) < 1 (nothing to gain).
-__device__ __noinline__ float subset_bound(const float* cl, int m, float om0, float om1, float om2, float t0,
-                                           float p, int mode, float am1)
+// Entries past the shared-memory capacity cap sit in the thread's spill slots gv[512 (k - cap)].
+__device__ __noinline__ float subset_bound(const float* cl, int cap, const float* gv, int m, float om0, float om1,
+                                           float om2, float t0, float p, int mode, float am1)
 {
     float t = t0;
     for (int it = 0; it < 3; ++it) {
         float f = 0.f, fd = 0.f;
         for (int k = 0; k < m; ++k) {
-            const float u = cl[32 * k] - t;
+            const float u = (k < cap ? cl[32 * k] : gv[(long long)(k - cap) * 512]) - t;
             if (u > 0.f) { f += ent_pow(u, p, mode); fd += ent_dpow(u, p, mode); }
         }
         const float om[3] = {om0, om1, om2};
@@ -129,7 +133,9 @@ template <int G>
 __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid_constant__ CUtensorMap tmP,
                                                                     const __nv_bfloat16* __restrict__ Q,
                                                                     const float* __restrict__ knorm, Shape s,
-                                                                    Routes rt, unsigned char* redo, int* err)
+                                                                    Routes rt, unsigned char* redo, int* err,
+                                                                    float* spill_v, unsigned short* spill_i,
+                                                                    int spill_cap)
 {
     extern __shared__ char smem_raw[];
     char* sm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -333,6 +339,18 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
         float* cl = lists + own_off;            // this thread's list, entry k at cl[32 k]
         unsigned short* ci = lidx + own_off;    // and its chunk index at ci[32 k]
         int cap = CAP;
+        // entries past the shared-memory capacity spill to this thread's slots of its SM's area in
+        // global memory (one block per SM, so the SM id names the area): entry k >= cap at
+        // gv[512 (k - cap)], up to gcap of them (none when the SM id is past the areas)
+        unsigned smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        const bool spills = spill_v && spill_i && spill_cap > 0 && smid < (unsigned)kSpillAreas;
+        const int gcap = spills ? spill_cap : 0;
+        const long long gbase = spills ? (long long)smid * spill_cap * 512 : 0;
+        float* const gv = spills ? spill_v + gbase + (tid - 64) : nullptr;
+        unsigned short* const gi = spills ? spill_i + gbase + (tid - 64) : nullptr;
+        auto LV = [&](int k) -> float& { return k < cap ? cl[32 * k] : gv[(long long)(k - cap) * 512]; };
+        auto LI = [&](int k) -> unsigned short& { return k < cap ? ci[32 * k] : gi[(long long)(k - cap) * 512]; };
         float mx = -INFINITY, lo = 0.f, t = 0.f;
         float hi = 0.f;
         float om[3] = {-INFINITY, -INFINITY, -INFINITY};   // lower bounds on the other column sets' maxima
@@ -376,19 +394,20 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                             uint32_t mask = 0u;
 #pragma unroll
                             for (int e = 0; e < 16; ++e) mask |= (v[e] > lo_t ? 1u : 0u) << e;
-                            if (m + __popc(mask) > cap && m <= cap) {
+                            if (m + __popc(mask) > cap + gcap && m <= cap + gcap) {
                                 // list full: raise the cut to this thread's subset bound on tau
                                 // (less the margin below) and drop the entries under it
-                                const float tb = subset_bound(cl, m, om[0], om[1], om[2], lo_t, p, mode, s.alpha - 1.f);
+                                const float tb = subset_bound(cl, cap, gv, m, om[0], om[1], om[2], lo_t, p, mode,
+                                                              s.alpha - 1.f);
                                 const float cut = tb - 1e-3f * fmaxf(1.f, fabsf(tb));
                                 if (cut > lo_t) {
                                     lo_t = cut;
                                     int j = 0;
                                     for (int kk = 0; kk < m; ++kk) {
-                                        const float x = cl[32 * kk];
+                                        const float x = LV(kk);
                                         if (x > cut) {
-                                            ci[32 * j] = ci[32 * kk];
-                                            cl[32 * j++] = x;
+                                            LI(j) = LI(kk);
+                                            LV(j++) = x;
                                         }
                                     }
                                     m = j;
@@ -398,12 +417,23 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                                 }
                             }
                             if (mask) {
+                                if (m + __popc(mask) <= cap) {   // the common case: shared memory only
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) {
-                                    const int kk = m + __popc(mask & ((1u << e) - 1u));
-                                    if (((mask >> e) & 1u) && kk < cap) {
-                                        cl[kk * 32] = v[e];
-                                        ci[kk * 32] = (unsigned short)(c0 + e);
+                                    for (int e = 0; e < 16; ++e) {
+                                        const int kk = m + __popc(mask & ((1u << e) - 1u));
+                                        if ((mask >> e) & 1u) {
+                                            cl[kk * 32] = v[e];
+                                            ci[kk * 32] = (unsigned short)(c0 + e);
+                                        }
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e) {
+                                        const int kk = m + __popc(mask & ((1u << e) - 1u));
+                                        if (((mask >> e) & 1u) && kk < cap + gcap) {
+                                            LV(kk) = v[e];
+                                            LI(kk) = (unsigned short)(c0 + e);
+                                        }
                                     }
                                 }
                                 m += __popc(mask);
@@ -436,14 +466,15 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
             // ---- after an extraction pass: threshold on the lists.  A list that overflowed
             // dropped entries, and the root on the entries kept is then a lower bound on tau
             // (a subset's f is smaller everywhere) from which the next extraction starts ----------
-            if (active && m > cap) atomicOr(overflow, 1);
+            if (active && m > cap + gcap) atomicOr(overflow, 1);
             workers_sync();   // also orders the reads of the maxima before the slots are reused
             const bool over = *overflow != 0;
             ++nextract;
             if (ok && active) {
-                const int mm = min(m, cap);
-                const int m4 = (mm + 3) >> 2;
-                for (int kk = mm; kk < 4 * m4; ++kk) cl[kk * 32] = -INFINITY;
+                const int mm = min(m, cap + gcap);   // entries kept: shared memory, then spill slots
+                const int ms = min(mm, cap);
+                const int m4 = (ms + 3) >> 2;
+                for (int kk = ms; kk < 4 * m4; ++kk) cl[kk * 32] = -INFINITY;
                 // every list holds all of its column set's entries above the largest of the
                 // four cuts (each cut is at most tau), so the solve starts there
                 red[(4 + cq) * kR + row].y = lo_t;
@@ -474,6 +505,7 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                     } else {
                         for (int kk = 0; kk < 4 * m4; ++kk) ent_add(S, cl[kk * 32] - t, p, mode);
                     }
+                    for (int kk = cap; kk < mm; ++kk) ent_add(S, gv[(long long)(kk - cap) * 512] - t, p, mode);
                     float4* slot = red + (it & 1) * 4 * kR;
                     slot[cq * kR + row] = make_float4(S.f, S.fd, S.n, S.um);
                     group_sync();
@@ -502,19 +534,33 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                 // lengths and thresholds are published in the (idle) plane ring.
                 int* pub_len = reinterpret_cast<int*>(sm + kOffRing);      // [4][kR]
                 int* pub_off = pub_len + 4 * kR;                            // [4][kR] list base (entries)
+                int* pub_cap = pub_off + 4 * kR;                            // [4][kR] shared-memory entries
+                int* pub_sp = pub_cap + 4 * kR;                             // [4][kR] spill column (tid - 64)
                 if (active) {
                     // the list in place becomes the support alone, each entry its head weight
-                    const int mm = min(m, cap);
+                    const int mm = min(m, cap + gcap);
                     int j = 0;
-                    for (int k = 0; k < mm; ++k) {
-                        const float uu = cl[32 * k] - t;
-                        if (uu > 0.f) {
-                            ci[32 * j] = ci[32 * k];
-                            cl[32 * j++] = ent_pow(uu, p, mode);
+                    if (mm <= cap) {   // the common case: shared memory only
+                        for (int k = 0; k < mm; ++k) {
+                            const float uu = cl[32 * k] - t;
+                            if (uu > 0.f) {
+                                ci[32 * j] = ci[32 * k];
+                                cl[32 * j++] = ent_pow(uu, p, mode);
+                            }
+                        }
+                    } else {
+                        for (int k = 0; k < mm; ++k) {
+                            const float uu = LV(k) - t;
+                            if (uu > 0.f) {
+                                LI(j) = LI(k);
+                                LV(j++) = ent_pow(uu, p, mode);
+                            }
                         }
                     }
                     pub_len[cq * kR + row] = j;
                     pub_off[cq * kR + row] = (int)(cl - lists);
+                    pub_cap[cq * kR + row] = cap;
+                    pub_sp[cq * kR + row] = tid - 64;
                 }
                 workers_sync();
                 for (int pp = warp - 2; pp < P; pp += 16) {
@@ -526,13 +572,20 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                     // (li / G) * G .. + G - 1 of one group, summed by a butterfly inside the group.
                     constexpr int NL = (4 * G + 31) / 32;   // lists per lane
                     constexpr int GW = G < 32 ? G : 32;     // lanes of a group
-                    int lcur[NL] = {}, llen[NL] = {}, loff[NL] = {}, lc[NL] = {};
+                    int lcur[NL] = {}, llen[NL] = {}, loff[NL] = {}, lcap[NL] = {}, lsp[NL] = {}, lc[NL] = {};
                     float lx[NL] = {};
                     auto advance = [&](int j) {
                         if (lcur[j] < llen[j]) {
-                            const int e = loff[j] + 32 * lcur[j]++;
-                            lc[j] = lidx[e];
-                            lx[j] = lists[e];
+                            const int k = lcur[j]++;
+                            if (k < lcap[j]) {
+                                const int e = loff[j] + 32 * k;
+                                lc[j] = lidx[e];
+                                lx[j] = lists[e];
+                            } else {
+                                const long long e = gbase + (long long)(k - lcap[j]) * 512 + lsp[j];
+                                lc[j] = spill_i[e];
+                                lx[j] = spill_v[e];
+                            }
                         } else {
                             lc[j] = INT_MAX;
                         }
@@ -545,6 +598,8 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
                         lcur[j] = 0;
                         llen[j] = has ? pub_len[cs * kR + rr] : 0;
                         loff[j] = has ? pub_off[cs * kR + rr] : 0;
+                        lcap[j] = has ? pub_cap[cs * kR + rr] : 0;
+                        lsp[j] = has ? pub_sp[cs * kR + rr] : 0;
                         advance(j);
                     }
                     const float inv_g = 1.f / G;
@@ -685,7 +740,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_l()
 
 template <int G>
 cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* planes, const float* knorm,
-                          const Routes& rt, unsigned char* redo, int* err, cudaStream_t st)
+                          const Routes& rt, unsigned char* redo, int* err, void* spill, cudaStream_t st)
 {
     auto fn = encode_fn_l();
     if (!fn) return cudaErrorInvalidValue;
@@ -709,7 +764,10 @@ cudaError_t launch_long_g(const Shape& s, const void* Q, const __nv_bfloat16* pl
     const long long nblk = (s.n + P - 1) / P;
     const unsigned grid = (unsigned)(nblk * s.batch * s.hkv);
     if (grid == 0) return cudaSuccess;
-    k<<<grid, 576, smem, st>>>(mp, static_cast<const __nv_bfloat16*>(Q), knorm, s, rt, redo, err);
+    const int sc = spill ? route_long_spill_entries(s) : 0;
+    float* sv = spill ? static_cast<float*>(spill) : nullptr;
+    unsigned short* si = spill ? reinterpret_cast<unsigned short*>(sv + (size_t)kSpillAreas * sc * 512) : nullptr;
+    k<<<grid, 576, smem, st>>>(mp, static_cast<const __nv_bfloat16*>(Q), knorm, s, rt, redo, err, sv, si, sc);
     return cudaGetLastError();
 }
 
@@ -724,13 +782,25 @@ bool route_long_supported(const Shape& s, int dtype)
 
 int route_long_positions(const Shape& s) { return kR / s.g; }
 
+int route_long_spill_entries(const Shape& s)
+{
+    // a thread's column set holds at most ceil(T / 128) pieces of 32 chunks
+    const long long most = (long long)(s.T + 127) / 128 * 32 - kCap;
+    return (int)std::max(0LL, std::min<long long>(most, 460));
+}
+
+size_t route_long_spill_bytes(const Shape& s)
+{
+    return (size_t)kSpillAreas * route_long_spill_entries(s) * 512 * (4 + 2);
+}
+
 cudaError_t launch_route_prefill_long(const Shape& s, const void* Q, const __nv_bfloat16* planes, const float* knorm,
-                                      const Routes& rt, unsigned char* redo, int* err, cudaStream_t st)
+                                      const Routes& rt, unsigned char* redo, int* err, void* spill, cudaStream_t st)
 {
     switch (s.g) {
-    case 4: return launch_long_g<4>(s, Q, planes, knorm, rt, redo, err, st);
-    case 8: return launch_long_g<8>(s, Q, planes, knorm, rt, redo, err, st);
-    default: return launch_long_g<16>(s, Q, planes, knorm, rt, redo, err, st);
+    case 4: return launch_long_g<4>(s, Q, planes, knorm, rt, redo, err, spill, st);
+    case 8: return launch_long_g<8>(s, Q, planes, knorm, rt, redo, err, spill, st);
+    default: return launch_long_g<16>(s, Q, planes, knorm, rt, redo, err, spill, st);
     }
 }
 
