@@ -622,10 +622,6 @@ def run_decode(steps, warmup, ranks, pk, pk_kind, name="decode_128k", paged=True
            "clocks": clk.summary(), "gpu_launches": 4 * (nst - 1),   # append, routing, attend, merge
            "l2": f"KV caches ({2 * wl.batch * wl.n * wl.h_kv * wl.d * 2 / 1e9:.2f} GB) larger than L2"}
     res["us_per_token"] = res["us_per_step"] / wl.batch   # per sequence-token, one GPU
-    try:
-        res["kernels"] = decode_kernel_split(st, qn, kn, vn, reset, dev, res["clocks"].get("sm_mhz"))
-    except Exception as e:   # a diagnostic: reported, not fatal
-        res["kernels"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     if not paged:
         return res
     try:
@@ -634,43 +630,6 @@ def run_decode(steps, warmup, ranks, pk, pk_kind, name="decode_128k", paged=True
     except Exception as e:   # reported, not fatal: the contiguous numbers above stand
         res["paged"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     return res
-
-
-def decode_kernel_split(st, qn, kn, vn, reset, dev, sm_mhz, nk=20):
-    """Device time of each kernel of an eager decode step (append + decode), from the CUDA
-    profiler's kernel records over nk steps, and the same in thousands of SM cycles at the median
-    SM clock sampled during the timed pass: which of append, routing, attend and merge keeps the
-    step from streaming K/V at HBM speed."""
-    import torch
-    from torch.profiler import profile, ProfilerActivity
-
-    reset()
-    torch.cuda.synchronize(dev)
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        for s in range(nk):
-            st.append(kn[s], vn[s])
-            st.decode(qn[s])
-        torch.cuda.synchronize(dev)
-    per = {}
-    for e in prof.events():
-        if e.device_type != torch.autograd.DeviceType.CUDA:
-            continue
-        name = e.name.replace("void ", "").replace("(anonymous namespace)::", "").replace("<unnamed>::", "")
-        name = name.replace("dash::", "").split("(")[0][:60]
-        t, n = per.get(name, (0.0, 0))
-        per[name] = (t + e.device_time_total, n + 1)
-    out = {}
-    for name, (t, n) in sorted(per.items(), key=lambda kv: -kv[1][0]):
-        us = t / nk
-        out[name] = {"us_per_step": us, "launches_per_step": n / nk}
-        if sm_mhz:
-            out[name]["kcycles_per_step"] = us * sm_mhz / 1e3
-    tot = sum(v["us_per_step"] for v in out.values()) or 1.0
-    for v in out.values():
-        v["share"] = v["us_per_step"] / tot
-    return {"eager_steps": nk, "per_kernel": out,
-            "note": "eager steps under the CUDA profiler (its instrumentation lengthens them: compare the "
-                    "shares); the timed graph step overlaps the launches"}
 
 
 def paged_decode(wl, st, qn, kn, vn, prefix, nst, reset, stream, bps, pk, pk_kind, ranks):
