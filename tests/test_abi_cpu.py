@@ -153,3 +153,14 @@ def test_wait_limit_knob_round_trips():
     assert prev == 1 << 23
     assert L.dash_set_wait_limit(-1) == -1
     assert L.dash_set_wait_limit(prev) == 5
+
+
+def test_prefill_order_offset_rejects_invalid_params():
+    """The diagnostic offset of Stage 2's position order: -1 for invalid params and for shapes whose
+    tensor-core Stage 2 keeps sequence order (g = 2); otherwise it lies inside the workspace."""
+    assert L.dash_prefill_order_offset(_p(h_q=6, h_kv=4)) == -1
+    assert L.dash_prefill_order_offset(_p(alpha=1.0)) == -1
+    assert L.dash_prefill_order_offset(_p(h_q=4, h_kv=2)) == -1
+    p = _p()
+    off = L.dash_prefill_order_offset(p)
+    assert off == -1 or 0 <= off < L.dash_workspace_size(p, L.DASH_OP_PREFILL)
