@@ -61,13 +61,14 @@ dec_attend_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();   // the routes of this step
     pdl_launch_dependents();
+    // tile counts of the (sequence, KV head) pairs: one load per thread, all in flight at once
+    // (blockDim >= kMaxBR >= BR), then their prefix in shared memory
+    static_assert(32 * (1 + kCons) >= kMaxBR, "one thread per pair");
+    if (threadIdx.x < BR) pre[threadIdx.x + 1] = (rt.counts[threadIdx.x] + 1) * NH;
+    __syncthreads();
     if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int x = 0; x < BR; ++x) {
-            pre[x] = acc;
-            acc += (rt.counts[x] + 1) * NH;
-        }
-        pre[BR] = acc;
+        pre[0] = 0;
+        for (int x = 1; x <= BR; ++x) pre[x] += pre[x - 1];
         for (int k = 0; k < kNSd; ++k) { tc::mbar_init(bar_full + 8 * k, 1); tc::mbar_init(bar_empty + 8 * k, 1); }
         *abort = 0;
         tc::mbar_fence_init();
@@ -330,12 +331,25 @@ __global__ void __launch_bounds__(D) dec_merge_kernel(Shape s, const float* __re
     pdl_wait();   // the partials of this step
     const int x = blockIdx.x / s.g, row = blockIdx.x % s.g, G = s.g, NH = s.B / 64;
     const int b = x / s.hkv, r = x % s.hkv, col = threadIdx.x;
-    long long lo = 0, total = 0;
-    for (int y = 0; y < s.batch * s.hkv; ++y) {
+    // tiles before this pair and in all: the pairs' counts loaded by the block's threads at once,
+    // summed by warp shuffles, then over the warps in order
+    __shared__ long long wsum_lo[D / 32], wsum_tot[D / 32];
+    long long lo_p = 0, tot_p = 0;
+    for (int y = threadIdx.x; y < s.batch * s.hkv; y += D) {
         const long long c = (long long)(rt.counts[y] + 1) * NH;
-        if (y < x) lo += c;
-        total += c;
+        if (y < x) lo_p += c;
+        tot_p += c;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo_p += __shfl_xor_sync(0xffffffffu, lo_p, o);
+        tot_p += __shfl_xor_sync(0xffffffffu, tot_p, o);
+    }
+    if ((threadIdx.x & 31) == 0) { wsum_lo[threadIdx.x >> 5] = lo_p; wsum_tot[threadIdx.x >> 5] = tot_p; }
+    __syncthreads();
+    long long lo = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) { lo += wsum_lo[w]; total += wsum_tot[w]; }
     const long long hi = lo + (long long)(rt.counts[x] + 1) * NH;
     // block c covers tiles [total c / n, total (c+1) / n); it wrote a partial for this pair iff
     // that range is nonempty and meets [lo, hi)
