@@ -341,7 +341,9 @@ __global__ void __launch_bounds__(576, 1) route_prefill_long_kernel(const __grid
         int cap = CAP;
         // entries past the shared-memory capacity spill to this thread's slots of its SM's area in
         // global memory (one block per SM, so the SM id names the area): entry k >= cap at
-        // gv[512 (k - cap)], up to gcap of them (none when the SM id is past the areas)
+        // gv[512 (k - cap)], up to gcap of them (none when the SM id is past the areas).  This
+        // relies on a block staying on its SM; a block resumed elsewhere after compute
+        // preemption could share an area (claiming areas atomically per block would lift that).
         unsigned smid;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
         const bool spills = spill_v && spill_i && spill_cap > 0 && smid < (unsigned)kSpillAreas;
